@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Benchmark of the GLM-5.2 MoE feed-forward layer forward pass on B200.
+
+One step = one moe_forward call over one batch (router logits, routing,
+grouping, row gather, gate/up GEMM with the SiLU gate, down GEMM, merge) on
+inputs already resident in HBM; the L2 cache is flushed (256 MiB memset)
+before every timed step, outside the step's events.  Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode]
+  python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Multi-GPU (torchrun, one process per GPU): every rank runs an independent
+replica on its own batch (the layer shards over tokens with no exchange), so
+scaling is weak; the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from datetime import timedelta
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec on 1 B200 and % of roofline (HBM or bf16 tensor peak)"
+FLUSH_BYTES = 256 << 20
+STAGES = ["router_logits", "route", "permute", "gather", "gateup_gemm", "down_gemm", "combine"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# accounting
+# ---------------------------------------------------------------------------
+def layer_bytes_flops(cfg, U: int):
+    """Algorithmic bytes and flops of one layer pass (touched experts only)."""
+    T, D, E, F, k, S, Fs = cfg.T, cfg.D, cfg.E, cfg.F, cfg.k, cfg.S, cfg.Fs
+    B = (U * 3 * D * F * 2 + S * 3 * D * Fs * 2 + E * D * 4 + E * 4 + T * D * 2 * 2 + T * k * 8)
+    FL = 2 * T * D * E + 6 * D * F * T * k + 6 * D * Fs * T * S
+    return B, FL
+
+
+def gateup_bytes(cfg, U: int):
+    """Algorithmic bytes of one gate/up GEMM launch: the W1 and W3 rows of the
+    touched routed experts and of the shared experts, the gathered input rows
+    and the bf16 activations written."""
+    T, D, F, k, S, Fs = cfg.T, cfg.D, cfg.F, cfg.k, cfg.S, cfg.Fs
+    return U * 2 * F * D * 2 + S * 2 * Fs * D * 2 + (T * k + S * T) * D * 2 + (T * k * F + S * T * Fs) * 2
+
+
+def gateup_flops(cfg):
+    return 4 * cfg.D * (cfg.F * cfg.T * cfg.k + cfg.Fs * cfg.T * cfg.S)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def stored_traffic(kernel_key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel_key)
+    if not rec:
+        return None
+    import hashlib
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != rec["source_sha256_16"]:
+            return None
+    return rec["dram_bytes_per_launch"]
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            gid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        mhz, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1].split()[0]))
+                maxs.append(float(parts[2].split()[0]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxs),
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (test infrastructure; the product path never imports it)
+# ---------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample_runner(cfg, h_rows: np.ndarray, Wr: np.ndarray, bias: np.ndarray, expert_fn,
+                         shared):
+    from oracle import moe_oracle as orc
+
+    def run():
+        return orc.moe_layer_tokens(h_rows, Wr, bias, cfg.k, cfg.scale, expert_fn, shared)
+    return run
+
+
+def time_oracle(run, n_tokens: int, min_s: float, max_s: float):
+    run()  # untimed: fills the host copies of the touched experts
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        run()
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_s or el >= max_s:
+            break
+    return n_tokens * reps / el, reps, el
+
+
+def cpu_baseline_from_device(cfg, inp, n_tokens: int):
+    h = inp["h"][:n_tokens].float().cpu().numpy()
+    Wr = inp["Wr"].cpu().numpy()
+    bias = inp["bias"].cpu().numpy()
+    cache = {}
+
+    def expert(e):
+        if e not in cache:
+            cache[e] = tuple(x[e].cpu().double().numpy() for x in (inp["W1"], inp["W3"], inp["W2"]))
+        return cache[e]
+    shared = [tuple(x[s].cpu().double().numpy() for x in (inp["Ws1"], inp["Ws3"], inp["Ws2"]))
+              for s in range(cfg.S)]
+    run = oracle_sample_runner(cfg, h, Wr, bias, expert, shared)
+    tps, reps, el = time_oracle(run, n_tokens, 10.0, 30.0)
+    return {"value": tps, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"first {n_tokens} tokens of the {cfg.name} batch, whole layer in numpy "
+                      f"(fp32 routing, fp64 experts), {reps} passes in {el:.1f} s; touched "
+                      f"expert weights pre-copied to the host"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import sparse_moe_layer_04_b200 as moe
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = mi.CONFIGS[args.config]
+    inp = mi.layer_weights(cfg, 0, device=dev)
+    inp["h"] = mi.hidden(cfg, seed=rank, device=dev)
+    d = moe.dims_of(cfg)
+    ws = moe.alloc_workspace(d, dev)
+    out = torch.empty((cfg.T, cfg.D), dtype=torch.bfloat16, device=dev)
+    idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
+    wgt = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        moe.moe_forward(inp["h"], inp["Wr"], inp["bias"], inp["W1"], inp["W3"], inp["W2"],
+                        inp["Ws1"], inp["Ws3"], inp["Ws2"], d, out, ws, idx, wgt)
+
+    sampler = ClockSampler(local_rank)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if moe.moe_get_device_status(ws) != 0:
+        raise RuntimeError("device status error during warm-up: " + moe.moe_last_error())
+    launches_per_step = moe.moe_last_launch_count()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_PROFILE_EVENTS)]
+          for _ in range(K)]
+    for evs in ev:  # create the CUDA events before the timed region
+        for e in evs:
+            e.record()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        moe.moe_set_profile_events(ev[i])
+        step()
+    moe.moe_set_profile_events(None)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if moe.moe_get_device_status(ws) != 0:
+        raise RuntimeError("device status error in the timed region: " + moe.moe_last_error())
+
+    step_ms = [ev[i][0].elapsed_time(ev[i][7]) for i in range(K)]
+    stage_ms = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K))
+                for j, name in enumerate(STAGES)}
+    ms = statistics.mean(step_ms)
+    gateup_ms = stage_ms["gateup_gemm"]
+    if world > 1:
+        t = torch.tensor([ms, gateup_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, gateup_ms = t.tolist()
+
+    counts = torch.bincount(idx.flatten().long(), minlength=cfg.E)
+    U = int((counts > 0).sum().item())
+
+    # end to end: pinned host input -> device -> layer -> pinned host output, per step
+    h_pin = inp["h"].cpu().pin_memory()
+    out_pin = torch.empty((cfg.T, cfg.D), dtype=torch.bfloat16).pin_memory()
+    h_dev = torch.empty_like(inp["h"])
+    e2e_steps = min(K, 200)
+    e2e_ms = []
+    for i in range(e2e_steps + 3):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        h_dev.copy_(h_pin, non_blocking=True)
+        moe.moe_forward(h_dev, inp["Wr"], inp["bias"], inp["W1"], inp["W3"], inp["W2"],
+                        inp["Ws1"], inp["Ws3"], inp["Ws2"], d, out, ws)
+        out_pin.copy_(out, non_blocking=True)
+        b.record()
+        b.synchronize()
+        if i >= 3:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e = statistics.mean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e = t.item()
+
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    bf16 = float(peaks["bf16_tflops"])
+    B, FL = layer_bytes_flops(cfg, U)
+    t_s = ms / 1e3
+    t_roof_hbm = B / (hbm * 1e9)
+    t_roof_tc = FL / (bf16 * 1e12)
+    gu_bytes = gateup_bytes(cfg, U)
+    gu_flops = gateup_flops(cfg)
+    gu_gbs = gu_bytes / (gateup_ms / 1e3) / 1e9
+    gu_tfs = gu_flops / (gateup_ms / 1e3) / 1e12
+    gu_bound = "hbm" if gu_bytes / (hbm * 1e9) >= gu_flops / (bf16 * 1e12) else "tensor"
+    if gu_bound == "hbm":
+        roof = {"bound": "hbm", "achieved": gu_gbs, "peak": hbm, "unit": "GB/s",
+                "frac": gu_gbs / hbm}
+    else:
+        roof = {"bound": "tensor", "achieved": gu_tfs, "peak": bf16, "unit": "TFLOP/s",
+                "frac": gu_tfs / bf16}
+    roof.update({"traffic": stored_traffic(f"grouped_gemm_gateup/{cfg.name}"),
+                 "kernel": "grouped_gemm_kernel<gate/up>", "ms": gateup_ms,
+                 "algorithmic_bytes": gu_bytes, "algorithmic_flops": gu_flops,
+                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured"
+                 else "fallback (profiling recipe)"})
+
+    res = {
+        "metric": METRIC,
+        "value": world * cfg.T / t_s,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded counter-based generator; random-init weights of the layer's shapes)",
+        "config": {"workload": f"{cfg.name}: GLM-5.2-shaped MoE layer T={cfg.T} D={cfg.D} "
+                               f"E={cfg.E} k={cfg.k} F={cfg.F} S={cfg.S} Fs={cfg.Fs} "
+                               f"scale={cfg.scale}" if cfg.weight_family != "glm45air" else
+                               f"{cfg.name}: GLM-4.5-Air-shaped MoE layer T={cfg.T} D={cfg.D} "
+                               f"E={cfg.E} k={cfg.k} F={cfg.F} S={cfg.S} Fs={cfg.Fs} "
+                               f"scale={cfg.scale}",
+                   "T": cfg.T, "touched_experts": U, "global_batch": world * cfg.T,
+                   "parallelism": f"replicas x{world} (token-parallel, no exchange)",
+                   "l2": "flushed: 256 MiB memset before every timed step, outside its events",
+                   "ms_p10_p90": [float(np.percentile(step_ms, 10)), float(np.percentile(step_ms, 90))],
+                   "stage_ms": stage_ms},
+        "roofline": roof,
+        "layer_roofline": {
+            "bytes": B, "flops": FL, "t_roof_ms": max(t_roof_hbm, t_roof_tc) * 1e3,
+            "binding": "hbm" if t_roof_hbm >= t_roof_tc else "tensor",
+            "frac": max(t_roof_hbm, t_roof_tc) / t_s,
+            "hbm_frac": t_roof_hbm / t_s, "tensor_frac": t_roof_tc / t_s,
+            "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "source": peak_src}},
+        "e2e": {"value": world * cfg.T / (e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": cfg.T * cfg.D * 2, "d2h_bytes_per_step": cfg.T * cfg.D * 2,
+                "ms_per_step": e2e},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_from_device(cfg, inp, min(cfg.T, args.cpu_tokens))
+    return res
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle, as it stands, on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    from oracle import moe_oracle as orc
+
+    cfg = mi.CONFIGS[args.config]
+    n = min(cfg.T, args.cpu_tokens)
+    h = mi.hidden(cfg, 0).float().numpy()[:n]
+    Wr = mi.router_weight(cfg, 0).numpy()
+    bias = mi.correction_bias(cfg, 0).numpy()
+    cache = {}
+
+    def expert(e):
+        if e not in cache:
+            cache[e] = tuple(x.double().numpy() for x in mi.expert_weights(cfg, e, 0))
+        return cache[e]
+    shared = [tuple(x.double().numpy() for x in mi.expert_weights(cfg, s, 0, shared=True))
+              for s in range(cfg.S)]
+
+    def step():
+        return orc.moe_layer_tokens(h, Wr, bias, cfg.k, cfg.scale, expert, shared)
+
+    step()  # untimed: generates the touched experts' weights
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t0)
+    ms = statistics.mean(times) * 1e3
+    value = n / (ms / 1e3)
+    cores = _blas_threads()
+    sample = (f"first {n} tokens of the {cfg.name} batch per step, whole layer in numpy "
+              f"(fp32 routing, fp64 experts); touched experts generated before timing")
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded counter-based generator)",
+        "config": {"workload": f"{cfg.name}: T={cfg.T} D={cfg.D} E={cfg.E} k={cfg.k} F={cfg.F} "
+                               f"S={cfg.S} Fs={cfg.Fs} scale={cfg.scale}", "T": cfg.T,
+                   "sample_tokens": n},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="decode", choices=sorted(mi.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=128,
+                    help="tokens of the batch the CPU oracle processes per pass")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,184 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) GLM-5.2 Mixture-of-Experts
+ * feed-forward layer forward pass.
+ *
+ * The layer ("Model anatomy -- GLM-5.2", frontier-model-atlas, Decoder
+ * microscope, Feed-forward / Mixture of Experts panel): E routed experts of
+ * which k are active per token, one (in general S) always-on shared expert,
+ * learned routing with sigmoid router scores; an expert-score correction bias
+ * takes part in the top-k selection only; the selected scores without the
+ * bias are renormalised and multiplied by the routed scaling factor (2.5 for
+ * GLM-5.2, 1.0 for GLM-4.5-Air per "GLM-4.5 Full Forward", How it works); the
+ * weighted expert outputs are merged with the shared expert's output.
+ * Sizes ("GLM-5.2", PocketLLM, Model specification): hidden 6144, 256 routed
+ * experts, top-8, expert width 2048, 1 shared expert.  Expert weights are
+ * named w1/w3 (input projections) and w2 (output projection) ("GLM-5.2",
+ * PocketLLM, Implemented execution path); each expert is read as the gated
+ * MLP y = w2 (silu(w1 x) * (w3 x)).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument is a DEVICE pointer unless stated otherwise; the
+ *    caller allocates and owns every buffer and the stream.  The library never
+ *    allocates device memory: all scratch lives in the caller's workspace.
+ *  - Arrays are dense and row-major.  Device pointers must be 16-byte aligned.
+ *  - bf16 means IEEE bfloat16 stored as uint16_t bit patterns.
+ *  - Calls only enqueue work on `stream` and return at once; results are
+ *    ready when the stream reaches them.
+ *  - Return value: MOE_OK (0), or a negative moe_status_t when the host-side
+ *    checks reject the arguments or a launch fails.  On a negative return
+ *    nothing was enqueued by the failing step (earlier steps of a composite
+ *    call may have been); moe_last_error() gives a message.
+ *  - Conditions only the device can see (a non-finite logit, an expert index
+ *    out of range, a repeated expert within a token, inconsistent group
+ *    offsets, a bounded wait that ran out) raise bits of a status word kept at
+ *    the start of the workspace; moe_get_device_status() reads and clears it.
+ *    The caller zeroes the workspace once after allocating it (the library
+ *    only ever ORs bits into the word).  Kernels never trap; after such an
+ *    error the outputs are unspecified.
+ *  - Limits: 1 <= E <= 1024, 1 <= k <= min(E, 32), 0 <= S <= 16,
+ *    T >= 0 (T = 0 enqueues nothing), D, F and Fs positive multiples of 8,
+ *    scale finite, T * k < 2^31, and every buffer smaller than 2^31 rows.
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI-compatible with cudaStream_t (a pointer to the opaque CUstream_st). */
+struct CUstream_st;
+typedef struct CUstream_st* moe_stream_t;
+
+/* Layer dimensions. */
+typedef struct moe_dims {
+  int32_t T;     /* tokens in the batch                                      */
+  int32_t D;     /* hidden size                                              */
+  int32_t E;     /* routed experts                                           */
+  int32_t F;     /* routed expert width (intermediate size)                  */
+  int32_t k;     /* experts selected per token                               */
+  int32_t S;     /* shared (always-on) experts, 0 allowed                    */
+  int32_t Fs;    /* shared expert width                                      */
+  float scale;   /* routed scaling factor                                    */
+} moe_dims_t;
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,  /* bad dimension, null or misaligned pointer    */
+  MOE_ERR_UNSUPPORTED = -2,  /* no sm_100 device / shape outside the limits  */
+  MOE_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed         */
+  MOE_ERR_WORKSPACE = -4,    /* workspace missing or smaller than required   */
+  MOE_ERR_NONFINITE = -5,    /* device: a router logit was NaN or infinite   */
+  MOE_ERR_TIMEOUT = -6,      /* device: a bounded wait gave up               */
+  MOE_ERR_BOUNDS = -7        /* device: index/offset out of range or repeated */
+} moe_status_t;
+
+/* Bytes of workspace that moe_forward needs for `dims` (a superset of what
+ * every other entry point needs).  The workspace must be 256-byte aligned.
+ * Returns 0 if the dimensions are invalid. */
+size_t moe_workspace_size(const moe_dims_t* dims);
+
+/* Router logits ("Routing: learned", MoE panel; fp32 router):
+ *   logits[t, e] = sum_d h[t, d] * Wr[e, d]
+ * h [T, D] bf16, Wr [E, D] fp32, logits [T, E] fp32 (output).  fp32 FMA
+ * arithmetic; the summation order over d is fixed, so repeated calls give
+ * identical bits.  `ws` (>= moe_workspace_size bytes) holds split-K partial
+ * sums. */
+int moe_router_logits(const void* h, const float* Wr, const moe_dims_t* dims, float* logits,
+                      void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Routing (MoE panel: sigmoid scores, bias for selection only, un-biased
+ * renormalised scores times the routed scale), one warp per token:
+ *   s[e]   = fp32(1 / (1 + exp(-(double)logits[t, e])))
+ *   key[e] = s[e] + bias[e]                                   (fp32 add)
+ *   idx[t, 0..k-1] = the k experts first under (key descending, index
+ *                    ascending), in that order
+ *   sum    = s[idx0] + s[idx1] + ... (fp32, slot order)
+ *   w[t, j] = (s[idx_j] / sum) * scale                        (fp32 ops)
+ * logits [T, E] fp32, bias [E] fp32 -> idx [T, k] int32, w [T, k] fp32.
+ * A non-finite logit raises MOE_ERR_NONFINITE in the status word of `ws`
+ * (ws may be NULL: then no status is kept). */
+int moe_route(const float* logits, const float* bias, const moe_dims_t* dims, int32_t* idx,
+              float* w, void* ws, moe_stream_t stream);
+
+/* Grouping of the (token, slot) pairs by expert (counting sort; the pages
+ * call the expert kernels "grouped"):
+ *   counts[e]  = number of pairs routed to expert e            [E] int32
+ *   offsets[e] = counts[0] + ... + counts[e-1]                 [E+1] int32
+ *   perm[r]    = token of grouped row r; rows offsets[e] .. offsets[e+1]-1
+ *                hold expert e's tokens in increasing (token, slot) order
+ *                                                              [T*k] int32
+ *   inv[t, j]  = grouped row of pair (t, j)                    [T, k] int32
+ * idx [T, k] int32 must hold k distinct experts in [0, E) per row; a value
+ * out of range or repeated raises MOE_ERR_BOUNDS.  Integer results are
+ * exact and deterministic. */
+int moe_permute(const int32_t* idx, const moe_dims_t* dims, int32_t* counts, int32_t* offsets,
+                int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Expert MLPs on grouped rows (gated MLP with w1/w3 -> SiLU gate -> w2):
+ *   routed row r (expert e, offsets[e] <= r < offsets[e+1], token perm[r]):
+ *     y[r] = W2[e] (silu(W1[e] h[perm[r]]) * (W3[e] h[perm[r]]))
+ *   shared row T*k + s*T + t:
+ *     y[T*k + s*T + t] = Ws2[s] (silu(Ws1[s] h[t]) * (Ws3[s] h[t]))
+ * h [T, D] bf16; perm [T*k], offsets [E+1] int32 as moe_permute writes them;
+ * W1, W3 [E, F, D], W2 [E, D, F], Ws1, Ws3 [S, Fs, D], Ws2 [S, D, Fs] bf16
+ * (nn.Linear layout: out-features x in-features).  y [T*k + S*T, D] fp32
+ * (output).  bf16 tensor-core products with fp32 accumulation; the gated
+ * activation is rounded to bf16 before the w2 product.  Ws* may be NULL when
+ * S = 0. */
+int moe_expert_ffn(const void* h, const int32_t* perm, const int32_t* offsets, const void* W1,
+                   const void* W3, const void* W2, const void* Ws1, const void* Ws3,
+                   const void* Ws2, const moe_dims_t* dims, float* y, void* ws, size_t ws_bytes,
+                   moe_stream_t stream);
+
+/* Merge (MoE panel: weighted expert outputs merged with the always-on shared
+ * expert; "Expert fan-out 8 + 1"), deterministic fixed order:
+ *   out[t] = bf16( sum_s y[T*k + s*T + t] + sum_j w[t, j] * y[inv[t, j]] )
+ * y [T*k + S*T, D] fp32, w [T, k] fp32, inv [T, k] int32 -> out [T, D] bf16.
+ * An inv entry outside [0, T*k) raises MOE_ERR_BOUNDS (ws may be NULL). */
+int moe_combine(const float* y, const float* w, const int32_t* inv, const moe_dims_t* dims,
+                void* out, void* ws, moe_stream_t stream);
+
+/* The whole layer: moe_router_logits, moe_route, moe_permute, the row
+ * gather, moe_expert_ffn and moe_combine in one call on one stream, with no
+ * host synchronisation (capturable in a CUDA graph).
+ * h [T, D] bf16; Wr [E, D] fp32; bias [E] fp32; weights as in
+ * moe_expert_ffn; out [T, D] bf16.  idx_out [T, k] int32 and w_out [T, k]
+ * fp32 are optional (NULL: kept in the workspace).  ws_bytes must be at
+ * least moe_workspace_size(dims). */
+int moe_forward(const void* h, const float* Wr, const float* bias, const void* W1,
+                const void* W3, const void* W2, const void* Ws1, const void* Ws3,
+                const void* Ws2, const moe_dims_t* dims, void* out, int32_t* idx_out,
+                float* w_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, returns the first error recorded in the status word
+ * of `ws` (MOE_OK if none) and clears the word. */
+int moe_get_device_status(void* ws, moe_stream_t stream);
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char* moe_last_error(void);
+
+/* Number of kernels the last successful call on this host thread enqueued. */
+int moe_last_launch_count(void);
+
+/* Stage timing of moe_forward (host-thread local).  `events` points to n
+ * cudaEvent_t handles created by the caller; while set, every moe_forward
+ * call on this thread records them on its stream at the stage boundaries:
+ *   events[0] before the router, [1] after the router logits, [2] after the
+ *   routing, [3] after the grouping, [4] after the row gather, [5] after the
+ *   gate/up GEMM, [6] after the down GEMM, [7] after the merge.
+ * n must be MOE_PROFILE_EVENTS (8) to enable, or 0 (events may be NULL) to
+ * disable.  The library keeps the pointer, not a copy: the array must stay
+ * valid while enabled. */
+#define MOE_PROFILE_EVENTS 8
+int moe_set_profile_events(void* const* events, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H_ */

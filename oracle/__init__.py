@@ -31,6 +31,7 @@ from .moe_oracle import (  # noqa: F401
     select_topk,
     routing_weights,
     route,
+    routing_alternatives,
     swiglu_expert,
     group_by_expert,
     combine,

@@ -109,6 +109,38 @@ def route(logits: np.ndarray, bias: np.ndarray, k: int, scale: float
     return idx, routing_weights(s, idx, scale)
 
 
+def routing_alternatives(logits_row: np.ndarray, bias: np.ndarray, k: int, scale: float,
+                         delta: float):
+    """Every routing of one token that is correct up to a logit perturbation.
+
+    Two implementations of the fp32 router sum the hidden dimension in
+    different orders, so their logits (and hence keys) may differ in the last
+    bits.  When the k-th and (k+1)-th selection keys lie within `delta` of
+    each other, either choice is a correct top-k.  Returns a list of
+    (idx [k] int32, w [k] fp32) candidates: the strict selection first, then
+    every other choice of the boundary experts among those whose key lies
+    within `delta` of the k-th key (at most 64 candidates).
+    """
+    s = sigmoid_scores(np.asarray(logits_row, F32)[None, :])
+    keys = selection_keys(s, bias)[0]
+    order = select_topk(keys[None, :], keys.shape[0])[0]
+    kth = float(keys[order[k - 1]])
+    near = [int(e) for e in order if abs(float(keys[e]) - kth) <= delta]
+    sure = [int(e) for e in order[:k] if int(e) not in near]
+    need = k - len(sure)
+    cands = []
+    from itertools import combinations
+    for pick in combinations(near, need):
+        chosen = set(sure) | set(pick)
+        idx = np.array([int(e) for e in order if int(e) in chosen], np.int32)[None, :]
+        cands.append((idx[0], routing_weights(s, idx, scale)[0]))
+        if len(cands) >= 64:
+            break
+    strict = order[:k].astype(np.int32)
+    cands.sort(key=lambda c: 0 if np.array_equal(c[0], strict) else 1)
+    return cands
+
+
 # ----------------------------------------------------------------------------
 # experts
 # ----------------------------------------------------------------------------

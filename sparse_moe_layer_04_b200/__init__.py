@@ -1,0 +1,210 @@
+"""Python binding of libmoe_b200.so, the B200 (sm_100a) GLM-5.2 MoE-layer forward.
+
+Argument marshalling only: every function here checks dtypes, shapes and
+devices of torch tensors, passes their device pointers and the current CUDA
+stream to the C ABI of the same name (``include/moe_b200.h``) and raises on a
+non-zero return code.  Every step of the layer runs in the library's CUDA
+kernels; there is no fallback.  If the library is missing the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED = -2
+MOE_ERR_CUDA = -3
+MOE_ERR_WORKSPACE = -4
+MOE_ERR_NONFINITE = -5
+MOE_ERR_TIMEOUT = -6
+MOE_ERR_BOUNDS = -7
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+class moe_dims_t(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("D", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("F", ctypes.c_int32), ("k", ctypes.c_int32), ("S", ctypes.c_int32),
+                ("Fs", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+    def __repr__(self):
+        return ("moe_dims_t(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_)
+                + ")")
+
+
+def dims(T: int, D: int, E: int, F: int, k: int, S: int = 1, Fs: Optional[int] = None,
+         scale: float = 2.5) -> moe_dims_t:
+    return moe_dims_t(T, D, E, F, k, S, F if Fs is None else Fs, scale)
+
+
+def dims_of(cfg, T: Optional[int] = None) -> moe_dims_t:
+    """moe_dims_t of a workload description with fields T, D, E, F, k, S, Fs, scale."""
+    return moe_dims_t(cfg.T if T is None else T, cfg.D, cfg.E, cfg.F, cfg.k, cfg.S, cfg.Fs,
+                      cfg.scale)
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m sparse_moe_layer_04_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    D = ctypes.POINTER(moe_dims_t)
+    sig = {
+        "moe_workspace_size": (Z, [D]),
+        "moe_router_logits": (I, [P, P, D, P, P, Z, P]),
+        "moe_route": (I, [P, P, D, P, P, P, P]),
+        "moe_permute": (I, [P, D, P, P, P, P, P, Z, P]),
+        "moe_expert_ffn": (I, [P, P, P, P, P, P, P, P, P, D, P, P, Z, P]),
+        "moe_combine": (I, [P, P, P, D, P, P, P]),
+        "moe_forward": (I, [P, P, P, P, P, P, P, P, P, D, P, P, P, P, Z, P]),
+        "moe_get_device_status": (I, [P, P]),
+        "moe_last_error": (ctypes.c_char_p, []),
+        "moe_last_launch_count": (I, []),
+        "moe_set_profile_events": (I, [ctypes.POINTER(P), I]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _check(rc: int) -> None:
+    if rc != MOE_OK:
+        raise MoeError(rc, _lib.moe_last_error().decode())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name: str = "tensor") -> Optional[int]:
+    if t is None:
+        return None
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _ws(ws: Optional[torch.Tensor]):
+    if ws is None:
+        return None, 0
+    return _ptr(ws, torch.uint8, "ws"), ws.numel()
+
+
+def moe_workspace_size(d: moe_dims_t) -> int:
+    n = _lib.moe_workspace_size(ctypes.byref(d))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, f"invalid dimensions {d}")
+    return n
+
+
+def alloc_workspace(d: moe_dims_t, device="cuda") -> torch.Tensor:
+    """A zeroed workspace of moe_workspace_size(d) bytes (torch allocations are 256-B aligned)."""
+    return torch.zeros(moe_workspace_size(d), dtype=torch.uint8, device=device)
+
+
+def moe_router_logits(h, Wr, d, logits, ws=None, stream=None) -> None:
+    wp, wn = _ws(ws)
+    _check(_lib.moe_router_logits(_ptr(h, torch.bfloat16, "h"), _ptr(Wr, torch.float32, "Wr"),
+                                  ctypes.byref(d), _ptr(logits, torch.float32, "logits"), wp, wn,
+                                  _stream(stream)))
+
+
+def moe_route(logits, bias, d, idx, w, ws=None, stream=None) -> None:
+    wp, _ = _ws(ws)
+    _check(_lib.moe_route(_ptr(logits, torch.float32, "logits"), _ptr(bias, torch.float32, "bias"),
+                          ctypes.byref(d), _ptr(idx, torch.int32, "idx"),
+                          _ptr(w, torch.float32, "w"), wp, _stream(stream)))
+
+
+def moe_permute(idx, d, counts, offsets, perm, inv, ws, stream=None) -> None:
+    wp, wn = _ws(ws)
+    _check(_lib.moe_permute(_ptr(idx, torch.int32, "idx"), ctypes.byref(d),
+                            _ptr(counts, torch.int32, "counts"),
+                            _ptr(offsets, torch.int32, "offsets"), _ptr(perm, torch.int32, "perm"),
+                            _ptr(inv, torch.int32, "inv"), wp, wn, _stream(stream)))
+
+
+def moe_expert_ffn(h, perm, offsets, W1, W3, W2, Ws1, Ws3, Ws2, d, y, ws, stream=None) -> None:
+    wp, wn = _ws(ws)
+    bf = torch.bfloat16
+    _check(_lib.moe_expert_ffn(_ptr(h, bf, "h"), _ptr(perm, torch.int32, "perm"),
+                               _ptr(offsets, torch.int32, "offsets"), _ptr(W1, bf, "W1"),
+                               _ptr(W3, bf, "W3"), _ptr(W2, bf, "W2"), _ptr(Ws1, bf, "Ws1"),
+                               _ptr(Ws3, bf, "Ws3"), _ptr(Ws2, bf, "Ws2"), ctypes.byref(d),
+                               _ptr(y, torch.float32, "y"), wp, wn, _stream(stream)))
+
+
+def moe_combine(y, w, inv, d, out, ws=None, stream=None) -> None:
+    wp, _ = _ws(ws)
+    _check(_lib.moe_combine(_ptr(y, torch.float32, "y"), _ptr(w, torch.float32, "w"),
+                            _ptr(inv, torch.int32, "inv"), ctypes.byref(d),
+                            _ptr(out, torch.bfloat16, "out"), wp, _stream(stream)))
+
+
+def moe_forward(h, Wr, bias, W1, W3, W2, Ws1, Ws3, Ws2, d, out, ws, idx_out=None, w_out=None,
+                stream=None) -> None:
+    wp, wn = _ws(ws)
+    bf = torch.bfloat16
+    _check(_lib.moe_forward(_ptr(h, bf, "h"), _ptr(Wr, torch.float32, "Wr"),
+                            _ptr(bias, torch.float32, "bias"), _ptr(W1, bf, "W1"),
+                            _ptr(W3, bf, "W3"), _ptr(W2, bf, "W2"), _ptr(Ws1, bf, "Ws1"),
+                            _ptr(Ws3, bf, "Ws3"), _ptr(Ws2, bf, "Ws2"), ctypes.byref(d),
+                            _ptr(out, bf, "out"), _ptr(idx_out, torch.int32, "idx_out"),
+                            _ptr(w_out, torch.float32, "w_out"), wp, wn, _stream(stream)))
+
+
+def moe_get_device_status(ws, stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the first device-side error code."""
+    return _lib.moe_get_device_status(_ptr(ws, torch.uint8, "ws"), _stream(stream))
+
+
+def moe_last_error() -> str:
+    return _lib.moe_last_error().decode()
+
+
+def moe_last_launch_count() -> int:
+    return _lib.moe_last_launch_count()
+
+
+MOE_PROFILE_EVENTS = 8
+_prof_keep = None
+
+
+def moe_set_profile_events(events) -> None:
+    """Record torch.cuda.Event objects at moe_forward's stage boundaries (None: stop)."""
+    global _prof_keep
+    if events is None:
+        _check(_lib.moe_set_profile_events(None, 0))
+        _prof_keep = None
+        return
+    if len(events) != MOE_PROFILE_EVENTS:
+        raise ValueError(f"need {MOE_PROFILE_EVENTS} events")
+    for ev in events:  # torch creates the underlying CUDA event on first record
+        if not ev.cuda_event:
+            ev.record()
+    arr = (ctypes.c_void_p * MOE_PROFILE_EVENTS)(*[ev.cuda_event for ev in events])
+    _check(_lib.moe_set_profile_events(arr, MOE_PROFILE_EVENTS))
+    _prof_keep = (arr, events)

@@ -1,0 +1,440 @@
+// C ABI of the library: argument checks, workspace layout, launches.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+thread_local std::string g_err;
+thread_local int g_launches = 0;
+thread_local void* const* g_prof_events = nullptr;
+
+// Records stage-boundary event i of moe_forward when profiling is enabled.
+cudaError_t mark(int i, cudaStream_t st) {
+  if (!g_prof_events) return cudaSuccess;
+  return cudaEventRecord(static_cast<cudaEvent_t>(g_prof_events[i]), st);
+}
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDev = 64;
+
+int check_device() {
+  static int checked[kMaxDev] = {0};  // 0 unknown, 1 ok, -1 unsupported
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDev) return fail(MOE_ERR_UNSUPPORTED, "device index %d", dev);
+  if (checked[dev] == 0) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    checked[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  if (checked[dev] < 0)
+    return fail(MOE_ERR_UNSUPPORTED, "this library is built for sm_100a (B200) devices only");
+  return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const moe_dims_t* d) {
+  if (!d) return fail(MOE_ERR_INVALID_ARG, "dims is NULL");
+  if (d->T < 0) return fail(MOE_ERR_INVALID_ARG, "T = %d < 0", d->T);
+  if (d->E < 1 || d->E > 1024) return fail(MOE_ERR_INVALID_ARG, "E = %d outside [1, 1024]", d->E);
+  if (d->k < 1 || d->k > 32 || d->k > d->E)
+    return fail(MOE_ERR_INVALID_ARG, "k = %d outside [1, min(E, 32)]", d->k);
+  if (d->D < 8 || d->D % 8) return fail(MOE_ERR_INVALID_ARG, "D = %d not a positive multiple of 8", d->D);
+  if (d->F < 8 || d->F % 8) return fail(MOE_ERR_INVALID_ARG, "F = %d not a positive multiple of 8", d->F);
+  if (d->S < 0 || d->S > 16) return fail(MOE_ERR_INVALID_ARG, "S = %d outside [0, 16]", d->S);
+  if (d->S > 0 && (d->Fs < 8 || d->Fs % 8))
+    return fail(MOE_ERR_INVALID_ARG, "Fs = %d not a positive multiple of 8", d->Fs);
+  if (!(d->scale == d->scale) || d->scale > 3.4e38f || d->scale < -3.4e38f)
+    return fail(MOE_ERR_INVALID_ARG, "scale is not finite");
+  const long long rows = (long long)d->T * d->k + (long long)d->S * d->T;
+  if (rows >= (1ll << 31)) return fail(MOE_ERR_UNSUPPORTED, "T*k + S*T >= 2^31");
+  if ((long long)d->E * d->F >= (1ll << 31) || (long long)d->E * d->D >= (1ll << 31))
+    return fail(MOE_ERR_UNSUPPORTED, "E*F or E*D >= 2^31");
+  return MOE_OK;
+}
+
+#define MOE_CHECK_PTR(p)                                                          \
+  do {                                                                            \
+    if (!(p)) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", #p);                 \
+    if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+  } while (0)
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Ws {
+  WsLayout L;
+  uint8_t* base;
+  template <typename T>
+  T* at(size_t off) const { return reinterpret_cast<T*>(base + off); }
+  int* status() const { return base ? reinterpret_cast<int*>(base + L.status) : nullptr; }
+};
+
+int check_ws(const moe_dims_t* d, void* ws, size_t ws_bytes, Ws* out) {
+  if (!ws_layout(*d, &out->L)) return fail(MOE_ERR_INVALID_ARG, "workspace layout overflow");
+  if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) & 255u)
+    return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (ws_bytes < out->L.total)
+    return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, out->L.total);
+  out->base = static_cast<uint8_t*>(ws);
+  return MOE_OK;
+}
+
+// Host-side checks come first and touch no CUDA API, so argument errors are
+// reported the same way with or without a device.
+int begin(const moe_dims_t* d) {
+  g_err.clear();
+  g_launches = 0;
+  return check_dims(d);
+}
+
+}  // namespace
+
+int num_sms() {
+  static int cache[kMaxDev] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= kMaxDev) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+bool ws_layout(const moe_dims_t& d, WsLayout* L) {
+  const size_t T = d.T, D = d.D, E = d.E, F = d.F, k = d.k, S = d.S, Fs = d.S > 0 ? d.Fs : 0;
+  const RouterSplit sp = router_split(d.T, d.D, d.E);
+  const size_t nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L->status = take(256);
+  L->partials = take((size_t)sp.nsplit * T * E * 4);
+  L->idx = take(T * k * 4);
+  L->w = take(T * k * 4);
+  L->counts = take(E * 4);
+  L->offsets = take((E + 1) * 4);
+  L->perm = take(T * k * 4);
+  L->inv = take(T * k * 4);
+  L->blk_base = take(nblk * E * 4);
+  L->xperm = take(T * k * D * 2);
+  L->act_r = take(T * k * F * 2);
+  L->act_s = take(S * T * Fs * 2);
+  L->y = take((T * k + S * T) * D * 4);
+  L->total = off;
+  return true;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_dims_t* dims) {
+  if (check_dims(dims) != MOE_OK) return 0;
+  WsLayout L;
+  ws_layout(*dims, &L);
+  return L.total;
+}
+
+const char* moe_last_error(void) { return g_err.c_str(); }
+
+int moe_last_launch_count(void) { return g_launches; }
+
+int moe_set_profile_events(void* const* events, int n) {
+  g_err.clear();
+  if (n == 0) {
+    g_prof_events = nullptr;
+    return MOE_OK;
+  }
+  if (n != MOE_PROFILE_EVENTS || !events)
+    return fail(MOE_ERR_INVALID_ARG, "profile events: need %d event handles", MOE_PROFILE_EVENTS);
+  for (int i = 0; i < n; ++i)
+    if (!events[i]) return fail(MOE_ERR_INVALID_ARG, "profile event %d is NULL", i);
+  g_prof_events = events;
+  return MOE_OK;
+}
+
+int moe_router_logits(const void* h, const float* Wr, const moe_dims_t* dims, float* logits,
+                      void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int rc = begin(dims);
+  if (rc) return rc;
+  if (dims->T == 0) return MOE_OK;
+  MOE_CHECK_PTR(h);
+  MOE_CHECK_PTR(Wr);
+  MOE_CHECK_PTR(logits);
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const RouterSplit sp = router_split(dims->T, dims->D, dims->E);
+  Ws w;
+  if (sp.nsplit > 1 && (rc = check_ws(dims, ws, ws_bytes, &w))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaError_t e;
+  if (sp.nsplit == 1) {
+    e = launch_router_partials(static_cast<const uint16_t*>(h), Wr, dims->T, dims->D, dims->E, sp,
+                               logits, st);
+    if (e != cudaSuccess) return cuda_fail(e, "router logits launch");
+    g_launches = 1;
+    return MOE_OK;
+  }
+  float* partials = w.at<float>(w.L.partials);
+  e = launch_router_partials(static_cast<const uint16_t*>(h), Wr, dims->T, dims->D, dims->E, sp,
+                             partials, st);
+  if (e != cudaSuccess) return cuda_fail(e, "router logits launch");
+  e = launch_reduce_partials(partials, sp.nsplit, (size_t)dims->T * dims->E, logits, st);
+  if (e != cudaSuccess) return cuda_fail(e, "router reduce launch");
+  g_launches = 2;
+  return MOE_OK;
+}
+
+int moe_route(const float* logits, const float* bias, const moe_dims_t* dims, int32_t* idx,
+              float* w, void* ws, moe_stream_t stream) {
+  int rc = begin(dims);
+  if (rc) return rc;
+  if (dims->T == 0) return MOE_OK;
+  MOE_CHECK_PTR(logits);
+  MOE_CHECK_PTR(bias);
+  MOE_CHECK_PTR(idx);
+  MOE_CHECK_PTR(w);
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  WsLayout L;
+  ws_layout(*dims, &L);
+  int* status = ws ? reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status) : nullptr;
+  if ((rc = check_device())) return rc;
+  cudaError_t e = launch_route(logits, 1, bias, dims->T, dims->E, dims->k, dims->scale, idx, w,
+                               status, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "route launch");
+  g_launches = 1;
+  return MOE_OK;
+}
+
+int moe_permute(const int32_t* idx, const moe_dims_t* dims, int32_t* counts, int32_t* offsets,
+                int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int rc = begin(dims);
+  if (rc) return rc;
+  MOE_CHECK_PTR(counts);
+  MOE_CHECK_PTR(offsets);
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->T == 0) {
+    if ((rc = check_device())) return rc;
+    // no pairs: every count and offset is zero
+    cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)dims->E * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, (size_t)(dims->E + 1) * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "memset");
+    return MOE_OK;
+  }
+  MOE_CHECK_PTR(idx);
+  MOE_CHECK_PTR(perm);
+  MOE_CHECK_PTR(inv);
+  Ws w;
+  if ((rc = check_ws(dims, ws, ws_bytes, &w))) return rc;
+  if ((rc = check_device())) return rc;
+  int n = 0;
+  cudaError_t e = launch_permute(idx, dims->T, dims->E, dims->k, counts, offsets, perm, inv,
+                                 w.at<int32_t>(w.L.blk_base), w.status(), st, &n);
+  if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  g_launches = n;
+  return MOE_OK;
+}
+
+int moe_expert_ffn(const void* h, const int32_t* perm, const int32_t* offsets, const void* W1,
+                   const void* W3, const void* W2, const void* Ws1, const void* Ws3,
+                   const void* Ws2, const moe_dims_t* dims, float* y, void* ws, size_t ws_bytes,
+                   moe_stream_t stream) {
+  int rc = begin(dims);
+  if (rc) return rc;
+  if (dims->T == 0) return MOE_OK;
+  MOE_CHECK_PTR(h);
+  MOE_CHECK_PTR(perm);
+  MOE_CHECK_PTR(offsets);
+  MOE_CHECK_PTR(W1);
+  MOE_CHECK_PTR(W3);
+  MOE_CHECK_PTR(W2);
+  MOE_CHECK_PTR(y);
+  if (dims->S > 0) {
+    MOE_CHECK_PTR(Ws1);
+    MOE_CHECK_PTR(Ws3);
+    MOE_CHECK_PTR(Ws2);
+  }
+  Ws w;
+  if ((rc = check_ws(dims, ws, ws_bytes, &w))) return rc;
+  if ((rc = check_device())) return rc;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int rows = dims->T * dims->k;
+  uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
+  cudaError_t e = launch_gather_rows(static_cast<const uint16_t*>(h), perm, rows, dims->D,
+                                     dims->T, xperm, st);
+  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  FfnArgs a;
+  a.xperm = xperm;
+  a.h = static_cast<const uint16_t*>(h);
+  a.offsets = offsets;
+  a.W1 = static_cast<const uint16_t*>(W1);
+  a.W3 = static_cast<const uint16_t*>(W3);
+  a.W2 = static_cast<const uint16_t*>(W2);
+  a.Ws1 = static_cast<const uint16_t*>(Ws1);
+  a.Ws3 = static_cast<const uint16_t*>(Ws3);
+  a.Ws2 = static_cast<const uint16_t*>(Ws2);
+  a.act_r = w.at<uint16_t>(w.L.act_r);
+  a.act_s = w.at<uint16_t>(w.L.act_s);
+  a.y = y;
+  a.status = w.status();
+  a.T = dims->T; a.D = dims->D; a.E = dims->E; a.F = dims->F; a.k = dims->k;
+  a.S = dims->S; a.Fs = dims->Fs;
+  int n = 1;
+  const char* why = "launch failed";
+  e = launch_expert_ffn(a, st, &n, &why, nullptr);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
+  g_launches = n;
+  return MOE_OK;
+}
+
+int moe_combine(const float* y, const float* w, const int32_t* inv, const moe_dims_t* dims,
+                void* out, void* ws, moe_stream_t stream) {
+  int rc = begin(dims);
+  if (rc) return rc;
+  if (dims->T == 0) return MOE_OK;
+  MOE_CHECK_PTR(y);
+  MOE_CHECK_PTR(w);
+  MOE_CHECK_PTR(inv);
+  MOE_CHECK_PTR(out);
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  WsLayout L;
+  ws_layout(*dims, &L);
+  int* status = ws ? reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status) : nullptr;
+  if ((rc = check_device())) return rc;
+  cudaError_t e = launch_combine(y, w, inv, dims->T, dims->D, dims->k, dims->S,
+                                 static_cast<uint16_t*>(out), status,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  g_launches = 1;
+  return MOE_OK;
+}
+
+int moe_forward(const void* h, const float* Wr, const float* bias, const void* W1,
+                const void* W3, const void* W2, const void* Ws1, const void* Ws3,
+                const void* Ws2, const moe_dims_t* dims, void* out, int32_t* idx_out,
+                float* w_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int rc = begin(dims);
+  if (rc) return rc;
+  if (dims->T == 0) return MOE_OK;
+  MOE_CHECK_PTR(h);
+  MOE_CHECK_PTR(Wr);
+  MOE_CHECK_PTR(bias);
+  MOE_CHECK_PTR(W1);
+  MOE_CHECK_PTR(W3);
+  MOE_CHECK_PTR(W2);
+  MOE_CHECK_PTR(out);
+  if (dims->S > 0) {
+    MOE_CHECK_PTR(Ws1);
+    MOE_CHECK_PTR(Ws3);
+    MOE_CHECK_PTR(Ws2);
+  }
+  if (idx_out && !aligned16(idx_out)) return fail(MOE_ERR_INVALID_ARG, "idx_out is not 16-byte aligned");
+  if (w_out && !aligned16(w_out)) return fail(MOE_ERR_INVALID_ARG, "w_out is not 16-byte aligned");
+  Ws w;
+  if ((rc = check_ws(dims, ws, ws_bytes, &w))) return rc;
+  if ((rc = check_device())) return rc;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int T = dims->T, D = dims->D, E = dims->E, k = dims->k;
+  const auto* hb = static_cast<const uint16_t*>(h);
+  int32_t* idx = idx_out ? idx_out : w.at<int32_t>(w.L.idx);
+  float* rw = w_out ? w_out : w.at<float>(w.L.w);
+  int32_t* counts = w.at<int32_t>(w.L.counts);
+  int32_t* offsets = w.at<int32_t>(w.L.offsets);
+  int32_t* perm = w.at<int32_t>(w.L.perm);
+  int32_t* inv = w.at<int32_t>(w.L.inv);
+  float* y = w.at<float>(w.L.y);
+  int n = 0;
+
+  const RouterSplit sp = router_split(T, D, E);
+  float* partials = w.at<float>(w.L.partials);
+  cudaError_t e = mark(0, st);
+  if (e == cudaSuccess) e = launch_router_partials(hb, Wr, T, D, E, sp, partials, st);
+  if (e == cudaSuccess) e = mark(1, st);
+  if (e != cudaSuccess) return cuda_fail(e, "router logits launch");
+  e = launch_route(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw, w.status(), st);
+  if (e == cudaSuccess) e = mark(2, st);
+  if (e != cudaSuccess) return cuda_fail(e, "route launch");
+  n += 2;
+  e = launch_permute(idx, T, E, k, counts, offsets, perm, inv, w.at<int32_t>(w.L.blk_base),
+                     w.status(), st, &n);
+  if (e == cudaSuccess) e = mark(3, st);
+  if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
+  e = launch_gather_rows(hb, perm, T * k, D, T, xperm, st);
+  if (e == cudaSuccess) e = mark(4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  n += 1;
+  FfnArgs a;
+  a.xperm = xperm;
+  a.h = hb;
+  a.offsets = offsets;
+  a.W1 = static_cast<const uint16_t*>(W1);
+  a.W3 = static_cast<const uint16_t*>(W3);
+  a.W2 = static_cast<const uint16_t*>(W2);
+  a.Ws1 = static_cast<const uint16_t*>(Ws1);
+  a.Ws3 = static_cast<const uint16_t*>(Ws3);
+  a.Ws2 = static_cast<const uint16_t*>(Ws2);
+  a.act_r = w.at<uint16_t>(w.L.act_r);
+  a.act_s = w.at<uint16_t>(w.L.act_s);
+  a.y = y;
+  a.status = w.status();
+  a.T = T; a.D = D; a.E = E; a.F = dims->F; a.k = k; a.S = dims->S; a.Fs = dims->Fs;
+  const char* why = "launch failed";
+  e = launch_expert_ffn(a, st, &n, &why, g_prof_events ? g_prof_events + 5 : nullptr);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
+  e = launch_combine(y, rw, inv, T, D, k, dims->S, static_cast<uint16_t*>(out), w.status(), st);
+  if (e == cudaSuccess) e = mark(7, st);
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  n += 1;
+  g_launches = n;
+  return MOE_OK;
+}
+
+int moe_get_device_status(void* ws, moe_stream_t stream) {
+  g_err.clear();
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (word & kStNonFinite) return fail(MOE_ERR_NONFINITE, "device: non-finite router logit or key");
+  if (word & kStBounds)
+    return fail(MOE_ERR_BOUNDS, "device: expert index, group offset or row index out of range");
+  if (word & kStTimeout) return fail(MOE_ERR_TIMEOUT, "device: a bounded wait gave up");
+  return MOE_OK;
+}
+
+}  // extern "C"

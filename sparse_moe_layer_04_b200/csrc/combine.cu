@@ -1,0 +1,65 @@
+// Merge of the weighted routed expert outputs with the always-on shared
+// expert(s) ("Model anatomy -- GLM-5.2", MoE panel: the renormalised, scaled
+// expert outputs are merged with one always-on shared expert; "Expert fan-out
+// 8 + 1").  Deterministic: each output element is summed in one fixed order,
+// shared experts first, then slots 0..k-1, without atomics.
+#include <cuda_bf16.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+constexpr int kCombineThreads = 256;
+constexpr int kMaxK = 32;
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(
+    const float* __restrict__ y, const float* __restrict__ w, const int32_t* __restrict__ inv,
+    int T, int D, int k, int S, uint16_t* __restrict__ out, int* __restrict__ status) {
+  __shared__ int s_row[kMaxK];
+  __shared__ float s_w[kMaxK];
+  const int t = blockIdx.x;
+  const size_t rows_r = (size_t)T * k;
+  if (threadIdx.x < k) {
+    int r = inv[(size_t)t * k + threadIdx.x];
+    if (r < 0 || (size_t)r >= rows_r) {
+      if (status) atomicOr(status, kStBounds);
+      r = -1;
+    }
+    s_row[threadIdx.x] = r;
+    s_w[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
+  }
+  __syncthreads();
+  const int nvec = D / 4;
+  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < S; ++s) {
+      const float4 a = reinterpret_cast<const float4*>(y + (rows_r + (size_t)s * T + t) * D)[v];
+      acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
+    }
+    for (int j = 0; j < k; ++j) {
+      const int r = s_row[j];
+      if (r < 0) continue;
+      const float wj = s_w[j];
+      const float4 a = reinterpret_cast<const float4*>(y + (size_t)r * D)[v];
+      acc.x = fmaf(wj, a.x, acc.x);
+      acc.y = fmaf(wj, a.y, acc.y);
+      acc.z = fmaf(wj, a.z, acc.z);
+      acc.w = fmaf(wj, a.w, acc.w);
+    }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(out + (size_t)t * D)[v] = pk;
+  }
+}
+
+cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, int T, int D,
+                           int k, int S, uint16_t* out, int* status, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  combine_kernel<<<T, kCombineThreads, 0, st>>>(y, w, inv, T, D, k, S, out, status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

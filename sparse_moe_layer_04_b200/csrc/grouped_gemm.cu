@@ -1,0 +1,494 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM),
+// operands staged by TMA.
+//
+// The expert MLP is y = w2 (silu(w1 x) * (w3 x)) with w1/w3 the input
+// projections and w2 the output projection ("GLM-5.2", PocketLLM,
+// Implemented execution path, names w1/w3 and w2; the gated form is the
+// reading taken where the pages are silent).  The routed experts see only the
+// rows grouped to them; the always-on shared expert sees every token ("Model
+// anatomy -- GLM-5.2", MoE panel, and "Expert fan-out 8 + 1").
+//
+// Two launches:
+//   gate/up : act[r, n] = silu(sum_d A[r, d] W1[e][n, d]) * (sum_d A[r, d] W3[e][n, d])
+//             128 x 128 output tile; the W1 and W3 row blocks of the tile are
+//             stacked into one 256-row B operand, so one N = 256 MMA feeds
+//             both accumulators (TMEM columns 0-127 gate, 128-255 up) and the
+//             epilogue applies the SiLU gate and rounds to bf16.
+//   down    : y[r, n] = sum_f act[r, f] W2[e][n, f], 128 x 256 fp32 tile.
+//
+// Kernel structure (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: 4-stage ring of (A 128x64, B 256x64) bf16 tiles,
+//               128-byte swizzled, completion counted on "full" mbarriers.
+//   warp 1      TMEM allocator and single-thread MMA issuer:
+//               tcgen05.mma.cta_group::1.kind::f16, M = 128, N = 256, K = 16,
+//               fp32 accumulators in TMEM, two accumulator buffers so the
+//               epilogue of tile i overlaps the main loop of tile i+1.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32*(w%4) .. +31), fused activation, global stores.
+// Tiles are numbered routed-first (expert, n-tile, m-tile with m fastest, so
+// CTAs that run at the same time share each weight tile through L2), then the
+// shared experts; CTA c takes tiles c, c + gridDim.x, ...  The routed tile
+// count comes from the device-side group offsets, so no host round trip.
+#include <cuda_bf16.h>
+
+#include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                    // one 128-byte swizzle row of bf16
+constexpr int STAGES = 4;
+constexpr int THREADS = 192;
+constexpr int MMA_N = 256;
+constexpr int A_BYTES = BM * BK * 2;      // 16 KiB
+constexpr int B_BYTES = MMA_N * BK * 2;   // 32 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int ACC_COLS = MMA_N;           // fp32 TMEM columns per accumulator
+constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+constexpr int MAX_E = 1024;
+constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, MMA_N);
+
+struct GemmParams {
+  CUtensorMap a_r;   // routed A  [rows_r, K_r]
+  CUtensorMap a_s;   // shared A  [.., K_s]
+  CUtensorMap b0_r;  // W1 [E*F, D] (gate/up) | W2 [E*D, F] (down)
+  CUtensorMap b1_r;  // W3 [E*F, D] (gate/up only)
+  CUtensorMap b0_s;  // Ws1 | Ws2
+  CUtensorMap b1_s;  // Ws3
+  const int32_t* offsets;
+  void* out_r;
+  void* out_s;
+  int* status;
+  int E, S, T;
+  int K_r, K_s;              // reduction lengths
+  int N_r, N_s;              // output columns (= output row strides)
+  int rows_r;                // T * k
+  int a_s_group_stride;      // rows between shared experts' A blocks (0 or T)
+  int b_r_group_rows;        // B rows per routed expert (F or D)
+  int b_s_group_rows;        // B rows per shared expert (Fs or D)
+  int bn_out;                // output columns per tile (128 or 256)
+};
+
+struct SharedState {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int routed_tiles;
+  int off[MAX_E + 1];        // group row offsets
+  int prefix[MAX_E + 1];     // routed tile prefix per expert
+};
+
+struct TileInfo {
+  bool shared;
+  int grp;      // expert (routed) or shared expert index
+  int m0;       // first row within the group
+  int n0;       // first output column
+  int rows;     // rows in the group
+  int row0;     // group's first row in the output (and routed A) matrix
+};
+
+__device__ __forceinline__ TileInfo decode_tile(int tile, const SharedState& ss,
+                                                const GemmParams& p) {
+  TileInfo ti;
+  if (tile < ss.routed_tiles) {
+    int lo = 0, hi = p.E - 1;  // find e with prefix[e] <= tile < prefix[e+1]
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (ss.prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int rows = ss.off[e + 1] - ss.off[e];
+    const int mt = (rows + BM - 1) / BM;
+    const int local = tile - ss.prefix[e];
+    ti.shared = false;
+    ti.grp = e;
+    ti.m0 = (local % mt) * BM;
+    ti.n0 = (local / mt) * p.bn_out;
+    ti.rows = rows;
+    ti.row0 = ss.off[e];
+  } else {
+    const int local = tile - ss.routed_tiles;
+    const int mt = (p.T + BM - 1) / BM;
+    const int nt = (p.N_s + p.bn_out - 1) / p.bn_out;
+    const int s = local / (mt * nt);
+    const int rem = local - s * mt * nt;
+    ti.shared = true;
+    ti.grp = s;
+    ti.m0 = (rem % mt) * BM;
+    ti.n0 = (rem / mt) * p.bn_out;
+    ti.rows = p.T;
+    ti.row0 = s * p.T;
+  }
+  return ti;
+}
+
+__device__ __forceinline__ float silu_times(float g, float u) {
+  return g / (1.0f + __expf(-g)) * u;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Waits for in-flight async work even after an abort (bounded by the same
+// clock budget); a timeout here raises the CTA's abort flag too.
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  int ignore_abort = 0;
+  if (!ptx::mbar_wait(bar, parity, &ignore_abort)) *abort = 1;
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned operand ring (128-byte swizzle atoms span 1024 bytes)
+  const uint32_t raw_addr = ptx::smem_addr(smem_raw);
+  uint8_t* ring = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  SharedState& ss = *reinterpret_cast<SharedState*>(ring + STAGES * STAGE_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (warp == 1) {
+    ptx::tmem_alloc(&ss.tmem_base, TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      ptx::mbar_init(&ss.full[i], 1);
+      ptx::mbar_init(&ss.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&ss.tmem_full[i], 1);
+      ptx::mbar_init(&ss.tmem_empty[i], 4);
+    }
+    ptx::mbar_init(&ss.drain, 1);
+    ss.abort = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::tma_prefetch_desc(&p.a_r);
+    ptx::tma_prefetch_desc(&p.b0_r);
+    if (GATEUP) ptx::tma_prefetch_desc(&p.b1_r);
+  }
+  // Routed tile prefix from the group offsets (warp 2 scans 32 experts at a time).
+  if (warp == 2) {
+    int carry = 0;
+    bool bad = false;
+    const int nt = (p.N_r + p.bn_out - 1) / p.bn_out;
+    for (int base = 0; base < p.E; base += 32) {
+      const int e = base + lane;
+      int cnt = 0;
+      if (e < p.E) {
+        const int a = p.offsets[e], b = p.offsets[e + 1];
+        ss.off[e] = a;
+        if (e == p.E - 1) ss.off[p.E] = b;
+        if (a < 0 || b < a || b > p.rows_r || (e == 0 && a != 0)) bad = true;
+        cnt = ((b - a + BM - 1) / BM) * nt;
+        if (b < a) cnt = 0;
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      if (e < p.E) ss.prefix[e] = carry + incl - cnt;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      ss.prefix[p.E] = carry;
+      ss.routed_tiles = bad ? 0 : carry;
+      if (bad && p.status) atomicOr(p.status, kStBounds);
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+
+  const uint32_t tmem_base = ss.tmem_base;
+  const int mt_s = (p.T + BM - 1) / BM;
+  const int nt_s = (p.N_s + p.bn_out - 1) / p.bn_out;
+  const int total = ss.routed_tiles + p.S * mt_s * nt_s;
+  volatile int* abort = &ss.abort;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, last_parity = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const TileInfo ti = decode_tile(tile, ss, p);
+        const CUtensorMap* amap = ti.shared ? &p.a_s : &p.a_r;
+        const CUtensorMap* b0 = ti.shared ? &p.b0_s : &p.b0_r;
+        const CUtensorMap* b1 = ti.shared ? &p.b1_s : &p.b1_r;
+        const int a_row = ti.shared ? ti.grp * p.a_s_group_stride + ti.m0 : ti.row0 + ti.m0;
+        const int b_row = ti.grp * (ti.shared ? p.b_s_group_rows : p.b_r_group_rows) + ti.n0;
+        const int K = ti.shared ? p.K_s : p.K_r;
+        const int nk = (K + BK - 1) / BK;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&ss.empty[stage], phase ^ 1u, abort)) { ok = false; break; }
+          uint8_t* sa = ring + stage * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          ptx::mbar_arrive_expect_tx(&ss.full[stage], STAGE_BYTES);
+          ptx::tma_load_2d(sa, amap, &ss.full[stage], kb * BK, a_row);
+          if (GATEUP) {
+            ptx::tma_load_2d(sb, b0, &ss.full[stage], kb * BK, b_row);
+            ptx::tma_load_2d(sb + B_BYTES / 2, b1, &ss.full[stage], kb * BK, b_row);
+          } else {
+            ptx::tma_load_2d(sb, b0, &ss.full[stage], kb * BK, b_row);
+          }
+          issued_mask |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      // every issued load has landed before the CTA may retire
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s)) wait_drain(&ss.full[s], (last_parity >> s) & 1u, abort);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const TileInfo ti = decode_tile(tile, ss, p);
+        const int K = ti.shared ? p.K_s : p.K_r;
+        const int nk = (K + BK - 1) / BK;
+        if (!ptx::mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1u, abort)) break;
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&ss.full[stage], phase, abort)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint32_t sa = ptx::smem_addr(ring + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            ptx::mma_f16_ss(d_tmem, ptx::smem_desc_sw128(sa + kk * 32),
+                            ptx::smem_desc_sw128(sb + kk * 32), IDESC,
+                            (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          ptx::mma_commit(&ss.empty[stage]);   // frees the smem stage when these MMAs finish
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        ptx::mma_commit(&ss.tmem_full[acc]);   // accumulator ready for the epilogue
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      ptx::mma_commit(&ss.drain);
+      wait_drain(&ss.drain, 0, abort);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const TileInfo ti = decode_tile(tile, ss, p);
+      if (!ptx::mbar_wait(&ss.tmem_full[acc], acc_phase, abort)) break;
+      ptx::tc_fence_after();
+      const int r = ti.m0 + q * 32 + lane;       // row within the group
+      const bool row_ok = r < ti.rows;
+      const int N = ti.shared ? p.N_s : p.N_r;
+      const size_t out_row = (size_t)ti.row0 + r;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * ACC_COLS;
+      if (GATEUP) {
+        uint16_t* out = static_cast<uint16_t*>(ti.shared ? p.out_s : p.out_r);
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 16) {
+          uint32_t g[16], u[16];
+          ptx::tmem_ld_x16(taddr + c, g);
+          ptx::tmem_ld_x16(taddr + 128 + c, u);
+          ptx::tmem_wait_ld();
+          const int col = ti.n0 + c;
+          if (row_ok && col < N) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              pk[i] = pack_bf16(silu_times(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                silu_times(__uint_as_float(g[2 * i + 1]),
+                                           __uint_as_float(u[2 * i + 1])));
+            uint4* dst = reinterpret_cast<uint4*>(out + out_row * N + col);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            if (col + 8 < N) dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else {
+        float* out = static_cast<float*>(ti.shared ? p.out_s : p.out_r);
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 16) {
+          uint32_t v[16];
+          ptx::tmem_ld_x16(taddr + c, v);
+          ptx::tmem_wait_ld();
+          const int col = ti.n0 + c;
+          if (row_ok && col < N) {
+            uint4* dst = reinterpret_cast<uint4*>(out + out_row * N + col);
+            dst[0] = make_uint4(v[0], v[1], v[2], v[3]);
+            dst[1] = make_uint4(v[4], v[5], v[6], v[7]);
+            if (col + 8 < N) {
+              dst[2] = make_uint4(v[8], v[9], v[10], v[11]);
+              dst[3] = make_uint4(v[12], v[13], v[14], v[15]);
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&ss.tmem_empty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && ss.abort && p.status) atomicOr(p.status, kStTimeout);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// bf16 row-major [rows, cols] matrix, box = box_rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {BK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(SharedState);
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+template <bool GATEUP>
+cudaError_t launch_one(const GemmParams& p, int tiles_upper, cudaStream_t st) {
+  static int configured_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured_dev = dev;
+  }
+  int grid = num_sms();
+  if (tiles_upper < grid) grid = tiles_upper;
+  if (grid < 1) grid = 1;
+  grouped_gemm_kernel<GATEUP><<<grid, THREADS, kSmemBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, const char** why,
+                              void* const* marks) {
+  const int rows_r = a.T * a.k;
+  const int mt_upper = (rows_r + BM - 1) / BM + a.E;  // sum over experts of ceil(count/BM)
+  const int mt_s = (a.T + BM - 1) / BM;
+
+  // ---- gate/up ----
+  GemmParams g{};
+  bool ok = make_map(&g.a_r, a.xperm, rows_r, a.D, BM) &&
+            make_map(&g.b0_r, a.W1, (uint64_t)a.E * a.F, a.D, 128) &&
+            make_map(&g.b1_r, a.W3, (uint64_t)a.E * a.F, a.D, 128);
+  if (ok && a.S > 0)
+    ok = make_map(&g.a_s, a.h, a.T, a.D, BM) &&
+         make_map(&g.b0_s, a.Ws1, (uint64_t)a.S * a.Fs, a.D, 128) &&
+         make_map(&g.b1_s, a.Ws3, (uint64_t)a.S * a.Fs, a.D, 128);
+  if (!ok) {
+    *why = "cuTensorMapEncodeTiled failed for a gate/up operand";
+    return cudaErrorInvalidValue;
+  }
+  g.offsets = a.offsets;
+  g.out_r = a.act_r;
+  g.out_s = a.act_s;
+  g.status = a.status;
+  g.E = a.E; g.S = a.S; g.T = a.T;
+  g.K_r = a.D; g.K_s = a.D;
+  g.N_r = a.F; g.N_s = a.Fs;
+  g.rows_r = rows_r;
+  g.a_s_group_stride = 0;
+  g.b_r_group_rows = a.F;
+  g.b_s_group_rows = a.Fs;
+  g.bn_out = 128;
+  const int tiles_g = mt_upper * ((a.F + 127) / 128) + a.S * mt_s * ((a.Fs + 127) / 128);
+  cudaError_t err = launch_one<true>(g, tiles_g, st);
+  if (err == cudaSuccess && marks) err = cudaEventRecord(static_cast<cudaEvent_t>(marks[0]), st);
+  if (err != cudaSuccess) return err;
+
+  // ---- down ----
+  GemmParams d{};
+  ok = make_map(&d.a_r, a.act_r, rows_r, a.F, BM) &&
+       make_map(&d.b0_r, a.W2, (uint64_t)a.E * a.D, a.F, 256);
+  if (ok && a.S > 0)
+    ok = make_map(&d.a_s, a.act_s, (uint64_t)a.S * a.T, a.Fs, BM) &&
+         make_map(&d.b0_s, a.Ws2, (uint64_t)a.S * a.D, a.Fs, 256);
+  if (!ok) {
+    *why = "cuTensorMapEncodeTiled failed for a down-projection operand";
+    return cudaErrorInvalidValue;
+  }
+  d.b1_r = d.b0_r;
+  d.b1_s = d.b0_s;
+  d.offsets = a.offsets;
+  d.out_r = a.y;
+  d.out_s = a.y + (size_t)rows_r * a.D;
+  d.status = a.status;
+  d.E = a.E; d.S = a.S; d.T = a.T;
+  d.K_r = a.F; d.K_s = a.Fs;
+  d.N_r = a.D; d.N_s = a.D;
+  d.rows_r = rows_r;
+  d.a_s_group_stride = a.T;
+  d.b_r_group_rows = a.D;
+  d.b_s_group_rows = a.D;
+  d.bn_out = 256;
+  const int nt_d = (a.D + 255) / 256;
+  const int tiles_d = mt_upper * nt_d + a.S * mt_s * nt_d;
+  err = launch_one<false>(d, tiles_d, st);
+  if (err == cudaSuccess && marks) err = cudaEventRecord(static_cast<cudaEvent_t>(marks[1]), st);
+  *nlaunch += 2;
+  return err;
+}
+
+}  // namespace moe

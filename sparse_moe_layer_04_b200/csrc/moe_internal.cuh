@@ -1,0 +1,75 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+// Bits of the device status word (first int32 of the workspace).
+constexpr int kStNonFinite = 1;
+constexpr int kStBounds = 2;
+constexpr int kStTimeout = 4;
+
+// Device count assumed when splitting small problems; the split depends on the
+// shape only, so results are bit-identical on every device.
+constexpr int kSplitTargetBlocks = 296;
+
+// Router logits tiling (fp32 FMA, split over D).
+constexpr int kRouterTileT = 64;
+constexpr int kRouterTileE = 64;
+constexpr int kRouterTileD = 32;
+
+struct RouterSplit {
+  int nsplit;  // partial sums over D
+  int chunk;   // D-range of one split (multiple of kRouterTileD)
+};
+RouterSplit router_split(int T, int D, int E);
+
+// Permute: tokens per counting block.
+constexpr int kPermBlockTokens = 256;
+
+// Workspace layout (byte offsets from the workspace base, 256-aligned).
+struct WsLayout {
+  size_t status, partials, idx, w, counts, offsets, perm, inv, blk_base, xperm, act_r, act_s,
+      y, total;
+};
+bool ws_layout(const moe_dims_t& d, WsLayout* out);
+
+// --- launchers (return cudaSuccess or the launch error) ---------------------
+cudaError_t launch_router_partials(const uint16_t* h, const float* Wr, int T, int D, int E,
+                                   RouterSplit sp, float* out, cudaStream_t st);
+cudaError_t launch_reduce_partials(const float* partials, int nsplit, size_t n, float* out,
+                                   cudaStream_t st);
+cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T, int E, int k,
+                         float scale, int32_t* idx, float* w, int* status, cudaStream_t st);
+cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* blk_base,
+                           int* status, cudaStream_t st, int* nlaunch);
+cudaError_t launch_gather_rows(const uint16_t* h, const int32_t* perm, int rows, int D, int T,
+                               uint16_t* xperm, cudaStream_t st);
+cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, int T, int D,
+                           int k, int S, uint16_t* out, int* status, cudaStream_t st);
+
+// Expert MLPs: gate/up GEMM with the SiLU gate fused, then the down GEMM.
+struct FfnArgs {
+  const uint16_t* xperm;    // [T*k, D] gathered routed rows
+  const uint16_t* h;        // [T, D] (A operand of the shared experts)
+  const int32_t* offsets;   // [E+1]
+  const uint16_t *W1, *W3, *W2, *Ws1, *Ws3, *Ws2;
+  uint16_t* act_r;          // [T*k, F]
+  uint16_t* act_s;          // [S*T, Fs]
+  float* y;                 // [T*k + S*T, D]
+  int* status;
+  int T, D, E, F, k, S, Fs;
+};
+// `marks` (nullable): two events recorded after the gate/up and the down GEMM.
+cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch,
+                              const char** why, void* const* marks);
+
+int num_sms();
+
+}  // namespace moe

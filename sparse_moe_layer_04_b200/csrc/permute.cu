@@ -1,0 +1,168 @@
+// Grouping of (token, slot) pairs by expert: a counting sort over blocks of
+// tokens.  The pages name the expert kernels "grouped" ("GLM-5.2", PocketLLM,
+// Implemented execution path); the grouping itself is the plain counting sort
+// that makes each expert's rows contiguous.
+//
+//   count   : per block of 256 tokens, per-expert counts (shared atomics)
+//   scan    : per-expert running sums over blocks, then an exclusive scan over
+//             experts -> counts, offsets and each block's base row per expert
+//   scatter : a per-block bitmask of the tokens that chose each expert gives
+//             every pair its rank among the block's tokens for that expert
+//             (tokens pick distinct experts, so one bit per token suffices):
+//             row = base[block][e] + rank.  Rows within an expert therefore
+//             follow increasing token order, i.e. (token, slot) order.
+// All integer work: exact and deterministic.
+#include "moe_internal.cuh"
+
+namespace moe {
+
+constexpr int kWordsPerBlock = kPermBlockTokens / 32;
+
+__global__ void __launch_bounds__(kPermBlockTokens) permute_count_kernel(
+    const int32_t* __restrict__ idx, int T, int E, int k, int32_t* __restrict__ blk_counts,
+    int* __restrict__ status) {
+  extern __shared__ int cnt[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int t = blockIdx.x * kPermBlockTokens + threadIdx.x;
+  bool bad = false;
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      if (e < 0 || e >= E) {
+        bad = true;
+        continue;
+      }
+      atomicAdd(&cnt[e], 1);
+    }
+  }
+  if (bad && status) atomicOr(status, kStBounds);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    blk_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// One block of 1024 threads: thread e owns expert e (E <= 1024).
+__global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ blk_base,
+                                                            int nblk, int E,
+                                                            int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E) {
+    for (int b = 0; b < nblk; ++b) {
+      const int c = blk_base[(size_t)b * E + e];
+      blk_base[(size_t)b * E + e] = total;  // exclusive within the expert
+      total += c;
+    }
+    counts[e] = total;
+  }
+  // exclusive scan of `total` over e
+  const int lane = e & 31, wid = e >> 5;
+  int incl = total;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    int v = warp_sums[lane];
+    int s = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += u;
+    }
+    warp_sums[lane] = s - v;  // exclusive over warps
+  }
+  __syncthreads();
+  const int excl = incl - total + warp_sums[wid];
+  if (e < E) {
+    offsets[e] = excl;
+    if (e == E - 1) offsets[E] = excl + total;
+    for (int b = 0; b < nblk; ++b) blk_base[(size_t)b * E + e] += excl;
+  }
+}
+
+__global__ void __launch_bounds__(kPermBlockTokens) permute_scatter_kernel(
+    const int32_t* __restrict__ idx, int T, int E, int k, const int32_t* __restrict__ blk_base,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv, int* __restrict__ status) {
+  extern __shared__ unsigned mask[];  // [E][kWordsPerBlock]
+  for (int i = threadIdx.x; i < E * kWordsPerBlock; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  const int tl = threadIdx.x;
+  const int t = blockIdx.x * kPermBlockTokens + tl;
+  const int word = tl >> 5;
+  const unsigned bit = 1u << (tl & 31);
+  bool bad = false;
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      if (e < 0 || e >= E) {
+        bad = true;
+        continue;
+      }
+      const unsigned old = atomicOr(&mask[e * kWordsPerBlock + word], bit);
+      if (old & bit) bad = true;  // the same expert twice in one token
+    }
+  }
+  __syncthreads();
+  if (t < T && !bad) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      const unsigned* m = mask + e * kWordsPerBlock;
+      int rank = __popc(m[word] & (bit - 1u));
+      for (int q = 0; q < word; ++q) rank += __popc(m[q]);
+      const int row = blk_base[(size_t)blockIdx.x * E + e] + rank;
+      perm[row] = t;
+      inv[(size_t)t * k + j] = row;
+    }
+  }
+  if (bad && status) atomicOr(status, kStBounds);
+}
+
+cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* blk_base,
+                           int* status, cudaStream_t st, int* nlaunch) {
+  const int nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+  permute_count_kernel<<<nblk, kPermBlockTokens, E * sizeof(int), st>>>(idx, T, E, k, blk_base,
+                                                                         status);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  permute_scan_kernel<<<1, 1024, 0, st>>>(blk_base, nblk, E, counts, offsets);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  permute_scatter_kernel<<<nblk, kPermBlockTokens, E * kWordsPerBlock * sizeof(unsigned), st>>>(
+      idx, T, E, k, blk_base, perm, inv, status);
+  *nlaunch += 3;
+  return cudaGetLastError();
+}
+
+// xperm[r] = h[perm[r]] for every grouped row r (16-byte vector copies).  A
+// token id outside [0, T) (left by an invalid routing) yields a zero row.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ h,
+                                                          const int32_t* __restrict__ perm,
+                                                          int D, int T,
+                                                          uint16_t* __restrict__ xperm) {
+  const int r = blockIdx.x;
+  const int t = perm[r];
+  uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)r * D);
+  if (t < 0 || t >= T) {
+    for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(h + (size_t)t * D);
+  for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = src[i];
+}
+
+cudaError_t launch_gather_rows(const uint16_t* h, const int32_t* perm, int rows, int D, int T,
+                               uint16_t* xperm, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  gather_rows_kernel<<<rows, 256, 0, st>>>(h, perm, D, T, xperm);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,109 @@
+"""The C ABI: the library loads, exports every declared entry point, and its
+host-side argument checks reject bad calls before touching the device.
+
+Only calls that must fail validation are made here (null or misaligned
+pointers, bad dimensions, short workspaces), so nothing is ever launched and
+no fake pointer is dereferenced, with or without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+@pytest.fixture(scope="module")
+def mod():
+    from sparse_moe_layer_04_b200 import build
+    build.build()
+    import sparse_moe_layer_04_b200 as m
+    return m
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(mod):
+    names = _declared_functions()
+    assert "moe_forward" in names and "moe_route" in names
+    lib = ctypes.CDLL(mod.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_workspace_size(mod):
+    d = mod.dims(T=128, D=6144, E=256, F=2048, k=8, S=1, Fs=2048, scale=2.5)
+    n = mod.moe_workspace_size(d)
+    # at least the fp32 expert outputs and the gathered rows
+    assert n >= (128 * 8 + 128) * 6144 * 4 + 128 * 8 * 6144 * 2
+    assert n % 256 == 0
+    assert mod._lib.moe_workspace_size(ctypes.byref(mod.dims(T=4, D=12, E=8, F=64, k=2))) == 0
+    assert mod._lib.moe_workspace_size(ctypes.byref(mod.dims(T=4, D=128, E=8, F=64, k=9))) == 0
+    assert mod._lib.moe_workspace_size(ctypes.byref(mod.dims(T=-1, D=128, E=8, F=64, k=2))) == 0
+    assert mod._lib.moe_workspace_size(ctypes.byref(mod.dims(T=4, D=128, E=2000, F=64, k=2))) == 0
+    assert mod._lib.moe_workspace_size(ctypes.byref(mod.dims(T=4, D=128, E=64, F=64, k=33))) == 0
+    assert mod._lib.moe_workspace_size(ctypes.byref(mod.dims(T=0, D=128, E=8, F=64, k=2))) > 0
+
+
+FAKE = 0x7F0000000000  # never dereferenced: every call below fails validation first
+
+
+def test_null_and_misaligned_pointers_rejected(mod):
+    lib = mod._lib
+    d = mod.dims(T=8, D=128, E=8, F=64, k=2)
+    ws_n = mod.moe_workspace_size(d)
+    rc = lib.moe_forward(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(d),
+                         FAKE, None, None, FAKE, ws_n, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "h is NULL" in mod.moe_last_error()
+    rc = lib.moe_forward(FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.byref(d),
+                         FAKE, None, None, FAKE, ws_n, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "aligned" in mod.moe_last_error()
+    rc = lib.moe_route(FAKE, None, ctypes.byref(d), FAKE, FAKE, None, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "bias" in mod.moe_last_error()
+    rc = lib.moe_combine(FAKE, FAKE, None, ctypes.byref(d), FAKE, None, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "inv" in mod.moe_last_error()
+    # shared weights are required when S > 0
+    rc = lib.moe_expert_ffn(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, ctypes.byref(d),
+                            FAKE, FAKE, ws_n, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "Ws1" in mod.moe_last_error()
+
+
+def test_workspace_checks(mod):
+    lib = mod._lib
+    d = mod.dims(T=8, D=128, E=8, F=64, k=2)
+    ws_n = mod.moe_workspace_size(d)
+    args = [FAKE] * 9
+    rc = lib.moe_forward(*args, ctypes.byref(d), FAKE, None, None, FAKE, ws_n - 256, None)
+    assert rc == mod.MOE_ERR_WORKSPACE and "needs" in mod.moe_last_error()
+    rc = lib.moe_forward(*args, ctypes.byref(d), FAKE, None, None, None, ws_n, None)
+    assert rc == mod.MOE_ERR_WORKSPACE
+    rc = lib.moe_forward(*args, ctypes.byref(d), FAKE, None, None, FAKE + 16, ws_n, None)
+    assert rc == mod.MOE_ERR_WORKSPACE and "256-byte" in mod.moe_last_error()
+    rc = lib.moe_permute(FAKE, ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 100, None)
+    assert rc == mod.MOE_ERR_WORKSPACE
+
+
+def test_bad_dims_rejected(mod):
+    lib = mod._lib
+    for bad in (dict(T=8, D=100, E=8, F=64, k=2), dict(T=8, D=128, E=8, F=60, k=2),
+                dict(T=8, D=128, E=8, F=64, k=0), dict(T=8, D=128, E=0, F=64, k=1),
+                dict(T=8, D=128, E=8, F=64, k=2, S=1, Fs=4)):
+        d = mod.dims(**bad)
+        rc = lib.moe_forward(*([FAKE] * 9), ctypes.byref(d), FAKE, None, None, FAKE, 1 << 40, None)
+        assert rc == mod.MOE_ERR_INVALID_ARG, bad
+    d = mod.dims(T=8, D=128, E=8, F=64, k=2, scale=float("nan"))
+    rc = lib.moe_route(FAKE, FAKE, ctypes.byref(d), FAKE, FAKE, None, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "scale" in mod.moe_last_error()
+    rc = lib.moe_route(FAKE, FAKE, None, FAKE, FAKE, None, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG
+
+
+def test_binding_names_match_the_abi(mod):
+    for n in _declared_functions():
+        assert hasattr(mod, n), n

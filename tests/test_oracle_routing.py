@@ -190,3 +190,24 @@ def test_worked_examples():
         assert idx[0].tolist() == case["idx"], case["name"]
         expect = np.array(case["w"])
         assert np.all(np.abs(w[0] - expect) <= 2 * _ulp(expect)), case["name"]
+
+
+def test_routing_alternatives_cover_near_ties():
+    # keys: expert 1 and 3 tie to within 2e-7 at the boundary of a top-2
+    ln3 = F32(math.log(3.0))
+    logits = np.array([ln3, 0.0, -ln3, 0.0], F32)
+    bias = np.array([0.0, 0.0, 0.0, 2e-7], F32)
+    cands = orc.routing_alternatives(logits, bias, 2, 2.5, delta=1e-5)
+    sets = [sorted(c[0].tolist()) for c in cands]
+    assert sets[0] == [0, 3]                      # the strict selection first
+    assert sorted(sets) == [[0, 1], [0, 3]]
+    for idx, w in cands:
+        assert abs(float(w.astype(np.float64).sum()) - 2.5) < 1e-6
+    # far from any tie there is exactly one candidate, equal to route()
+    rng = np.random.default_rng(12)
+    for _ in range(20):
+        lg = rng.standard_normal(16).astype(F32)
+        b = (rng.standard_normal(16) * 0.1).astype(F32)
+        c = orc.routing_alternatives(lg, b, 4, 2.5, delta=0.0)
+        idx, w = orc.route(lg[None, :], b, 4, 2.5)
+        assert len(c) == 1 and np.array_equal(c[0][0], idx[0]) and np.array_equal(c[0][1], w[0])
