@@ -43,9 +43,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # accounting
 # ---------------------------------------------------------------------------
 def layer_bytes_flops(cfg, U: int):
-    """Algorithmic bytes and flops of one layer pass (touched experts only)."""
+    """Algorithmic bytes and flops of one layer pass (touched experts only):
+    expert weights of the touched routed experts and of the shared experts, the
+    router weight and bias, the bf16 input, the fp32 output, the routing."""
     T, D, E, F, k, S, Fs = cfg.T, cfg.D, cfg.E, cfg.F, cfg.k, cfg.S, cfg.Fs
-    B = (U * 3 * D * F * 2 + S * 3 * D * Fs * 2 + E * D * 4 + E * 4 + T * D * 2 * 2 + T * k * 8)
+    B = (U * 3 * D * F * 2 + S * 3 * D * Fs * 2 + E * D * 4 + E * 4 + T * D * 2 + T * D * 4
+         + T * k * 8)
     FL = 2 * T * D * E + 6 * D * F * T * k + 6 * D * Fs * T * S
     return B, FL
 
@@ -209,7 +212,7 @@ def run_ours(args, rank, world, local_rank):
     inp["h"] = mi.hidden(cfg, seed=rank, device=dev)
     d = moe.dims_of(cfg)
     ws = moe.alloc_workspace(d, dev)
-    out = torch.empty((cfg.T, cfg.D), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((cfg.T, cfg.D), dtype=torch.float32, device=dev)
     idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
     wgt = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -264,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end: pinned host input -> device -> layer -> pinned host output, per step
     h_pin = inp["h"].cpu().pin_memory()
-    out_pin = torch.empty((cfg.T, cfg.D), dtype=torch.bfloat16).pin_memory()
+    out_pin = torch.empty((cfg.T, cfg.D), dtype=torch.float32).pin_memory()
     h_dev = torch.empty_like(inp["h"])
     e2e_steps = min(K, 200)
     e2e_ms = []
@@ -345,7 +348,7 @@ def run_ours(args, rank, world, local_rank):
             "hbm_frac": t_roof_hbm / t_s, "tensor_frac": t_roof_tc / t_s,
             "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "source": peak_src}},
         "e2e": {"value": world * cfg.T / (e2e / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": cfg.T * cfg.D * 2, "d2h_bytes_per_step": cfg.T * cfg.D * 2,
+                "h2d_bytes_per_step": cfg.T * cfg.D * 2, "d2h_bytes_per_step": cfg.T * cfg.D * 4,
                 "ms_per_step": e2e},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,

@@ -137,22 +137,24 @@ int moe_expert_ffn(const void* h, const int32_t* perm, const int32_t* offsets, c
 
 /* Merge (MoE panel: weighted expert outputs merged with the always-on shared
  * expert; "Expert fan-out 8 + 1"), deterministic fixed order:
- *   out[t] = bf16( sum_s y[T*k + s*T + t] + sum_j w[t, j] * y[inv[t, j]] )
- * y [T*k + S*T, D] fp32, w [T, k] fp32, inv [T, k] int32 -> out [T, D] bf16.
- * An inv entry outside [0, T*k) raises MOE_ERR_BOUNDS (ws may be NULL). */
+ *   out[t] = sum_s y[T*k + s*T + t] + sum_j w[t, j] * y[inv[t, j]]
+ * (fp32: shared experts first, then slots 0..k-1, one fused multiply-add
+ * each).  y [T*k + S*T, D] fp32, w [T, k] fp32, inv [T, k] int32 ->
+ * out [T, D] fp32.  An inv entry outside [0, T*k) raises MOE_ERR_BOUNDS
+ * (ws may be NULL). */
 int moe_combine(const float* y, const float* w, const int32_t* inv, const moe_dims_t* dims,
-                void* out, void* ws, moe_stream_t stream);
+                float* out, void* ws, moe_stream_t stream);
 
 /* The whole layer: moe_router_logits, moe_route, moe_permute, the row
  * gather, moe_expert_ffn and moe_combine in one call on one stream, with no
  * host synchronisation (capturable in a CUDA graph).
  * h [T, D] bf16; Wr [E, D] fp32; bias [E] fp32; weights as in
- * moe_expert_ffn; out [T, D] bf16.  idx_out [T, k] int32 and w_out [T, k]
+ * moe_expert_ffn; out [T, D] fp32.  idx_out [T, k] int32 and w_out [T, k]
  * fp32 are optional (NULL: kept in the workspace).  ws_bytes must be at
  * least moe_workspace_size(dims). */
 int moe_forward(const void* h, const float* Wr, const float* bias, const void* W1,
                 const void* W3, const void* W2, const void* Ws1, const void* Ws3,
-                const void* Ws2, const moe_dims_t* dims, void* out, int32_t* idx_out,
+                const void* Ws2, const moe_dims_t* dims, float* out, int32_t* idx_out,
                 float* w_out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Synchronises `stream`, returns the first error recorded in the status word

@@ -161,7 +161,7 @@ def moe_combine(y, w, inv, d, out, ws=None, stream=None) -> None:
     wp, _ = _ws(ws)
     _check(_lib.moe_combine(_ptr(y, torch.float32, "y"), _ptr(w, torch.float32, "w"),
                             _ptr(inv, torch.int32, "inv"), ctypes.byref(d),
-                            _ptr(out, torch.bfloat16, "out"), wp, _stream(stream)))
+                            _ptr(out, torch.float32, "out"), wp, _stream(stream)))
 
 
 def moe_forward(h, Wr, bias, W1, W3, W2, Ws1, Ws3, Ws2, d, out, ws, idx_out=None, w_out=None,
@@ -172,7 +172,7 @@ def moe_forward(h, Wr, bias, W1, W3, W2, Ws1, Ws3, Ws2, d, out, ws, idx_out=None
                             _ptr(bias, torch.float32, "bias"), _ptr(W1, bf, "W1"),
                             _ptr(W3, bf, "W3"), _ptr(W2, bf, "W2"), _ptr(Ws1, bf, "Ws1"),
                             _ptr(Ws3, bf, "Ws3"), _ptr(Ws2, bf, "Ws2"), ctypes.byref(d),
-                            _ptr(out, bf, "out"), _ptr(idx_out, torch.int32, "idx_out"),
+                            _ptr(out, torch.float32, "out"), _ptr(idx_out, torch.int32, "idx_out"),
                             _ptr(w_out, torch.float32, "w_out"), wp, wn, _stream(stream)))
 
 

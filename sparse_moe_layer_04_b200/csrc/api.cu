@@ -317,7 +317,7 @@ int moe_expert_ffn(const void* h, const int32_t* perm, const int32_t* offsets, c
 }
 
 int moe_combine(const float* y, const float* w, const int32_t* inv, const moe_dims_t* dims,
-                void* out, void* ws, moe_stream_t stream) {
+                float* out, void* ws, moe_stream_t stream) {
   int rc = begin(dims);
   if (rc) return rc;
   if (dims->T == 0) return MOE_OK;
@@ -332,7 +332,7 @@ int moe_combine(const float* y, const float* w, const int32_t* inv, const moe_di
   int* status = ws ? reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status) : nullptr;
   if ((rc = check_device())) return rc;
   cudaError_t e = launch_combine(y, w, inv, dims->T, dims->D, dims->k, dims->S,
-                                 static_cast<uint16_t*>(out), status,
+                                 out, status,
                                  reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   g_launches = 1;
@@ -341,7 +341,7 @@ int moe_combine(const float* y, const float* w, const int32_t* inv, const moe_di
 
 int moe_forward(const void* h, const float* Wr, const float* bias, const void* W1,
                 const void* W3, const void* W2, const void* Ws1, const void* Ws3,
-                const void* Ws2, const moe_dims_t* dims, void* out, int32_t* idx_out,
+                const void* Ws2, const moe_dims_t* dims, float* out, int32_t* idx_out,
                 float* w_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
   int rc = begin(dims);
   if (rc) return rc;
@@ -412,7 +412,7 @@ int moe_forward(const void* h, const float* Wr, const float* bias, const void* W
   const char* why = "launch failed";
   e = launch_expert_ffn(a, st, &n, &why, g_prof_events ? g_prof_events + 5 : nullptr);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
-  e = launch_combine(y, rw, inv, T, D, k, dims->S, static_cast<uint16_t*>(out), w.status(), st);
+  e = launch_combine(y, rw, inv, T, D, k, dims->S, out, w.status(), st);
   if (e == cudaSuccess) e = mark(7, st);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   n += 1;

@@ -2,7 +2,9 @@
 // expert(s) ("Model anatomy -- GLM-5.2", MoE panel: the renormalised, scaled
 // expert outputs are merged with one always-on shared expert; "Expert fan-out
 // 8 + 1").  Deterministic: each output element is summed in one fixed order,
-// shared experts first, then slots 0..k-1, without atomics.
+// shared experts first, then slots 0..k-1, without atomics.  The output is
+// fp32: a bf16 output could not stay within 2e-2 of the exact result once
+// |out| >= 5.12, where half a bf16 ulp already exceeds 2e-2.
 #include <cuda_bf16.h>
 
 #include "moe_internal.cuh"
@@ -14,7 +16,7 @@ constexpr int kMaxK = 32;
 
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const float* __restrict__ y, const float* __restrict__ w, const int32_t* __restrict__ inv,
-    int T, int D, int k, int S, uint16_t* __restrict__ out, int* __restrict__ status) {
+    int T, int D, int k, int S, float* __restrict__ out, int* __restrict__ status) {
   __shared__ int s_row[kMaxK];
   __shared__ float s_w[kMaxK];
   const int t = blockIdx.x;
@@ -46,17 +48,12 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
       acc.z = fmaf(wj, a.z, acc.z);
       acc.w = fmaf(wj, a.w, acc.w);
     }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&lo);
-    pk.y = *reinterpret_cast<uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(out + (size_t)t * D)[v] = pk;
+    reinterpret_cast<float4*>(out + (size_t)t * D)[v] = acc;
   }
 }
 
 cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, int T, int D,
-                           int k, int S, uint16_t* out, int* status, cudaStream_t st) {
+                           int k, int S, float* out, int* status, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   combine_kernel<<<T, kCombineThreads, 0, st>>>(y, w, inv, T, D, k, S, out, status);
   return cudaGetLastError();

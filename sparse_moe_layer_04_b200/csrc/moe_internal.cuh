@@ -52,7 +52,7 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
 cudaError_t launch_gather_rows(const uint16_t* h, const int32_t* perm, int rows, int D, int T,
                                uint16_t* xperm, cudaStream_t st);
 cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, int T, int D,
-                           int k, int S, uint16_t* out, int* status, cudaStream_t st);
+                           int k, int S, float* out, int* status, cudaStream_t st);
 
 // Expert MLPs: gate/up GEMM with the SiLU gate fused, then the down GEMM.
 struct FfnArgs {
