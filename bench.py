@@ -208,6 +208,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     cfg = mi.CONFIGS[args.config]
+    if args.experts:
+        cfg = mi.custom_config(args.config, E=args.experts)
     inp = mi.layer_weights(cfg, 0, device=dev)
     inp["h"] = mi.hidden(cfg, seed=rank, device=dev)
     d = moe.dims_of(cfg)
@@ -419,6 +421,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=128,
                     help="tokens of the batch the CPU oracle processes per pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E (small cases for profiler captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -84,10 +84,13 @@ size_t moe_workspace_size(const moe_dims_t* dims);
 
 /* Router logits ("Routing: learned", MoE panel; fp32 router):
  *   logits[t, e] = sum_d h[t, d] * Wr[e, d]
- * h [T, D] bf16, Wr [E, D] fp32, logits [T, E] fp32 (output).  fp32 FMA
- * arithmetic; the summation order over d is fixed, so repeated calls give
- * identical bits.  `ws` (>= moe_workspace_size bytes) holds split-K partial
- * sums. */
+ * h [T, D] bf16, Wr [E, D] fp32, logits [T, E] fp32 (output).  fp32-accurate:
+ * when D % 64 == 0 and E % 8 == 0 the products run on the tensor cores
+ * against an exact three-piece bf16 split of Wr (hi + mid + lo, within 2^-24
+ * relative of Wr) with fp32 accumulation; otherwise with fp32 FMAs.  Either
+ * way the summation order is fixed, so repeated calls give identical bits.
+ * `ws` (>= moe_workspace_size bytes) holds the split weight and the partial
+ * sums; it may be NULL only when neither is needed (small FMA cases). */
 int moe_router_logits(const void* h, const float* Wr, const moe_dims_t* dims, float* logits,
                       void* ws, size_t ws_bytes, moe_stream_t stream);
 

@@ -109,6 +109,27 @@ int begin(const moe_dims_t* d) {
   return check_dims(d);
 }
 
+// Router logits into `dst` (nsplit partial planes, or the logits themselves
+// when nsplit == 1).
+cudaError_t launch_router(const uint16_t* h, const float* Wr, const moe_dims_t& d,
+                          const RouterSplit& sp, const Ws& w, float* dst, cudaStream_t st, int* n,
+                          const char** why) {
+  if (sp.tensor) {
+    uint16_t* wr3 = w.at<uint16_t>(w.L.wr3);
+    cudaError_t e = launch_split_router(Wr, d.E, d.D, wr3, st);
+    if (e != cudaSuccess) {
+      *why = "router weight split launch";
+      return e;
+    }
+    e = launch_router_tc(h, wr3, d.T, d.D, d.E, sp.nsplit, sp.chunk, dst, st, why);
+    *n += 2;
+    return e;
+  }
+  *why = "router logits launch";
+  *n += 1;
+  return launch_router_partials(h, Wr, d.T, d.D, d.E, sp, dst, st);
+}
+
 }  // namespace
 
 int num_sms() {
@@ -136,6 +157,7 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
   };
   L->status = take(256);
   L->partials = take((size_t)sp.nsplit * T * E * 4);
+  L->wr3 = take(sp.tensor ? E * 3 * D * 2 : 0);
   L->idx = take(T * k * 4);
   L->w = take(T * k * 4);
   L->counts = take(E * 4);
@@ -192,24 +214,20 @@ int moe_router_logits(const void* h, const float* Wr, const moe_dims_t* dims, fl
   MOE_CHECK_PTR(logits);
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const RouterSplit sp = router_split(dims->T, dims->D, dims->E);
-  Ws w;
-  if (sp.nsplit > 1 && (rc = check_ws(dims, ws, ws_bytes, &w))) return rc;
+  Ws w{};
+  if ((sp.nsplit > 1 || sp.tensor) && (rc = check_ws(dims, ws, ws_bytes, &w))) return rc;
   if ((rc = check_device())) return rc;
-  cudaError_t e;
-  if (sp.nsplit == 1) {
-    e = launch_router_partials(static_cast<const uint16_t*>(h), Wr, dims->T, dims->D, dims->E, sp,
-                               logits, st);
-    if (e != cudaSuccess) return cuda_fail(e, "router logits launch");
-    g_launches = 1;
-    return MOE_OK;
+  float* dst = sp.nsplit == 1 ? logits : w.at<float>(w.L.partials);
+  int n = 0;
+  const char* why = "router launch";
+  cudaError_t e = launch_router(static_cast<const uint16_t*>(h), Wr, *dims, sp, w, dst, st, &n, &why);
+  if (e != cudaSuccess) return cuda_fail(e, why);
+  if (sp.nsplit > 1) {
+    e = launch_reduce_partials(dst, sp.nsplit, (size_t)dims->T * dims->E, logits, st);
+    if (e != cudaSuccess) return cuda_fail(e, "router reduce launch");
+    n += 1;
   }
-  float* partials = w.at<float>(w.L.partials);
-  e = launch_router_partials(static_cast<const uint16_t*>(h), Wr, dims->T, dims->D, dims->E, sp,
-                             partials, st);
-  if (e != cudaSuccess) return cuda_fail(e, "router logits launch");
-  e = launch_reduce_partials(partials, sp.nsplit, (size_t)dims->T * dims->E, logits, st);
-  if (e != cudaSuccess) return cuda_fail(e, "router reduce launch");
-  g_launches = 2;
+  g_launches = n;
   return MOE_OK;
 }
 
@@ -377,14 +395,15 @@ int moe_forward(const void* h, const float* Wr, const float* bias, const void* W
 
   const RouterSplit sp = router_split(T, D, E);
   float* partials = w.at<float>(w.L.partials);
+  const char* rwhy = "router launch";
   cudaError_t e = mark(0, st);
-  if (e == cudaSuccess) e = launch_router_partials(hb, Wr, T, D, E, sp, partials, st);
+  if (e == cudaSuccess) e = launch_router(hb, Wr, *dims, sp, w, partials, st, &n, &rwhy);
   if (e == cudaSuccess) e = mark(1, st);
-  if (e != cudaSuccess) return cuda_fail(e, "router logits launch");
+  if (e != cudaSuccess) return cuda_fail(e, rwhy);
   e = launch_route(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw, w.status(), st);
   if (e == cudaSuccess) e = mark(2, st);
   if (e != cudaSuccess) return cuda_fail(e, "route launch");
-  n += 2;
+  n += 1;
   e = launch_permute(idx, T, E, k, counts, offsets, perm, inv, w.at<int32_t>(w.L.blk_base),
                      w.status(), st, &n);
   if (e == cudaSuccess) e = mark(3, st);

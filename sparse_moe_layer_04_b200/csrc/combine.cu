@@ -14,6 +14,8 @@ namespace moe {
 constexpr int kCombineThreads = 256;
 constexpr int kMaxK = 32;
 
+// Block (t, c) merges columns [c*1024, c*1024 + 1024) of token t; one float4
+// per thread, the k + S row loads issued together.
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const float* __restrict__ y, const float* __restrict__ w, const int32_t* __restrict__ inv,
     int T, int D, int k, int S, float* __restrict__ out, int* __restrict__ status) {
@@ -31,31 +33,39 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     s_w[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
   }
   __syncthreads();
-  const int nvec = D / 4;
-  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < S; ++s) {
-      const float4 a = reinterpret_cast<const float4*>(y + (rows_r + (size_t)s * T + t) * D)[v];
-      acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
-    }
-    for (int j = 0; j < k; ++j) {
-      const int r = s_row[j];
-      if (r < 0) continue;
-      const float wj = s_w[j];
-      const float4 a = reinterpret_cast<const float4*>(y + (size_t)r * D)[v];
-      acc.x = fmaf(wj, a.x, acc.x);
-      acc.y = fmaf(wj, a.y, acc.y);
-      acc.z = fmaf(wj, a.z, acc.z);
-      acc.w = fmaf(wj, a.w, acc.w);
-    }
-    reinterpret_cast<float4*>(out + (size_t)t * D)[v] = acc;
+  const int v = blockIdx.y * kCombineThreads + threadIdx.x;
+  if (v >= D / 4) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < S; ++s) {
+    const float4 a = reinterpret_cast<const float4*>(y + (rows_r + (size_t)s * T + t) * D)[v];
+    acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
   }
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    float4 a[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int r = (j0 + q < k) ? s_row[j0 + q] : -1;
+      a[q] = r >= 0 ? reinterpret_cast<const float4*>(y + (size_t)r * D)[v]
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (j0 + q >= k || s_row[j0 + q] < 0) continue;
+      const float wj = s_w[j0 + q];
+      acc.x = fmaf(wj, a[q].x, acc.x);
+      acc.y = fmaf(wj, a[q].y, acc.y);
+      acc.z = fmaf(wj, a[q].z, acc.z);
+      acc.w = fmaf(wj, a[q].w, acc.w);
+    }
+  }
+  reinterpret_cast<float4*>(out + (size_t)t * D)[v] = acc;
 }
 
 cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, int T, int D,
                            int k, int S, float* out, int* status, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  combine_kernel<<<T, kCombineThreads, 0, st>>>(y, w, inv, T, D, k, S, out, status);
+  const dim3 grid(T, (D / 4 + kCombineThreads - 1) / kCombineThreads);
+  combine_kernel<<<grid, kCombineThreads, 0, st>>>(y, w, inv, T, D, k, S, out, status);
   return cudaGetLastError();
 }
 

@@ -10,17 +10,21 @@
 //
 // Two launches:
 //   gate/up : act[r, n] = silu(sum_d A[r, d] W1[e][n, d]) * (sum_d A[r, d] W3[e][n, d])
-//             128 x 128 output tile; the W1 and W3 row blocks of the tile are
-//             stacked into one 256-row B operand, so one N = 256 MMA feeds
-//             both accumulators (TMEM columns 0-127 gate, 128-255 up) and the
+//             128 x N/2 output tile; the W1 and W3 row blocks of the tile are
+//             stacked into one N-row B operand, so one MMA feeds both
+//             accumulators (TMEM columns [0, N/2) gate, [N/2, N) up) and the
 //             epilogue applies the SiLU gate and rounds to bf16.
-//   down    : y[r, n] = sum_f act[r, f] W2[e][n, f], 128 x 256 fp32 tile.
+//   down    : y[r, n] = sum_f act[r, f] W2[e][n, f], 128 x N fp32 tile.
+// N (the MMA width) is 256 for large batches and 128 for small ones, where
+// each expert has only a row tile or two and the weight stream must be cut
+// finer to keep all 148 SMs busy.
 //
 // Kernel structure (one persistent CTA per SM, 192 threads):
-//   warp 0      TMA producer: 4-stage ring of (A 128x64, B 256x64) bf16 tiles,
-//               128-byte swizzled, completion counted on "full" mbarriers.
+//   warp 0      TMA producer: ring of (A 128x64, B Nx64) bf16 tiles (4 stages
+//               for N = 256, 6 for N = 128), 128-byte swizzled, completion
+//               counted on "full" mbarriers.
 //   warp 1      TMEM allocator and single-thread MMA issuer:
-//               tcgen05.mma.cta_group::1.kind::f16, M = 128, N = 256, K = 16,
+//               tcgen05.mma.cta_group::1.kind::f16, M = 128, N, K = 16,
 //               fp32 accumulators in TMEM, two accumulator buffers so the
 //               epilogue of tile i overlaps the main loop of tile i+1.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
@@ -39,16 +43,23 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                    // one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
 constexpr int THREADS = 192;
-constexpr int MMA_N = 256;
 constexpr int A_BYTES = BM * BK * 2;      // 16 KiB
-constexpr int B_BYTES = MMA_N * BK * 2;   // 32 KiB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int ACC_COLS = MMA_N;           // fp32 TMEM columns per accumulator
-constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
 constexpr int MAX_E = 1024;
-constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, MMA_N);
+constexpr int RING_BYTES = 192 * 1024;    // operand ring budget
+
+// Tile shape of one instantiation: MMA N = 256 (large batches) or 128 (small
+// batches, twice as many tiles to spread the weight stream over every SM).
+template <int MMA_N>
+struct Shape {
+  static constexpr int B_BYTES = MMA_N * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = RING_BYTES / STAGE_BYTES;    // 4 (N=256) or 6 (N=128)
+  static constexpr int ACC_COLS = MMA_N;                     // fp32 TMEM columns per accumulator
+  static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;        // double buffered
+  static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, MMA_N);
+};
+constexpr int MAX_STAGES = 6;
 
 struct GemmParams {
   CUtensorMap a_r;   // routed A  [rows_r, K_r]
@@ -68,12 +79,14 @@ struct GemmParams {
   int a_s_group_stride;      // rows between shared experts' A blocks (0 or T)
   int b_r_group_rows;        // B rows per routed expert (F or D)
   int b_s_group_rows;        // B rows per shared expert (Fs or D)
-  int bn_out;                // output columns per tile (128 or 256)
+  int bn_out;                // output columns per tile (MMA_N, or MMA_N / 2 for gate/up)
+  int k_chunk;               // > 0: shared group g covers K range [g*k_chunk, (g+1)*k_chunk)
+  int a_k_mod;               // > 0: the A operand's K coordinate wraps modulo this
 };
 
 struct SharedState {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t drain;
@@ -128,6 +141,19 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const SharedState& ss,
   return ti;
 }
 
+// K range of a tile: the whole reduction, or one chunk of it when the shared
+// groups split K (the router's split-K partial sums).
+__device__ __forceinline__ void tile_k_range(const TileInfo& ti, const GemmParams& p, int* kbeg,
+                                             int* K) {
+  if (ti.shared && p.k_chunk > 0) {
+    *kbeg = ti.grp * p.k_chunk;
+    *K = min(p.k_chunk, p.K_s - *kbeg);
+  } else {
+    *kbeg = 0;
+    *K = ti.shared ? p.K_s : p.K_r;
+  }
+}
+
 __device__ __forceinline__ float silu_times(float g, float u) {
   return g / (1.0f + __expf(-g)) * u;
 }
@@ -144,8 +170,16 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, volat
   if (!ptx::mbar_wait(bar, parity, &ignore_abort)) *abort = 1;
 }
 
-template <bool GATEUP>
+template <bool GATEUP, int MMA_N>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
+  using Sh = Shape<MMA_N>;
+  constexpr int STAGES = Sh::STAGES;
+  constexpr int STAGE_BYTES = Sh::STAGE_BYTES;
+  constexpr int B_BYTES = Sh::B_BYTES;
+  constexpr int ACC_COLS = Sh::ACC_COLS;
+  constexpr uint32_t TMEM_COLS = Sh::TMEM_COLS;
+  constexpr uint32_t IDESC = Sh::IDESC;
+  constexpr int HALF = MMA_N / 2;  // gate/up: W1 rows [0, HALF), W3 rows [HALF, MMA_N)
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned operand ring (128-byte swizzle atoms span 1024 bytes)
   const uint32_t raw_addr = ptx::smem_addr(smem_raw);
@@ -232,20 +266,23 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         const CUtensorMap* b1 = ti.shared ? &p.b1_s : &p.b1_r;
         const int a_row = ti.shared ? ti.grp * p.a_s_group_stride + ti.m0 : ti.row0 + ti.m0;
         const int b_row = ti.grp * (ti.shared ? p.b_s_group_rows : p.b_r_group_rows) + ti.n0;
-        const int K = ti.shared ? p.K_s : p.K_r;
+        int kbeg, K;
+        tile_k_range(ti, p, &kbeg, &K);
         const int nk = (K + BK - 1) / BK;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
           if (!ptx::mbar_wait(&ss.empty[stage], phase ^ 1u, abort)) { ok = false; break; }
           uint8_t* sa = ring + stage * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
+          const int xb = kbeg + kb * BK;
+          const int xa = p.a_k_mod > 0 ? xb % p.a_k_mod : xb;
           ptx::mbar_arrive_expect_tx(&ss.full[stage], STAGE_BYTES);
-          ptx::tma_load_2d(sa, amap, &ss.full[stage], kb * BK, a_row);
+          ptx::tma_load_2d(sa, amap, &ss.full[stage], xa, a_row);
           if (GATEUP) {
-            ptx::tma_load_2d(sb, b0, &ss.full[stage], kb * BK, b_row);
-            ptx::tma_load_2d(sb + B_BYTES / 2, b1, &ss.full[stage], kb * BK, b_row);
+            ptx::tma_load_2d(sb, b0, &ss.full[stage], xb, b_row);
+            ptx::tma_load_2d(sb + HALF * BK * 2, b1, &ss.full[stage], xb, b_row);
           } else {
-            ptx::tma_load_2d(sb, b0, &ss.full[stage], kb * BK, b_row);
+            ptx::tma_load_2d(sb, b0, &ss.full[stage], xb, b_row);
           }
           issued_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -266,7 +303,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       uint32_t acc_phase = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
         const TileInfo ti = decode_tile(tile, ss, p);
-        const int K = ti.shared ? p.K_s : p.K_r;
+        int kbeg, K;
+        tile_k_range(ti, p, &kbeg, &K);
         const int nk = (K + BK - 1) / BK;
         if (!ptx::mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1u, abort)) break;
         ptx::tc_fence_after();
@@ -310,10 +348,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       if (GATEUP) {
         uint16_t* out = static_cast<uint16_t*>(ti.shared ? p.out_s : p.out_r);
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 16) {
+        for (int c = 0; c < HALF; c += 16) {
           uint32_t g[16], u[16];
           ptx::tmem_ld_x16(taddr + c, g);
-          ptx::tmem_ld_x16(taddr + 128 + c, u);
+          ptx::tmem_ld_x16(taddr + HALF + c, u);
           ptx::tmem_wait_ld();
           const int col = ti.n0 + c;
           if (row_ok && col < N) {
@@ -331,7 +369,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       } else {
         float* out = static_cast<float*>(ti.shared ? p.out_s : p.out_r);
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 16) {
+        for (int c = 0; c < MMA_N; c += 16) {
           uint32_t v[16];
           ptx::tmem_ld_x16(taddr + c, v);
           ptx::tmem_wait_ld();
@@ -398,45 +436,96 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(SharedState);
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+template <int MMA_N>
+constexpr size_t smem_bytes() {
+  return 1024 + Shape<MMA_N>::STAGES * Shape<MMA_N>::STAGE_BYTES + sizeof(SharedState);
+}
+static_assert(smem_bytes<256>() <= 227 * 1024 && smem_bytes<128>() <= 227 * 1024,
+              "shared memory budget");
 
-template <bool GATEUP>
+template <bool GATEUP, int MMA_N>
 cudaError_t launch_one(const GemmParams& p, int tiles_upper, cudaStream_t st) {
   static int configured_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP, MMA_N>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+                                         (int)smem_bytes<MMA_N>());
     if (e != cudaSuccess) return e;
     configured_dev = dev;
   }
   int grid = num_sms();
   if (tiles_upper < grid) grid = tiles_upper;
   if (grid < 1) grid = 1;
-  grouped_gemm_kernel<GATEUP><<<grid, THREADS, kSmemBytes, st>>>(p);
+  grouped_gemm_kernel<GATEUP, MMA_N><<<grid, THREADS, smem_bytes<MMA_N>(), st>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+// Router logits on the tensor cores.  The fp32 router weight is split exactly
+// into three bf16 pieces (hi + mid + lo, each the bf16 rounding of what the
+// previous pieces leave; together they carry the 24-bit fp32 significand),
+// stored side by side as wr3 [E, 3D].  h is bf16 and so exact in the MMA, so
+//   logits = [h | h | h] . wr3^T
+// is a dense GEMM over K' = 3D with fp32 accumulation.  It runs on the
+// grouped kernel as `nsplit` shared groups that each take one K' chunk and
+// write their own partial-sum plane [T, E]; the consumer adds the planes in
+// order.
+cudaError_t launch_router_tc(const uint16_t* h, const uint16_t* wr3, int T, int D, int E,
+                             int nsplit, int chunk, float* partials, cudaStream_t st,
+                             const char** why) {
+  const int bn = router_tile_n(T, E);
+  const bool narrow = bn == 128;
+  GemmParams p{};
+  if (!make_map(&p.a_s, h, T, D, BM) || !make_map(&p.b0_s, wr3, E, 3ull * D, bn)) {
+    *why = "cuTensorMapEncodeTiled failed for a router operand";
+    return cudaErrorInvalidValue;
+  }
+  p.a_r = p.a_s;
+  p.b0_r = p.b1_r = p.b1_s = p.b0_s;
+  p.offsets = nullptr;
+  p.out_r = nullptr;
+  p.out_s = partials;
+  p.status = nullptr;
+  p.E = 0; p.S = nsplit; p.T = T;
+  p.K_r = 0; p.K_s = 3 * D;
+  p.N_r = 0; p.N_s = E;
+  p.rows_r = 0;
+  p.a_s_group_stride = 0;
+  p.b_r_group_rows = 0;
+  p.b_s_group_rows = 0;
+  p.bn_out = bn;
+  p.k_chunk = chunk;
+  p.a_k_mod = D;
+  const int tiles = nsplit * ((T + BM - 1) / BM) * ((E + bn - 1) / bn);
+  return narrow ? launch_one<false, 128>(p, tiles, st) : launch_one<false, 256>(p, tiles, st);
+}
+
+// Small batches (T <= 512) leave each expert with at most a few row tiles, so
+// the weight stream is the whole cost: 128-wide tiles double the tile count
+// and keep every SM streaming.  Larger batches use 256-wide tiles.
+bool use_narrow_tiles(int T) { return T <= 512; }
 
 cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, const char** why,
                               void* const* marks) {
   const int rows_r = a.T * a.k;
   const int mt_upper = (rows_r + BM - 1) / BM + a.E;  // sum over experts of ceil(count/BM)
   const int mt_s = (a.T + BM - 1) / BM;
+  const bool narrow = use_narrow_tiles(a.T);
+  const int nmma = narrow ? 128 : 256;
+  const int half = nmma / 2;
 
   // ---- gate/up ----
   GemmParams g{};
   bool ok = make_map(&g.a_r, a.xperm, rows_r, a.D, BM) &&
-            make_map(&g.b0_r, a.W1, (uint64_t)a.E * a.F, a.D, 128) &&
-            make_map(&g.b1_r, a.W3, (uint64_t)a.E * a.F, a.D, 128);
+            make_map(&g.b0_r, a.W1, (uint64_t)a.E * a.F, a.D, half) &&
+            make_map(&g.b1_r, a.W3, (uint64_t)a.E * a.F, a.D, half);
   if (ok && a.S > 0)
     ok = make_map(&g.a_s, a.h, a.T, a.D, BM) &&
-         make_map(&g.b0_s, a.Ws1, (uint64_t)a.S * a.Fs, a.D, 128) &&
-         make_map(&g.b1_s, a.Ws3, (uint64_t)a.S * a.Fs, a.D, 128);
+         make_map(&g.b0_s, a.Ws1, (uint64_t)a.S * a.Fs, a.D, half) &&
+         make_map(&g.b1_s, a.Ws3, (uint64_t)a.S * a.Fs, a.D, half);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed for a gate/up operand";
     return cudaErrorInvalidValue;
@@ -452,19 +541,20 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, c
   g.a_s_group_stride = 0;
   g.b_r_group_rows = a.F;
   g.b_s_group_rows = a.Fs;
-  g.bn_out = 128;
-  const int tiles_g = mt_upper * ((a.F + 127) / 128) + a.S * mt_s * ((a.Fs + 127) / 128);
-  cudaError_t err = launch_one<true>(g, tiles_g, st);
+  g.bn_out = half;
+  const int tiles_g = mt_upper * ((a.F + half - 1) / half) + a.S * mt_s * ((a.Fs + half - 1) / half);
+  cudaError_t err = narrow ? launch_one<true, 128>(g, tiles_g, st)
+                           : launch_one<true, 256>(g, tiles_g, st);
   if (err == cudaSuccess && marks) err = cudaEventRecord(static_cast<cudaEvent_t>(marks[0]), st);
   if (err != cudaSuccess) return err;
 
   // ---- down ----
   GemmParams d{};
   ok = make_map(&d.a_r, a.act_r, rows_r, a.F, BM) &&
-       make_map(&d.b0_r, a.W2, (uint64_t)a.E * a.D, a.F, 256);
+       make_map(&d.b0_r, a.W2, (uint64_t)a.E * a.D, a.F, nmma);
   if (ok && a.S > 0)
     ok = make_map(&d.a_s, a.act_s, (uint64_t)a.S * a.T, a.Fs, BM) &&
-         make_map(&d.b0_s, a.Ws2, (uint64_t)a.S * a.D, a.Fs, 256);
+         make_map(&d.b0_s, a.Ws2, (uint64_t)a.S * a.D, a.Fs, nmma);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed for a down-projection operand";
     return cudaErrorInvalidValue;
@@ -482,10 +572,10 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, c
   d.a_s_group_stride = a.T;
   d.b_r_group_rows = a.D;
   d.b_s_group_rows = a.D;
-  d.bn_out = 256;
-  const int nt_d = (a.D + 255) / 256;
+  d.bn_out = nmma;
+  const int nt_d = (a.D + nmma - 1) / nmma;
   const int tiles_d = mt_upper * nt_d + a.S * mt_s * nt_d;
-  err = launch_one<false>(d, tiles_d, st);
+  err = narrow ? launch_one<false, 128>(d, tiles_d, st) : launch_one<false, 256>(d, tiles_d, st);
   if (err == cudaSuccess && marks) err = cudaEventRecord(static_cast<cudaEvent_t>(marks[1]), st);
   *nlaunch += 2;
   return err;

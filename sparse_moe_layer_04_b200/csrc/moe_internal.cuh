@@ -14,34 +14,44 @@ constexpr int kStNonFinite = 1;
 constexpr int kStBounds = 2;
 constexpr int kStTimeout = 4;
 
-// Device count assumed when splitting small problems; the split depends on the
-// shape only, so results are bit-identical on every device.
-constexpr int kSplitTargetBlocks = 296;
+// Block count a small problem is split into (one wave on the 148 SMs of a
+// B200); the split depends on the shape only, so results are bit-identical
+// on every device.
+constexpr int kSplitTargetBlocks = 148;
 
 // Router logits tiling (fp32 FMA, split over D).
 constexpr int kRouterTileT = 64;
 constexpr int kRouterTileE = 64;
 constexpr int kRouterTileD = 32;
 
+// How the router logits are computed: on the tensor cores (three-way bf16
+// split of the router weight, needs D % 64 == 0 and E % 8 == 0) or with fp32
+// FMAs; both produce `nsplit` partial-sum planes [T, E] added in order.
 struct RouterSplit {
-  int nsplit;  // partial sums over D
-  int chunk;   // D-range of one split (multiple of kRouterTileD)
+  bool tensor;  // tensor-core path
+  int nsplit;   // partial-sum planes
+  int chunk;    // reduction range of one plane (over D for FMA, over 3D for tensor)
 };
 RouterSplit router_split(int T, int D, int E);
+int router_tile_n(int T, int E);  // MMA N of the tensor-core router
 
 // Permute: tokens per counting block.
 constexpr int kPermBlockTokens = 256;
 
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
 struct WsLayout {
-  size_t status, partials, idx, w, counts, offsets, perm, inv, blk_base, xperm, act_r, act_s,
-      y, total;
+  size_t status, partials, wr3, idx, w, counts, offsets, perm, inv, blk_base, xperm, act_r,
+      act_s, y, total;
 };
 bool ws_layout(const moe_dims_t& d, WsLayout* out);
 
 // --- launchers (return cudaSuccess or the launch error) ---------------------
 cudaError_t launch_router_partials(const uint16_t* h, const float* Wr, int T, int D, int E,
                                    RouterSplit sp, float* out, cudaStream_t st);
+cudaError_t launch_split_router(const float* Wr, int E, int D, uint16_t* wr3, cudaStream_t st);
+cudaError_t launch_router_tc(const uint16_t* h, const uint16_t* wr3, int T, int D, int E,
+                             int nsplit, int chunk, float* partials, cudaStream_t st,
+                             const char** why);
 cudaError_t launch_reduce_partials(const float* partials, int nsplit, size_t n, float* out,
                                    cudaStream_t st);
 cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T, int E, int k,

@@ -11,7 +11,8 @@
 //             (tokens pick distinct experts, so one bit per token suffices):
 //             row = base[block][e] + rank.  Rows within an expert therefore
 //             follow increasing token order, i.e. (token, slot) order.
-// All integer work: exact and deterministic.
+// Batches of at most 256 tokens (one counting block) run all three phases in
+// one launch.  All integer work: exact and deterministic.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -124,10 +125,86 @@ __global__ void __launch_bounds__(kPermBlockTokens) permute_scatter_kernel(
   if (bad && status) atomicOr(status, kStBounds);
 }
 
+// All three phases for T <= 256 in one block of 256 threads.
+__global__ void __launch_bounds__(kPermBlockTokens) permute_single_block_kernel(
+    const int32_t* __restrict__ idx, int T, int E, int k, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+    int* __restrict__ status) {
+  extern __shared__ int sm[];
+  int* cnt = sm;                                          // [E]
+  unsigned* mask = reinterpret_cast<unsigned*>(sm + E);   // [E][kWordsPerBlock]
+  __shared__ int warp_tot[kPermBlockTokens / 32];
+  for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
+  for (int i = threadIdx.x; i < E * kWordsPerBlock; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  const int t = threadIdx.x;
+  const int word = t >> 5;
+  const unsigned bit = 1u << (t & 31);
+  bool bad = false;
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      if (e < 0 || e >= E) {
+        bad = true;
+        continue;
+      }
+      atomicAdd(&cnt[e], 1);
+      const unsigned old = atomicOr(&mask[e * kWordsPerBlock + word], bit);
+      if (old & bit) bad = true;
+    }
+  }
+  __syncthreads();
+  // exclusive scan of cnt over experts: thread i owns experts [i*per, (i+1)*per)
+  const int per = (E + kPermBlockTokens - 1) / kPermBlockTokens;
+  const int e0 = threadIdx.x * per;
+  int local = 0;
+  for (int e = e0; e < e0 + per && e < E; ++e) local += cnt[e];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_tot[wid] = incl;
+  __syncthreads();
+  int base = incl - local;
+  for (int q = 0; q < wid; ++q) base += warp_tot[q];
+  __syncthreads();  // everyone has read warp_tot; cnt becomes the offsets
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    const int c = cnt[e];
+    counts[e] = c;
+    offsets[e] = base;
+    cnt[e] = base;
+    base += c;
+  }
+  if (threadIdx.x == kPermBlockTokens - 1) offsets[E] = base;  // the last thread ends at the total
+  __syncthreads();
+  if (t < T && !bad) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      const unsigned* m = mask + e * kWordsPerBlock;
+      int rank = __popc(m[word] & (bit - 1u));
+      for (int q = 0; q < word; ++q) rank += __popc(m[q]);
+      const int row = cnt[e] + rank;
+      perm[row] = t;
+      inv[(size_t)t * k + j] = row;
+    }
+  }
+  if (bad && status) atomicOr(status, kStBounds);
+}
+
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* blk_base,
                            int* status, cudaStream_t st, int* nlaunch) {
   const int nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+  if (nblk == 1) {
+    const size_t smem = (size_t)E * sizeof(int) + (size_t)E * kWordsPerBlock * sizeof(unsigned);
+    permute_single_block_kernel<<<1, kPermBlockTokens, smem, st>>>(idx, T, E, k, counts, offsets,
+                                                                   perm, inv, status);
+    *nlaunch += 1;
+    return cudaGetLastError();
+  }
   permute_count_kernel<<<nblk, kPermBlockTokens, E * sizeof(int), st>>>(idx, T, E, k, blk_base,
                                                                          status);
   cudaError_t err = cudaGetLastError();

@@ -20,17 +20,78 @@
 
 namespace moe {
 
+int router_tile_n(int T, int E) { return (E <= 128 || T <= 512) ? 128 : 256; }
+
 RouterSplit router_split(int T, int D, int E) {
+  RouterSplit sp;
+  if (D % 64 == 0 && E % 8 == 0) {
+    // tensor path: enough (row tile, column tile, K' chunk) work units for
+    // about one wave; at most 64 planes
+    const int kblocks = 3 * D / 64;
+    const int bn = router_tile_n(T, E);
+    const int tiles = ((T + 127) / 128) * ((E + bn - 1) / bn);
+    int want = (kSplitTargetBlocks + tiles - 1) / (tiles > 0 ? tiles : 1);
+    want = want < 1 ? 1 : (want > 64 ? 64 : want);
+    const int kb_per = (kblocks + want - 1) / want;
+    sp.tensor = true;
+    sp.chunk = kb_per * 64;
+    sp.nsplit = (kblocks + kb_per - 1) / kb_per;
+    return sp;
+  }
   const int tiles = ((T + kRouterTileT - 1) / kRouterTileT) * ((E + kRouterTileE - 1) / kRouterTileE);
   int want = (kSplitTargetBlocks + tiles - 1) / (tiles > 0 ? tiles : 1);
   if (want < 1) want = 1;
   if (want > 32) want = 32;
   int chunk = (D + want - 1) / want;
   chunk = (chunk + kRouterTileD - 1) / kRouterTileD * kRouterTileD;
-  RouterSplit sp;
+  sp.tensor = false;
   sp.chunk = chunk;
   sp.nsplit = (D + chunk - 1) / chunk;
   return sp;
+}
+
+// wr3[e] = [hi | mid | lo] with hi = bf16(w), mid = bf16(w - hi),
+// lo = bf16(w - hi - mid); both subtractions are exact (Sterbenz), and each
+// bf16 rounding leaves at most 2^-8 of what it rounds, so
+// |w - (hi + mid + lo)| <= 2^-24 |w|: the fp32 value to within its own
+// rounding.
+__global__ void split_router_kernel(const float* __restrict__ Wr, int E, int D,
+                                    uint16_t* __restrict__ wr3) {
+  const size_t n4 = (size_t)E * D / 4;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float4 w = reinterpret_cast<const float4*>(Wr)[i];
+    const size_t flat = i * 4;
+    const size_t e = flat / D, d = flat % D;
+    const float wv[4] = {w.x, w.y, w.z, w.w};
+    uint16_t hi[4], mid[4], lo[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat16 bh = __float2bfloat16_rn(wv[q]);
+      const float r1 = __fsub_rn(wv[q], __bfloat162float(bh));
+      const __nv_bfloat16 bm = __float2bfloat16_rn(r1);
+      const float r2 = __fsub_rn(r1, __bfloat162float(bm));
+      const __nv_bfloat16 bl = __float2bfloat16_rn(r2);
+      hi[q] = __bfloat16_as_ushort(bh);
+      mid[q] = __bfloat16_as_ushort(bm);
+      lo[q] = __bfloat16_as_ushort(bl);
+    }
+    uint16_t* row = wr3 + e * 3 * (size_t)D;
+    *reinterpret_cast<uint2*>(row + d) =
+        make_uint2(hi[0] | ((uint32_t)hi[1] << 16), hi[2] | ((uint32_t)hi[3] << 16));
+    *reinterpret_cast<uint2*>(row + D + d) =
+        make_uint2(mid[0] | ((uint32_t)mid[1] << 16), mid[2] | ((uint32_t)mid[3] << 16));
+    *reinterpret_cast<uint2*>(row + 2 * (size_t)D + d) =
+        make_uint2(lo[0] | ((uint32_t)lo[1] << 16), lo[2] | ((uint32_t)lo[3] << 16));
+  }
+}
+
+cudaError_t launch_split_router(const float* Wr, int E, int D, uint16_t* wr3, cudaStream_t st) {
+  const size_t n4 = (size_t)E * D / 4;
+  size_t blocks = (n4 + 255) / 256;
+  if (blocks > 2048) blocks = 2048;
+  split_router_kernel<<<(unsigned)blocks, 256, 0, st>>>(Wr, E, D, wr3);
+  return cudaGetLastError();
 }
 
 // out[s][t][e] = sum over d in split s of h[t, d] * Wr[e, d], d ascending.
@@ -57,41 +118,37 @@ __global__ void __launch_bounds__(256) router_partials_kernel(const uint16_t* __
 
   const int lrow = tid >> 2;          // 0..63: token (h tile) / expert (Wr tile)
   const int lcol = (tid & 3) * 8;     // 0, 8, 16, 24 within the 32-wide d slice
+  const int t_ld = t0 + lrow, e_ld = e0 + lrow;
+  uint4 hraw = make_uint4(0, 0, 0, 0);
+  float4 wa = make_float4(0.f, 0.f, 0.f, 0.f), wb = wa;
+  // global -> registers for the slice at d0 (zeros outside the tensor)
+  auto fetch = [&](int d0) {
+    const int d = d0 + lcol;
+    hraw = make_uint4(0, 0, 0, 0);
+    wa = wb = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (d < dend) {
+      if (t_ld < T) hraw = *reinterpret_cast<const uint4*>(h + (size_t)t_ld * D + d);
+      if (e_ld < E) {
+        wa = *reinterpret_cast<const float4*>(Wr + (size_t)e_ld * D + d);
+        wb = *reinterpret_cast<const float4*>(Wr + (size_t)e_ld * D + d + 4);
+      }
+    }
+  };
+  if (dbeg < dend) fetch(dbeg);
   for (int d0 = dbeg; d0 < dend; d0 += kRouterTileD) {
     {
-      const int t = t0 + lrow, d = d0 + lcol;
-      float v[8];
-      if (t < T && d < dend) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(h + (size_t)t * D + d);
-        const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+      const uint32_t u[4] = {hraw.x, hraw.y, hraw.z, hraw.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v[2 * i] = __uint_as_float(u[i] << 16);
-          v[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      for (int i = 0; i < 4; ++i) {
+        hs[lcol + 2 * i][lrow] = __uint_as_float(u[i] << 16);
+        hs[lcol + 2 * i + 1][lrow] = __uint_as_float(u[i] & 0xFFFF0000u);
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) hs[lcol + i][lrow] = v[i];
-    }
-    {
-      const int e = e0 + lrow, d = d0 + lcol;
-      float v[8];
-      if (e < E && d < dend) {
-        const float4 a = *reinterpret_cast<const float4*>(Wr + (size_t)e * D + d);
-        const float4 b = *reinterpret_cast<const float4*>(Wr + (size_t)e * D + d + 4);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.f;
-      }
+      const float v[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
       for (int i = 0; i < 8; ++i) wsm[lcol + i][lrow] = v[i];
     }
     __syncthreads();
+    if (d0 + kRouterTileD < dend) fetch(d0 + kRouterTileD);  // in flight during the FMAs
 #pragma unroll 8
     for (int kk = 0; kk < kRouterTileD; ++kk) {
       const float4 a = *reinterpret_cast<const float4*>(&hs[kk][ty * 4]);
@@ -147,76 +204,105 @@ cudaError_t launch_reduce_partials(const float* partials, int nsplit, size_t n, 
 }
 
 // ---------------------------------------------------------------------------
-// routing
+// routing: one block per token, one thread per expert
 // ---------------------------------------------------------------------------
-constexpr int kRouteWarps = 4;
-
 // (key, expert) pair a precedes b under (key descending, index ascending).
 __device__ __forceinline__ bool precedes(float ka, int ea, float kb, int eb) {
   return ka > kb || (ka == kb && ea < eb);
 }
 
-template <int EPL>
-__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(
+// Arg-max of (key, index) pairs across a warp; every lane gets the winner.
+__device__ __forceinline__ void warp_best(float& bk, int& be, float& bs) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+    const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+    if (precedes(ok, oe, bk, be)) {
+      bk = ok;
+      be = oe;
+      bs = os;
+    }
+  }
+}
+
+constexpr int kMaxSlots = 32;
+
+// Thread e sums expert e's partial-sum planes in plane order, takes the
+// sigmoid in fp64 (rounded once to fp32) and adds the bias.  Each warp then
+// extracts its k best (key, index) pairs by warp arg-max rounds; the union
+// of the warps' lists holds the token's top k, which warp 0 extracts the same
+// way, in selection order.  The weights use the un-biased scores.
+__global__ void __launch_bounds__(1024) route_kernel(
     const float* __restrict__ src, int nsplit, const float* __restrict__ bias, int T, int E,
     int k, float scale, int32_t* __restrict__ idx, float* __restrict__ w,
     int* __restrict__ status) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
-  if (t >= T) return;
+  __shared__ float c_key[kMaxSlots * kMaxSlots];
+  __shared__ float c_sc[kMaxSlots * kMaxSlots];
+  __shared__ int c_e[kMaxSlots * kMaxSlots];
+  const int t = blockIdx.x;
+  const int e = threadIdx.x;
+  const int lane = e & 31, wid = e >> 5, nw = blockDim.x >> 5;
   const size_t plane = (size_t)T * E;
+  int bad = 0;
 
-  float key[EPL], sc[EPL];
-  bool bad = false;
+  float key = -INFINITY, sc = 0.f;
+  int me = INT_MAX;
+  if (e < E) {
+    const float* p = src + (size_t)t * E + e;
+    float l = p[0];
+    for (int s0 = 1; s0 < nsplit; s0 += 16) {
+      float v[16];
 #pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E) {
-      float l = src[(size_t)t * E + e];
-      for (int s = 1; s < nsplit; ++s) l = __fadd_rn(l, src[s * plane + (size_t)t * E + e]);
-      // sigmoid in fp64 from the fp32 logit, rounded once to fp32
-      const double sd = 1.0 / (1.0 + exp(-(double)l));
-      sc[i] = __double2float_rn(sd);
-      key[i] = __fadd_rn(sc[i], bias[e]);
-      if (!isfinite(l) || !isfinite(key[i])) bad = true;
-    } else {
-      sc[i] = 0.f;
-      key[i] = -FLT_MAX;
+      for (int q = 0; q < 16; ++q) v[q] = (s0 + q < nsplit) ? p[(s0 + q) * plane] : 0.f;
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (s0 + q < nsplit) l = __fadd_rn(l, v[q]);
     }
-  }
-  if (__any_sync(0xffffffffu, bad)) {
-    if (lane == 0 && status) atomicOr(status, kStNonFinite);
+    const double sd = 1.0 / (1.0 + exp(-(double)l));
+    sc = __double2float_rn(sd);
+    key = __fadd_rn(sc, bias[e]);
+    me = e;
+    bad = !isfinite(l) || !isfinite(key);
   }
 
-  unsigned taken = 0u;          // bit i: expert lane + 32 i already selected
-  int my_e = 0;                 // slot `lane`'s expert (lanes < k)
-  float my_s = 0.f;             // and its un-biased score
-  float sum = 0.f;
+  // per-warp top-k candidates
+  bool taken = false;
   for (int j = 0; j < k; ++j) {
-    float bk = -INFINITY;
-    int be = INT_MAX;
-    float bs = 0.f;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !(taken & (1u << i)) && precedes(key[i], e, bk, be)) {
-        bk = key[i];
-        be = e;
-        bs = sc[i];
+    float bk = taken ? -INFINITY : key;
+    int be = taken ? INT_MAX : me;
+    float bs = sc;
+    warp_best(bk, be, bs);
+    if (lane == 0) {
+      c_key[wid * k + j] = bk;
+      c_e[wid * k + j] = be;
+      c_sc[wid * k + j] = bs;
+    }
+    if (be == me) taken = true;
+  }
+  if (__syncthreads_or(bad) && e == 0 && status) atomicOr(status, kStNonFinite);
+  if (wid != 0) return;
+
+  // warp 0: the token's top k among the nw * k candidates
+  const int nc = nw * k;
+  unsigned done = 0u;  // bit q: candidate lane + 32 q already selected
+  int my_e = 0;
+  float my_s = 0.f, sum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float bk = -INFINITY, bs = 0.f;
+    int be = INT_MAX, bq = -1;
+    for (int q = 0, c = lane; c < nc; ++q, c += 32) {
+      if ((done >> q) & 1u) continue;
+      if (c_e[c] != INT_MAX && precedes(c_key[c], c_e[c], bk, be)) {
+        bk = c_key[c];
+        be = c_e[c];
+        bs = c_sc[c];
+        bq = q;
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-      if (precedes(ok, oe, bk, be)) {
-        bk = ok;
-        be = oe;
-        bs = os;
-      }
-    }
-    if (be != INT_MAX && (be & 31) == lane) taken |= 1u << (be >> 5);
+    const int mine = be;
+    warp_best(bk, be, bs);
+    if (bq >= 0 && mine == be) done |= 1u << bq;
     if (lane == j) {
       my_e = be;
       my_s = bs;
@@ -231,21 +317,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(
 
 cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T, int E, int k,
                          float scale, int32_t* idx, float* w, int* status, cudaStream_t st) {
-  const dim3 grid((T + kRouteWarps - 1) / kRouteWarps);
-  const dim3 block(kRouteWarps * 32);
-  const int epl = (E + 31) / 32;
-  if (epl <= 1)
-    route_kernel<1><<<grid, block, 0, st>>>(src, nsplit, bias, T, E, k, scale, idx, w, status);
-  else if (epl <= 2)
-    route_kernel<2><<<grid, block, 0, st>>>(src, nsplit, bias, T, E, k, scale, idx, w, status);
-  else if (epl <= 4)
-    route_kernel<4><<<grid, block, 0, st>>>(src, nsplit, bias, T, E, k, scale, idx, w, status);
-  else if (epl <= 8)
-    route_kernel<8><<<grid, block, 0, st>>>(src, nsplit, bias, T, E, k, scale, idx, w, status);
-  else if (epl <= 16)
-    route_kernel<16><<<grid, block, 0, st>>>(src, nsplit, bias, T, E, k, scale, idx, w, status);
-  else
-    route_kernel<32><<<grid, block, 0, st>>>(src, nsplit, bias, T, E, k, scale, idx, w, status);
+  const int threads = (E + 31) / 32 * 32;
+  route_kernel<<<T, threads, 0, st>>>(src, nsplit, bias, T, E, k, scale, idx, w, status);
   return cudaGetLastError();
 }
 

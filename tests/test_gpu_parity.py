@@ -88,10 +88,19 @@ def test_router_logits(moe, T, D, E):
     assert torch.equal(out, out2)
     hf, wf = h.float().numpy().astype(np.float64), Wr.numpy().astype(np.float64)
     ref = orc.router_logits(hf, wf).astype(np.float64)
-    # fp32 FMA summation error bound: (D + splits) * 2^-24 * sum_d |h w|, plus
-    # the final rounding of the reference itself
-    bound = (D + 33) * 2.0 ** -24 * (np.abs(hf) @ np.abs(wf).T) + np.abs(ref) * 2.0 ** -24
-    assert np.all(np.abs(out.cpu().numpy() - ref) <= bound)
+    mag = np.abs(hf) @ np.abs(wf).T
+    err = np.abs(out.cpu().numpy() - ref)
+    if D % 64 == 0 and E % 8 == 0:
+        # tensor path: 3D exact bf16 products (the split of Wr is within 2^-24)
+        # summed in fp32 inside the tensor core; allow a full ulp per add
+        bound = (3 * D + 64) * 2.0 ** -23 * mag + np.abs(ref) * 2.0 ** -24
+    else:
+        # fp32 FMA chain: (D + splits) * 2^-24 * sum_d |h w|
+        bound = (D + 33) * 2.0 ** -24 * mag + np.abs(ref) * 2.0 ** -24
+    assert np.all(err <= bound)
+    # typical error stays at fp32 level (a dropped middle piece of the split
+    # would leave ~2^-9 relative errors)
+    assert np.sqrt(np.mean(err ** 2)) <= 1e-5 * np.sqrt(np.mean(ref ** 2)) + 1e-9
 
 
 # ---------------------------------------------------------------------------
