@@ -122,6 +122,30 @@ int moe_route(const float* logits, const float* bias, const moe_dims_t* dims, in
 int moe_permute(const int32_t* idx, const moe_dims_t* dims, int32_t* counts, int32_t* offsets,
                 int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_permute for callers that cannot allocate device memory: the same
+ * grouping, bit for bit, with its scratch in a fixed array inside the library
+ * instead of a caller workspace.  There is no counterpart on the pages; it
+ * exists for callers that must not call cudaMalloc, for example code that
+ * runs while another component owns all device memory through a fixed pool,
+ * or a serving loop that may not take the device-wide synchronisation an
+ * allocation implies, and that therefore cannot provide a workspace.
+ *  - Limits: T <= 16384 (64 counting blocks of 256 tokens) and E <= 1024;
+ *    larger sizes return MOE_ERR_UNSUPPORTED and enqueue nothing.  The
+ *    array (256 KiB) is held by every GPU that loads the library until the
+ *    process exits.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array and leaves the last call's contents in
+ *    it; each call overwrites every entry it reads, so nothing needs
+ *    clearing.  Calls whose work overlaps on the GPU (different streams, or
+ *    different host threads) race on the array and give wrong groupings.
+ *  - Device-detected errors (an expert index out of range or repeated) are
+ *    not recorded: there is no workspace to hold a status word. */
+int moe_permute_noalloc(const int32_t* idx, const moe_dims_t* dims, int32_t* counts,
+                        int32_t* offsets, int32_t* perm, int32_t* inv, moe_stream_t stream);
+
 /* Expert MLPs on grouped rows (gated MLP with w1/w3 -> SiLU gate -> w2):
  *   routed row r (expert e, offsets[e] <= r < offsets[e+1], token perm[r]):
  *     y[r] = W2[e] (silu(W1[e] h[perm[r]]) * (W3[e] h[perm[r]]))

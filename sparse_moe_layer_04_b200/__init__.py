@@ -66,6 +66,7 @@ def _load() -> ctypes.CDLL:
         "moe_router_logits": (I, [P, P, D, P, P, Z, P]),
         "moe_route": (I, [P, P, D, P, P, P, P]),
         "moe_permute": (I, [P, D, P, P, P, P, P, Z, P]),
+        "moe_permute_noalloc": (I, [P, D, P, P, P, P, P]),
         "moe_expert_ffn": (I, [P, P, P, P, P, P, P, P, P, D, P, P, Z, P]),
         "moe_combine": (I, [P, P, P, D, P, P, P]),
         "moe_forward": (I, [P, P, P, P, P, P, P, P, P, D, P, P, P, P, Z, P]),
@@ -145,6 +146,15 @@ def moe_permute(idx, d, counts, offsets, perm, inv, ws, stream=None) -> None:
                             _ptr(counts, torch.int32, "counts"),
                             _ptr(offsets, torch.int32, "offsets"), _ptr(perm, torch.int32, "perm"),
                             _ptr(inv, torch.int32, "inv"), wp, wn, _stream(stream)))
+
+
+def moe_permute_noalloc(idx, d, counts, offsets, perm, inv, stream=None) -> None:
+    """moe_permute without a workspace (scratch inside the library; T <= 16384, E <= 1024)."""
+    _check(_lib.moe_permute_noalloc(_ptr(idx, torch.int32, "idx"), ctypes.byref(d),
+                                    _ptr(counts, torch.int32, "counts"),
+                                    _ptr(offsets, torch.int32, "offsets"),
+                                    _ptr(perm, torch.int32, "perm"), _ptr(inv, torch.int32, "inv"),
+                                    _stream(stream)))
 
 
 def moe_expert_ffn(h, perm, offsets, W1, W3, W2, Ws1, Ws3, Ws2, d, y, ws, stream=None) -> None:

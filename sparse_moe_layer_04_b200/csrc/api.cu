@@ -282,6 +282,40 @@ int moe_permute(const int32_t* idx, const moe_dims_t* dims, int32_t* counts, int
   return MOE_OK;
 }
 
+int moe_permute_noalloc(const int32_t* idx, const moe_dims_t* dims, int32_t* counts,
+                        int32_t* offsets, int32_t* perm, int32_t* inv, moe_stream_t stream) {
+  int rc = begin(dims);
+  if (rc) return rc;
+  MOE_CHECK_PTR(counts);
+  MOE_CHECK_PTR(offsets);
+  const int nblk = (dims->T + kPermBlockTokens - 1) / kPermBlockTokens;
+  if (nblk > kNoAllocMaxBlocks || dims->E > kNoAllocMaxExperts)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_permute_noalloc: T = %d, E = %d exceeds the static scratch (T <= %d, E <= %d)",
+                dims->T, dims->E, kNoAllocMaxBlocks * kPermBlockTokens, kNoAllocMaxExperts);
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dims->T == 0) {
+    if ((rc = check_device())) return rc;
+    cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)dims->E * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, (size_t)(dims->E + 1) * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "memset");
+    return MOE_OK;
+  }
+  MOE_CHECK_PTR(idx);
+  MOE_CHECK_PTR(perm);
+  MOE_CHECK_PTR(inv);
+  if ((rc = check_device())) return rc;
+  int32_t* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_permute_noalloc: scratch address lookup");
+  int n = 0;
+  e = launch_permute(idx, dims->T, dims->E, dims->k, counts, offsets, perm, inv, scratch,
+                     nullptr, st, &n);
+  if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  g_launches = n;
+  return MOE_OK;
+}
+
 int moe_expert_ffn(const void* h, const int32_t* perm, const int32_t* offsets, const void* W1,
                    const void* W3, const void* W2, const void* Ws1, const void* Ws3,
                    const void* Ws2, const moe_dims_t* dims, float* y, void* ws, size_t ws_bytes,

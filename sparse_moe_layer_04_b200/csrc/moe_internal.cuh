@@ -37,6 +37,11 @@ int router_tile_n(int T, int E);  // MMA N of the tensor-core router
 
 // Permute: tokens per counting block.
 constexpr int kPermBlockTokens = 256;
+// Capacity of the grouping's static scratch (allocation-free variant):
+// 64 counting blocks (T <= 16384) x 1024 experts, 256 KiB.
+constexpr int kNoAllocMaxBlocks = 64;
+constexpr int kNoAllocMaxExperts = 1024;
+cudaError_t noalloc_scratch(int32_t** out);
 
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
 struct WsLayout {

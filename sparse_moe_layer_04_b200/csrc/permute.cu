@@ -194,6 +194,34 @@ __global__ void __launch_bounds__(kPermBlockTokens) permute_single_block_kernel(
   if (bad && status) atomicOr(status, kStBounds);
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for the allocation-free variant of the grouping.  It lives in the
+// library's own device memory, so callers that cannot allocate device memory
+// still get the multi-block path.  Every GPU that loads the library holds it
+// until the process exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) int32_t g_perm_scratch[kNoAllocMaxBlocks * kNoAllocMaxExperts];
+
+// Device address of the scratch array on the current device.  Host code only
+// sees a stand-in symbol for a __device__ array, so the address is looked up
+// with cudaGetSymbolAddress, once per device, with that device current.
+cudaError_t noalloc_scratch(int32_t** out) {
+  constexpr int kMaxDevices = 64;
+  static int32_t* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_perm_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* blk_base,
                            int* status, cudaStream_t st, int* nlaunch) {
