@@ -35,7 +35,7 @@ import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE-layer tokens/sec on 1 B200 and % of roofline (HBM or bf16 tensor peak)"
 FLUSH_BYTES = 256 << 20
-STAGES = ["router_logits", "route", "permute", "gather", "gateup_gemm", "down_gemm", "combine"]
+STAGES = ["router_logits", "route", "permute", "gather", "expert_ffn", "combine"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -53,16 +53,19 @@ def layer_bytes_flops(cfg, U: int):
     return B, FL
 
 
-def gateup_bytes(cfg, U: int):
-    """Algorithmic bytes of one gate/up GEMM launch: the W1 and W3 rows of the
-    touched routed experts and of the shared experts, the gathered input rows
-    and the bf16 activations written."""
+def ffn_bytes(cfg, U: int):
+    """Algorithmic bytes of one expert-FFN launch (gate/up and down GEMMs in one
+    kernel): W1, W3 and W2 of the touched routed experts and of the shared
+    experts, the gathered bf16 input rows, and the fp32 expert outputs written.
+    The gated activations stay inside the kernel's working set and are not
+    counted."""
     T, D, F, k, S, Fs = cfg.T, cfg.D, cfg.F, cfg.k, cfg.S, cfg.Fs
-    return U * 2 * F * D * 2 + S * 2 * Fs * D * 2 + (T * k + S * T) * D * 2 + (T * k * F + S * T * Fs) * 2
+    return (U * 3 * F * D * 2 + S * 3 * Fs * D * 2 + (T * k + S * T) * D * 2
+            + (T * k + S * T) * D * 4)
 
 
-def gateup_flops(cfg):
-    return 4 * cfg.D * (cfg.F * cfg.T * cfg.k + cfg.Fs * cfg.T * cfg.S)
+def ffn_flops(cfg):
+    return 6 * cfg.D * (cfg.F * cfg.T * cfg.k + cfg.Fs * cfg.T * cfg.S)
 
 
 def load_peaks():
@@ -233,13 +236,33 @@ def run_ours(args, rank, world, local_rank):
     launches_per_step = moe.moe_last_launch_count()
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_PROFILE_EVENTS)]
-          for _ in range(K)]
-    for evs in ev:  # create the CUDA events before the timed region
-        for e in evs:
-            e.record()
+    # headline loop: one event pair around each step (nothing recorded between
+    # the step's kernels, so their programmatic launch overlap is intact)
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for e in ev0 + ev1:  # create the CUDA events before the timed region
+        e.record()
     if world > 1:
         torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        ev0[i].record()
+        step()
+        ev1[i].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    step_ms = [ev0[i].elapsed_time(ev1[i]) for i in range(K)]
+
+    # profiled loop: events at every stage boundary (stage times and the
+    # dominant kernel's duration, measured on the launching stream)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_PROFILE_EVENTS)]
+          for _ in range(K)]
+    for evs in ev:
+        for e in evs:
+            e.record()
     torch.cuda.synchronize()
     for i in range(K):
         flush.zero_()
@@ -247,22 +270,19 @@ def run_ours(args, rank, world, local_rank):
         step()
     moe.moe_set_profile_events(None)
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
     clocks = sampler.stop()
     if moe.moe_get_device_status(ws) != 0:
         raise RuntimeError("device status error in the timed region: " + moe.moe_last_error())
 
-    step_ms = [ev[i][0].elapsed_time(ev[i][7]) for i in range(K)]
     stage_ms = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K))
                 for j, name in enumerate(STAGES)}
+    profiled_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][len(STAGES)]) for i in range(K))
     ms = statistics.mean(step_ms)
-    gateup_ms = stage_ms["gateup_gemm"]
+    ffn_ms = stage_ms["expert_ffn"]
     if world > 1:
-        t = torch.tensor([ms, gateup_ms], device=dev, dtype=torch.float64)
+        t = torch.tensor([ms, ffn_ms], device=dev, dtype=torch.float64)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, gateup_ms = t.tolist()
+        ms, ffn_ms = t.tolist()
 
     counts = torch.bincount(idx.flatten().long(), minlength=cfg.E)
     U = int((counts > 0).sum().item())
@@ -301,20 +321,20 @@ def run_ours(args, rank, world, local_rank):
     t_s = ms / 1e3
     t_roof_hbm = B / (hbm * 1e9)
     t_roof_tc = FL / (bf16 * 1e12)
-    gu_bytes = gateup_bytes(cfg, U)
-    gu_flops = gateup_flops(cfg)
-    gu_gbs = gu_bytes / (gateup_ms / 1e3) / 1e9
-    gu_tfs = gu_flops / (gateup_ms / 1e3) / 1e12
-    gu_bound = "hbm" if gu_bytes / (hbm * 1e9) >= gu_flops / (bf16 * 1e12) else "tensor"
-    if gu_bound == "hbm":
-        roof = {"bound": "hbm", "achieved": gu_gbs, "peak": hbm, "unit": "GB/s",
-                "frac": gu_gbs / hbm}
+    f_bytes = ffn_bytes(cfg, U)
+    f_flops = ffn_flops(cfg)
+    f_gbs = f_bytes / (ffn_ms / 1e3) / 1e9
+    f_tfs = f_flops / (ffn_ms / 1e3) / 1e12
+    f_bound = "hbm" if f_bytes / (hbm * 1e9) >= f_flops / (bf16 * 1e12) else "tensor"
+    if f_bound == "hbm":
+        roof = {"bound": "hbm", "achieved": f_gbs, "peak": hbm, "unit": "GB/s",
+                "frac": f_gbs / hbm}
     else:
-        roof = {"bound": "tensor", "achieved": gu_tfs, "peak": bf16, "unit": "TFLOP/s",
-                "frac": gu_tfs / bf16}
-    roof.update({"traffic": stored_traffic(f"grouped_gemm_gateup/{cfg.name}"),
-                 "kernel": "grouped_gemm_kernel<gate/up>", "ms": gateup_ms,
-                 "algorithmic_bytes": gu_bytes, "algorithmic_flops": gu_flops,
+        roof = {"bound": "tensor", "achieved": f_tfs, "peak": bf16, "unit": "TFLOP/s",
+                "frac": f_tfs / bf16}
+    roof.update({"traffic": stored_traffic(f"expert_ffn/{cfg.name}"),
+                 "kernel": "grouped_gemm_kernel (fused gate/up + down expert FFN)", "ms": ffn_ms,
+                 "algorithmic_bytes": f_bytes, "algorithmic_flops": f_flops,
                  "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured"
                  else "fallback (profiling recipe)"})
 
@@ -341,7 +361,7 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world} (token-parallel, no exchange)",
                    "l2": "flushed: 256 MiB memset before every timed step, outside its events",
                    "ms_p10_p90": [float(np.percentile(step_ms, 10)), float(np.percentile(step_ms, 90))],
-                   "stage_ms": stage_ms},
+                   "stage_ms": stage_ms, "profiled_step_ms": profiled_ms},
         "roofline": roof,
         "layer_roofline": {
             "bytes": B, "flops": FL, "t_roof_ms": max(t_roof_hbm, t_roof_tc) * 1e3,
@@ -353,6 +373,7 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": cfg.T * cfg.D * 2, "d2h_bytes_per_step": cfg.T * cfg.D * 4,
                 "ms_per_step": e2e},
         "gpu_launches": launches_per_step * K,
+        "gpu_launches_note": "kernels of the headline timed loop (the profiled loop runs as many again)",
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -199,11 +199,13 @@ int moe_last_launch_count(void);
  * call on this thread records them on its stream at the stage boundaries:
  *   events[0] before the router, [1] after the router logits, [2] after the
  *   routing, [3] after the grouping, [4] after the row gather, [5] after the
- *   gate/up GEMM, [6] after the down GEMM, [7] after the merge.
- * n must be MOE_PROFILE_EVENTS (8) to enable, or 0 (events may be NULL) to
+ *   expert FFN (gate/up and down GEMMs, one kernel), [6] after the merge.
+ * Recording events between the kernels costs their overlapped launches, so
+ * profiled steps run a little slower than unprofiled ones.
+ * n must be MOE_PROFILE_EVENTS (7) to enable, or 0 (events may be NULL) to
  * disable.  The library keeps the pointer, not a copy: the array must stay
  * valid while enabled. */
-#define MOE_PROFILE_EVENTS 8
+#define MOE_PROFILE_EVENTS 7
 int moe_set_profile_events(void* const* events, int n);
 
 #ifdef __cplusplus

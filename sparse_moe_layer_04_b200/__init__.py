@@ -199,7 +199,7 @@ def moe_last_launch_count() -> int:
     return _lib.moe_last_launch_count()
 
 
-MOE_PROFILE_EVENTS = 8
+MOE_PROFILE_EVENTS = 7
 _prof_keep = None
 
 

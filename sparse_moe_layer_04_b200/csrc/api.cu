@@ -165,6 +165,7 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
   L->perm = take(T * k * 4);
   L->inv = take(T * k * 4);
   L->blk_base = take(nblk * E * 4);
+  L->counters = take((E + S) * 4);
   L->xperm = take(T * k * D * 2);
   L->act_r = take(T * k * F * 2);
   L->act_s = take(S * T * Fs * 2);
@@ -341,8 +342,9 @@ int moe_expert_ffn(const void* h, const int32_t* perm, const int32_t* offsets, c
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int rows = dims->T * dims->k;
   uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
+  int32_t* counters = w.at<int32_t>(w.L.counters);
   cudaError_t e = launch_gather_rows(static_cast<const uint16_t*>(h), perm, rows, dims->D,
-                                     dims->T, xperm, st);
+                                     dims->T, xperm, counters, dims->E + dims->S, st);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   FfnArgs a;
   a.xperm = xperm;
@@ -358,6 +360,7 @@ int moe_expert_ffn(const void* h, const int32_t* perm, const int32_t* offsets, c
   a.act_s = w.at<uint16_t>(w.L.act_s);
   a.y = y;
   a.status = w.status();
+  a.counters = counters;
   a.T = dims->T; a.D = dims->D; a.E = dims->E; a.F = dims->F; a.k = dims->k;
   a.S = dims->S; a.Fs = dims->Fs;
   int n = 1;
@@ -443,7 +446,8 @@ int moe_forward(const void* h, const float* Wr, const float* bias, const void* W
   if (e == cudaSuccess) e = mark(3, st);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
-  e = launch_gather_rows(hb, perm, T * k, D, T, xperm, st);
+  int32_t* counters = w.at<int32_t>(w.L.counters);
+  e = launch_gather_rows(hb, perm, T * k, D, T, xperm, counters, E + dims->S, st);
   if (e == cudaSuccess) e = mark(4, st);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   n += 1;
@@ -461,12 +465,13 @@ int moe_forward(const void* h, const float* Wr, const float* bias, const void* W
   a.act_s = w.at<uint16_t>(w.L.act_s);
   a.y = y;
   a.status = w.status();
+  a.counters = counters;
   a.T = T; a.D = D; a.E = E; a.F = dims->F; a.k = k; a.S = dims->S; a.Fs = dims->Fs;
   const char* why = "launch failed";
   e = launch_expert_ffn(a, st, &n, &why, g_prof_events ? g_prof_events + 5 : nullptr);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
   e = launch_combine(y, rw, inv, T, D, k, dims->S, out, w.status(), st);
-  if (e == cudaSuccess) e = mark(7, st);
+  if (e == cudaSuccess) e = mark(6, st);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   n += 1;
   g_launches = n;

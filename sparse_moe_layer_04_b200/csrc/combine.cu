@@ -8,6 +8,7 @@
 #include <cuda_bf16.h>
 
 #include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 
@@ -19,6 +20,8 @@ constexpr int kMaxK = 32;
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const float* __restrict__ y, const float* __restrict__ w, const int32_t* __restrict__ inv,
     int T, int D, int k, int S, float* __restrict__ out, int* __restrict__ status) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
   __shared__ int s_row[kMaxK];
   __shared__ float s_w[kMaxK];
   const int t = blockIdx.x;
@@ -65,8 +68,8 @@ cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, i
                            int k, int S, float* out, int* status, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const dim3 grid(T, (D / 4 + kCombineThreads - 1) / kCombineThreads);
-  combine_kernel<<<grid, kCombineThreads, 0, st>>>(y, w, inv, T, D, k, S, out, status);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, grid, dim3(kCombineThreads), 0, st, y, w, inv, T, D, k, S, out,
+                    status);
 }
 
 }  // namespace moe

@@ -8,18 +8,32 @@
 // rows grouped to them; the always-on shared expert sees every token ("Model
 // anatomy -- GLM-5.2", MoE panel, and "Expert fan-out 8 + 1").
 //
-// Two launches:
-//   gate/up : act[r, n] = silu(sum_d A[r, d] W1[e][n, d]) * (sum_d A[r, d] W3[e][n, d])
+// One persistent kernel runs up to two grouped GEMM "problems" back to back
+// in a single tile space:
+//   problem 0 (gate/up): act[r, n] = silu(A[r] . W1[e][n]) * (A[r] . W3[e][n])
 //             128 x N/2 output tile; the W1 and W3 row blocks of the tile are
 //             stacked into one N-row B operand, so one MMA feeds both
 //             accumulators (TMEM columns [0, N/2) gate, [N/2, N) up) and the
 //             epilogue applies the SiLU gate and rounds to bf16.
-//   down    : y[r, n] = sum_f act[r, f] W2[e][n, f], 128 x N fp32 tile.
+//   problem 1 (down):    y[r, n] = act[r] . W2[e][n], 128 x N fp32 tile.
+// Tiles are numbered problem 0 first, then problem 1; within a problem routed
+// experts first (expert, column tile, row tile with the row tile fastest, so
+// CTAs running at the same time share each weight tile through L2), then the
+// shared experts.  CTA c takes tiles c, c + gridDim.x, ...  A down tile of an
+// expert waits until every gate/up tile of that expert has been stored: each
+// gate/up epilogue warp releases a per-expert counter after a proxy fence, and
+// the producer acquires it before its TMA loads read the activations.  Down tiles
+// therefore fill the SMs that the tail of the gate/up tiles leaves idle.
+// Because every CTA takes its tiles in increasing order and all CTAs are
+// resident (one per SM), every counter a CTA waits on is advanced by tiles that
+// precede it, so the waits always end; they are bounded all the same.
+//
 // N (the MMA width) is 256 for large batches and 128 for small ones, where
 // each expert has only a row tile or two and the weight stream must be cut
-// finer to keep all 148 SMs busy.
+// finer to keep all 148 SMs busy.  The same kernel also computes the router
+// logits as a dense split-K GEMM (one problem, one shared group per K chunk).
 //
-// Kernel structure (one persistent CTA per SM, 192 threads):
+// CTA structure (192 threads, one CTA per SM):
 //   warp 0      TMA producer: ring of (A 128x64, B Nx64) bf16 tiles (4 stages
 //               for N = 256, 6 for N = 128), 128-byte swizzled, completion
 //               counted on "full" mbarriers.
@@ -29,10 +43,6 @@
 //               epilogue of tile i overlaps the main loop of tile i+1.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
 //               lanes 32*(w%4) .. +31), fused activation, global stores.
-// Tiles are numbered routed-first (expert, n-tile, m-tile with m fastest, so
-// CTAs that run at the same time share each weight tile through L2), then the
-// shared experts; CTA c takes tiles c, c + gridDim.x, ...  The routed tile
-// count comes from the device-side group offsets, so no host round trip.
 #include <cuda_bf16.h>
 
 #include "moe_internal.cuh"
@@ -47,9 +57,9 @@ constexpr int THREADS = 192;
 constexpr int A_BYTES = BM * BK * 2;      // 16 KiB
 constexpr int MAX_E = 1024;
 constexpr int RING_BYTES = 192 * 1024;    // operand ring budget
+constexpr int MAX_STAGES = 6;
+constexpr int EPI_WARPS = 4;              // each releases its rows of a gate/up tile
 
-// Tile shape of one instantiation: MMA N = 256 (large batches) or 128 (small
-// batches, twice as many tiles to spread the weight stream over every SM).
 template <int MMA_N>
 struct Shape {
   static constexpr int B_BYTES = MMA_N * BK * 2;
@@ -59,29 +69,38 @@ struct Shape {
   static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;        // double buffered
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, MMA_N);
 };
-constexpr int MAX_STAGES = 6;
 
-struct GemmParams {
+// One grouped GEMM.  Routed group e has rows [off[e], off[e+1]) of the routed
+// A / output matrices; shared group s has rows s*T .. s*T + T - 1 of the
+// shared output (its A rows start at s * a_s_group_stride).
+struct alignas(64) Problem {
   CUtensorMap a_r;   // routed A  [rows_r, K_r]
-  CUtensorMap a_s;   // shared A  [.., K_s]
+  CUtensorMap a_s;   // shared A
   CUtensorMap b0_r;  // W1 [E*F, D] (gate/up) | W2 [E*D, F] (down)
   CUtensorMap b1_r;  // W3 [E*F, D] (gate/up only)
   CUtensorMap b0_s;  // Ws1 | Ws2
   CUtensorMap b1_s;  // Ws3
-  const int32_t* offsets;
   void* out_r;
   void* out_s;
-  int* status;
-  int E, S, T;
   int K_r, K_s;              // reduction lengths
   int N_r, N_s;              // output columns (= output row strides)
-  int rows_r;                // T * k
-  int a_s_group_stride;      // rows between shared experts' A blocks (0 or T)
+  int a_s_group_stride;      // rows between shared groups' A blocks (0 or T)
   int b_r_group_rows;        // B rows per routed expert (F or D)
-  int b_s_group_rows;        // B rows per shared expert (Fs or D)
-  int bn_out;                // output columns per tile (MMA_N, or MMA_N / 2 for gate/up)
+  int b_s_group_rows;        // B rows per shared expert (Fs, D or 0)
+  int bn_out;                // output columns per tile (N or N/2)
   int k_chunk;               // > 0: shared group g covers K range [g*k_chunk, (g+1)*k_chunk)
   int a_k_mod;               // > 0: the A operand's K coordinate wraps modulo this
+  int gateup;                // epilogue: 1 = SiLU gate -> bf16, 0 = fp32 store
+};
+
+struct GemmParams {
+  Problem pr[2];
+  const int32_t* offsets;    // [E+1] routed group row offsets (E > 0)
+  int* status;
+  int* counters;             // [E+S] gate/up tiles stored per group (two problems)
+  int nprob;                 // 1 or 2
+  int E, S, T;
+  int rows_r;                // T * k
 };
 
 struct SharedState {
@@ -92,65 +111,84 @@ struct SharedState {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  int routed_tiles;
+  int mt_total;              // routed row tiles over all experts
   int off[MAX_E + 1];        // group row offsets
-  int prefix[MAX_E + 1];     // routed tile prefix per expert
+  int mt_prefix[MAX_E + 1];  // routed row-tile prefix per expert
 };
 
 struct TileInfo {
+  int prob;
   bool shared;
   int grp;      // expert (routed) or shared expert index
   int m0;       // first row within the group
   int n0;       // first output column
   int rows;     // rows in the group
   int row0;     // group's first row in the output (and routed A) matrix
+  int mt;       // row tiles of the group
 };
 
+__device__ __forceinline__ int col_tiles(int N, int bn) { return (N + bn - 1) / bn; }
+
+__device__ __forceinline__ int problem_tiles(const Problem& P, const SharedState& ss,
+                                             const GemmParams& p) {
+  const int mt_s = (p.T + BM - 1) / BM;
+  return ss.mt_total * col_tiles(P.N_r, P.bn_out) + p.S * mt_s * col_tiles(P.N_s, P.bn_out);
+}
+
 __device__ __forceinline__ TileInfo decode_tile(int tile, const SharedState& ss,
-                                                const GemmParams& p) {
+                                                const GemmParams& p, int tiles0) {
   TileInfo ti;
-  if (tile < ss.routed_tiles) {
-    int lo = 0, hi = p.E - 1;  // find e with prefix[e] <= tile < prefix[e+1]
+  ti.prob = (tile >= tiles0) ? 1 : 0;
+  const Problem& P = p.pr[ti.prob];
+  const int lt = tile - (ti.prob ? tiles0 : 0);
+  const int nt_r = col_tiles(P.N_r, P.bn_out);
+  const int routed = ss.mt_total * nt_r;
+  if (lt < routed) {
+    // expert e: largest with mt_prefix[e] * nt_r <= lt
+    const int q = lt / nt_r;
+    int lo = 0, hi = p.E - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (ss.prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+      if (ss.mt_prefix[mid] <= q) lo = mid; else hi = mid - 1;
     }
     const int e = lo;
     const int rows = ss.off[e + 1] - ss.off[e];
     const int mt = (rows + BM - 1) / BM;
-    const int local = tile - ss.prefix[e];
+    const int local = lt - ss.mt_prefix[e] * nt_r;
     ti.shared = false;
     ti.grp = e;
     ti.m0 = (local % mt) * BM;
-    ti.n0 = (local / mt) * p.bn_out;
+    ti.n0 = (local / mt) * P.bn_out;
     ti.rows = rows;
     ti.row0 = ss.off[e];
+    ti.mt = mt;
   } else {
-    const int local = tile - ss.routed_tiles;
+    const int ls = lt - routed;
     const int mt = (p.T + BM - 1) / BM;
-    const int nt = (p.N_s + p.bn_out - 1) / p.bn_out;
-    const int s = local / (mt * nt);
-    const int rem = local - s * mt * nt;
+    const int nt = col_tiles(P.N_s, P.bn_out);
+    const int s = ls / (mt * nt);
+    const int rem = ls - s * mt * nt;
     ti.shared = true;
     ti.grp = s;
     ti.m0 = (rem % mt) * BM;
-    ti.n0 = (rem / mt) * p.bn_out;
+    ti.n0 = (rem / mt) * P.bn_out;
     ti.rows = p.T;
     ti.row0 = s * p.T;
+    ti.mt = mt;
   }
   return ti;
 }
 
 // K range of a tile: the whole reduction, or one chunk of it when the shared
 // groups split K (the router's split-K partial sums).
-__device__ __forceinline__ void tile_k_range(const TileInfo& ti, const GemmParams& p, int* kbeg,
+__device__ __forceinline__ void tile_k_range(const TileInfo& ti, const Problem& P, int* kbeg,
                                              int* K) {
-  if (ti.shared && p.k_chunk > 0) {
-    *kbeg = ti.grp * p.k_chunk;
-    *K = min(p.k_chunk, p.K_s - *kbeg);
+  if (ti.shared && P.k_chunk > 0) {
+    *kbeg = ti.grp * P.k_chunk;
+    *K = min(P.k_chunk, P.K_s - *kbeg);
   } else {
     *kbeg = 0;
-    *K = ti.shared ? p.K_s : p.K_r;
+    *K = ti.shared ? P.K_s : P.K_r;
   }
 }
 
@@ -170,12 +208,26 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, volat
   if (!ptx::mbar_wait(bar, parity, &ignore_abort)) *abort = 1;
 }
 
-template <bool GATEUP, int MMA_N>
+// Waits until *ctr >= target (acquire), bounded like the mbarrier waits.
+__device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatile int* abort) {
+  if (ptx::ld_acquire_gpu(ctr) >= target) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    __nanosleep(128);
+    if (ptx::ld_acquire_gpu(ctr) >= target) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > ptx::kWaitBudgetCycles) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+template <int MMA_N>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   using Sh = Shape<MMA_N>;
   constexpr int STAGES = Sh::STAGES;
   constexpr int STAGE_BYTES = Sh::STAGE_BYTES;
-  constexpr int B_BYTES = Sh::B_BYTES;
   constexpr int ACC_COLS = Sh::ACC_COLS;
   constexpr uint32_t TMEM_COLS = Sh::TMEM_COLS;
   constexpr uint32_t IDESC = Sh::IDESC;
@@ -189,6 +241,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  ptx::pdl_launch_dependents();
   if (warp == 1) {
     ptx::tmem_alloc(&ss.tmem_base, TMEM_COLS);
     ptx::tmem_relinquish();
@@ -207,15 +260,17 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     ptx::fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    ptx::tma_prefetch_desc(&p.a_r);
-    ptx::tma_prefetch_desc(&p.b0_r);
-    if (GATEUP) ptx::tma_prefetch_desc(&p.b1_r);
+    ptx::tma_prefetch_desc(&p.pr[0].a_r);
+    ptx::tma_prefetch_desc(&p.pr[0].b0_r);
+    ptx::tma_prefetch_desc(&p.pr[0].b1_r);
   }
-  // Routed tile prefix from the group offsets (warp 2 scans 32 experts at a time).
+  // everything below reads what earlier kernels in the stream wrote
+  ptx::pdl_wait();
+
+  // Routed row-tile prefix from the group offsets (warp 2 scans 32 experts at a time).
   if (warp == 2) {
     int carry = 0;
     bool bad = false;
-    const int nt = (p.N_r + p.bn_out - 1) / p.bn_out;
     for (int base = 0; base < p.E; base += 32) {
       const int e = base + lane;
       int cnt = 0;
@@ -224,8 +279,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         ss.off[e] = a;
         if (e == p.E - 1) ss.off[p.E] = b;
         if (a < 0 || b < a || b > p.rows_r || (e == 0 && a != 0)) bad = true;
-        cnt = ((b - a + BM - 1) / BM) * nt;
-        if (b < a) cnt = 0;
+        cnt = b >= a ? (b - a + BM - 1) / BM : 0;
       }
       int incl = cnt;
 #pragma unroll
@@ -233,13 +287,13 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         const int v = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += v;
       }
-      if (e < p.E) ss.prefix[e] = carry + incl - cnt;
+      if (e < p.E) ss.mt_prefix[e] = carry + incl - cnt;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
     bad = __any_sync(0xffffffffu, bad);
     if (lane == 0) {
-      ss.prefix[p.E] = carry;
-      ss.routed_tiles = bad ? 0 : carry;
+      ss.mt_prefix[p.E] = carry;
+      ss.mt_total = bad ? 0 : carry;
       if (bad && p.status) atomicOr(p.status, kStBounds);
     }
   }
@@ -248,9 +302,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   ptx::tc_fence_after();
 
   const uint32_t tmem_base = ss.tmem_base;
-  const int mt_s = (p.T + BM - 1) / BM;
-  const int nt_s = (p.N_s + p.bn_out - 1) / p.bn_out;
-  const int total = ss.routed_tiles + p.S * mt_s * nt_s;
+  const int tiles0 = problem_tiles(p.pr[0], ss, p);
+  const int total = tiles0 + (p.nprob > 1 ? problem_tiles(p.pr[1], ss, p) : 0);
   volatile int* abort = &ss.abort;
 
   if (warp == 0) {
@@ -260,14 +313,23 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       uint32_t phase = 0;
       uint32_t issued_mask = 0, last_parity = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(tile, ss, p);
-        const CUtensorMap* amap = ti.shared ? &p.a_s : &p.a_r;
-        const CUtensorMap* b0 = ti.shared ? &p.b0_s : &p.b0_r;
-        const CUtensorMap* b1 = ti.shared ? &p.b1_s : &p.b1_r;
-        const int a_row = ti.shared ? ti.grp * p.a_s_group_stride + ti.m0 : ti.row0 + ti.m0;
-        const int b_row = ti.grp * (ti.shared ? p.b_s_group_rows : p.b_r_group_rows) + ti.n0;
+        const TileInfo ti = decode_tile(tile, ss, p, tiles0);
+        const Problem& P = p.pr[ti.prob];
+        if (ti.prob == 1) {
+          // the activations of this group come from problem 0's epilogues
+          const int g = ti.shared ? p.E + ti.grp : ti.grp;
+          const int nt0 = ti.shared ? col_tiles(p.pr[0].N_s, p.pr[0].bn_out)
+                                    : col_tiles(p.pr[0].N_r, p.pr[0].bn_out);
+          if (!wait_counter(p.counters + g, EPI_WARPS * ti.mt * nt0, abort)) break;
+          ptx::fence_proxy_async_global();
+        }
+        const CUtensorMap* amap = ti.shared ? &P.a_s : &P.a_r;
+        const CUtensorMap* b0 = ti.shared ? &P.b0_s : &P.b0_r;
+        const CUtensorMap* b1 = ti.shared ? &P.b1_s : &P.b1_r;
+        const int a_row = ti.shared ? ti.grp * P.a_s_group_stride + ti.m0 : ti.row0 + ti.m0;
+        const int b_row = ti.grp * (ti.shared ? P.b_s_group_rows : P.b_r_group_rows) + ti.n0;
         int kbeg, K;
-        tile_k_range(ti, p, &kbeg, &K);
+        tile_k_range(ti, P, &kbeg, &K);
         const int nk = (K + BK - 1) / BK;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
@@ -275,10 +337,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           uint8_t* sa = ring + stage * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
           const int xb = kbeg + kb * BK;
-          const int xa = p.a_k_mod > 0 ? xb % p.a_k_mod : xb;
+          const int xa = P.a_k_mod > 0 ? xb % P.a_k_mod : xb;
           ptx::mbar_arrive_expect_tx(&ss.full[stage], STAGE_BYTES);
           ptx::tma_load_2d(sa, amap, &ss.full[stage], xa, a_row);
-          if (GATEUP) {
+          if (P.gateup) {
             ptx::tma_load_2d(sb, b0, &ss.full[stage], xb, b_row);
             ptx::tma_load_2d(sb + HALF * BK * 2, b1, &ss.full[stage], xb, b_row);
           } else {
@@ -302,9 +364,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(tile, ss, p);
+        const TileInfo ti = decode_tile(tile, ss, p, tiles0);
         int kbeg, K;
-        tile_k_range(ti, p, &kbeg, &K);
+        tile_k_range(ti, p.pr[ti.prob], &kbeg, &K);
         const int nk = (K + BK - 1) / BK;
         if (!ptx::mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1u, abort)) break;
         ptx::tc_fence_after();
@@ -337,16 +399,17 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const TileInfo ti = decode_tile(tile, ss, p);
+      const TileInfo ti = decode_tile(tile, ss, p, tiles0);
+      const Problem& P = p.pr[ti.prob];
       if (!ptx::mbar_wait(&ss.tmem_full[acc], acc_phase, abort)) break;
       ptx::tc_fence_after();
       const int r = ti.m0 + q * 32 + lane;       // row within the group
       const bool row_ok = r < ti.rows;
-      const int N = ti.shared ? p.N_s : p.N_r;
+      const int N = ti.shared ? P.N_s : P.N_r;
       const size_t out_row = (size_t)ti.row0 + r;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * ACC_COLS;
-      if (GATEUP) {
-        uint16_t* out = static_cast<uint16_t*>(ti.shared ? p.out_s : p.out_r);
+      if (P.gateup) {
+        uint16_t* out = static_cast<uint16_t*>(ti.shared ? P.out_s : P.out_r);
 #pragma unroll 1
         for (int c = 0; c < HALF; c += 16) {
           uint32_t g[16], u[16];
@@ -367,7 +430,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           }
         }
       } else {
-        float* out = static_cast<float*>(ti.shared ? p.out_s : p.out_r);
+        float* out = static_cast<float*>(ti.shared ? P.out_s : P.out_r);
 #pragma unroll 1
         for (int c = 0; c < MMA_N; c += 16) {
           uint32_t v[16];
@@ -389,6 +452,15 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ss.tmem_empty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (p.nprob > 1 && ti.prob == 0) {
+        // release this warp's rows of the tile to the down tiles of its
+        // group: make the stores visible to the async proxy and to the whole
+        // GPU, then count them (four counts per tile, one per epilogue warp)
+        ptx::fence_proxy_async_global();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.counters + (ti.shared ? p.E + ti.grp : ti.grp), 1);
+      }
     }
   }
 
@@ -443,13 +515,13 @@ constexpr size_t smem_bytes() {
 static_assert(smem_bytes<256>() <= 227 * 1024 && smem_bytes<128>() <= 227 * 1024,
               "shared memory budget");
 
-template <bool GATEUP, int MMA_N>
+template <int MMA_N>
 cudaError_t launch_one(const GemmParams& p, int tiles_upper, cudaStream_t st) {
   static int configured_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<GATEUP, MMA_N>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MMA_N>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_bytes<MMA_N>());
     if (e != cudaSuccess) return e;
@@ -458,8 +530,8 @@ cudaError_t launch_one(const GemmParams& p, int tiles_upper, cudaStream_t st) {
   int grid = num_sms();
   if (tiles_upper < grid) grid = tiles_upper;
   if (grid < 1) grid = 1;
-  grouped_gemm_kernel<GATEUP, MMA_N><<<grid, THREADS, smem_bytes<MMA_N>(), st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_kernel<MMA_N>, dim3(grid), dim3(THREADS), smem_bytes<MMA_N>(),
+                    st, p);
 }
 
 }  // namespace
@@ -469,38 +541,40 @@ cudaError_t launch_one(const GemmParams& p, int tiles_upper, cudaStream_t st) {
 // previous pieces leave; together they carry the 24-bit fp32 significand),
 // stored side by side as wr3 [E, 3D].  h is bf16 and so exact in the MMA, so
 //   logits = [h | h | h] . wr3^T
-// is a dense GEMM over K' = 3D with fp32 accumulation.  It runs on the
-// grouped kernel as `nsplit` shared groups that each take one K' chunk and
-// write their own partial-sum plane [T, E]; the consumer adds the planes in
-// order.
+// is a dense GEMM over K' = 3D with fp32 accumulation.  It runs as `nsplit`
+// shared groups that each take one K' chunk and write their own partial-sum
+// plane [T, E]; the consumer adds the planes in order.
 cudaError_t launch_router_tc(const uint16_t* h, const uint16_t* wr3, int T, int D, int E,
                              int nsplit, int chunk, float* partials, cudaStream_t st,
                              const char** why) {
   const int bn = router_tile_n(T, E);
-  const bool narrow = bn == 128;
   GemmParams p{};
-  if (!make_map(&p.a_s, h, T, D, BM) || !make_map(&p.b0_s, wr3, E, 3ull * D, bn)) {
+  Problem& P = p.pr[0];
+  if (!make_map(&P.a_s, h, T, D, BM) || !make_map(&P.b0_s, wr3, E, 3ull * D, bn)) {
     *why = "cuTensorMapEncodeTiled failed for a router operand";
     return cudaErrorInvalidValue;
   }
-  p.a_r = p.a_s;
-  p.b0_r = p.b1_r = p.b1_s = p.b0_s;
+  P.a_r = P.a_s;
+  P.b0_r = P.b1_r = P.b1_s = P.b0_s;
+  P.out_r = nullptr;
+  P.out_s = partials;
+  P.K_r = 0; P.K_s = 3 * D;
+  P.N_r = 0; P.N_s = E;
+  P.a_s_group_stride = 0;
+  P.b_r_group_rows = 0;
+  P.b_s_group_rows = 0;
+  P.bn_out = bn;
+  P.k_chunk = chunk;
+  P.a_k_mod = D;
+  P.gateup = 0;
   p.offsets = nullptr;
-  p.out_r = nullptr;
-  p.out_s = partials;
   p.status = nullptr;
+  p.counters = nullptr;
+  p.nprob = 1;
   p.E = 0; p.S = nsplit; p.T = T;
-  p.K_r = 0; p.K_s = 3 * D;
-  p.N_r = 0; p.N_s = E;
   p.rows_r = 0;
-  p.a_s_group_stride = 0;
-  p.b_r_group_rows = 0;
-  p.b_s_group_rows = 0;
-  p.bn_out = bn;
-  p.k_chunk = chunk;
-  p.a_k_mod = D;
   const int tiles = nsplit * ((T + BM - 1) / BM) * ((E + bn - 1) / bn);
-  return narrow ? launch_one<false, 128>(p, tiles, st) : launch_one<false, 256>(p, tiles, st);
+  return bn == 128 ? launch_one<128>(p, tiles, st) : launch_one<256>(p, tiles, st);
 }
 
 // Small batches (T <= 512) leave each expert with at most a few row tiles, so
@@ -517,67 +591,66 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, c
   const int nmma = narrow ? 128 : 256;
   const int half = nmma / 2;
 
-  // ---- gate/up ----
-  GemmParams g{};
-  bool ok = make_map(&g.a_r, a.xperm, rows_r, a.D, BM) &&
-            make_map(&g.b0_r, a.W1, (uint64_t)a.E * a.F, a.D, half) &&
-            make_map(&g.b1_r, a.W3, (uint64_t)a.E * a.F, a.D, half);
+  GemmParams p{};
+  // ---- problem 0: gate/up ----
+  Problem& G = p.pr[0];
+  bool ok = make_map(&G.a_r, a.xperm, rows_r, a.D, BM) &&
+            make_map(&G.b0_r, a.W1, (uint64_t)a.E * a.F, a.D, half) &&
+            make_map(&G.b1_r, a.W3, (uint64_t)a.E * a.F, a.D, half);
   if (ok && a.S > 0)
-    ok = make_map(&g.a_s, a.h, a.T, a.D, BM) &&
-         make_map(&g.b0_s, a.Ws1, (uint64_t)a.S * a.Fs, a.D, half) &&
-         make_map(&g.b1_s, a.Ws3, (uint64_t)a.S * a.Fs, a.D, half);
+    ok = make_map(&G.a_s, a.h, a.T, a.D, BM) &&
+         make_map(&G.b0_s, a.Ws1, (uint64_t)a.S * a.Fs, a.D, half) &&
+         make_map(&G.b1_s, a.Ws3, (uint64_t)a.S * a.Fs, a.D, half);
+  // ---- problem 1: down ----
+  Problem& Dn = p.pr[1];
+  ok = ok && make_map(&Dn.a_r, a.act_r, rows_r, a.F, BM) &&
+       make_map(&Dn.b0_r, a.W2, (uint64_t)a.E * a.D, a.F, nmma);
+  if (ok && a.S > 0)
+    ok = make_map(&Dn.a_s, a.act_s, (uint64_t)a.S * a.T, a.Fs, BM) &&
+         make_map(&Dn.b0_s, a.Ws2, (uint64_t)a.S * a.D, a.Fs, nmma);
   if (!ok) {
-    *why = "cuTensorMapEncodeTiled failed for a gate/up operand";
+    *why = "cuTensorMapEncodeTiled failed for an expert operand";
     return cudaErrorInvalidValue;
   }
-  g.offsets = a.offsets;
-  g.out_r = a.act_r;
-  g.out_s = a.act_s;
-  g.status = a.status;
-  g.E = a.E; g.S = a.S; g.T = a.T;
-  g.K_r = a.D; g.K_s = a.D;
-  g.N_r = a.F; g.N_s = a.Fs;
-  g.rows_r = rows_r;
-  g.a_s_group_stride = 0;
-  g.b_r_group_rows = a.F;
-  g.b_s_group_rows = a.Fs;
-  g.bn_out = half;
-  const int tiles_g = mt_upper * ((a.F + half - 1) / half) + a.S * mt_s * ((a.Fs + half - 1) / half);
-  cudaError_t err = narrow ? launch_one<true, 128>(g, tiles_g, st)
-                           : launch_one<true, 256>(g, tiles_g, st);
-  if (err == cudaSuccess && marks) err = cudaEventRecord(static_cast<cudaEvent_t>(marks[0]), st);
-  if (err != cudaSuccess) return err;
+  G.out_r = a.act_r;
+  G.out_s = a.act_s;
+  G.K_r = a.D; G.K_s = a.D;
+  G.N_r = a.F; G.N_s = a.Fs;
+  G.a_s_group_stride = 0;
+  G.b_r_group_rows = a.F;
+  G.b_s_group_rows = a.Fs;
+  G.bn_out = half;
+  G.k_chunk = 0;
+  G.a_k_mod = 0;
+  G.gateup = 1;
 
-  // ---- down ----
-  GemmParams d{};
-  ok = make_map(&d.a_r, a.act_r, rows_r, a.F, BM) &&
-       make_map(&d.b0_r, a.W2, (uint64_t)a.E * a.D, a.F, nmma);
-  if (ok && a.S > 0)
-    ok = make_map(&d.a_s, a.act_s, (uint64_t)a.S * a.T, a.Fs, BM) &&
-         make_map(&d.b0_s, a.Ws2, (uint64_t)a.S * a.D, a.Fs, nmma);
-  if (!ok) {
-    *why = "cuTensorMapEncodeTiled failed for a down-projection operand";
-    return cudaErrorInvalidValue;
-  }
-  d.b1_r = d.b0_r;
-  d.b1_s = d.b0_s;
-  d.offsets = a.offsets;
-  d.out_r = a.y;
-  d.out_s = a.y + (size_t)rows_r * a.D;
-  d.status = a.status;
-  d.E = a.E; d.S = a.S; d.T = a.T;
-  d.K_r = a.F; d.K_s = a.Fs;
-  d.N_r = a.D; d.N_s = a.D;
-  d.rows_r = rows_r;
-  d.a_s_group_stride = a.T;
-  d.b_r_group_rows = a.D;
-  d.b_s_group_rows = a.D;
-  d.bn_out = nmma;
+  Dn.b1_r = Dn.b0_r;
+  Dn.b1_s = Dn.b0_s;
+  Dn.out_r = a.y;
+  Dn.out_s = a.y + (size_t)rows_r * a.D;
+  Dn.K_r = a.F; Dn.K_s = a.Fs;
+  Dn.N_r = a.D; Dn.N_s = a.D;
+  Dn.a_s_group_stride = a.T;
+  Dn.b_r_group_rows = a.D;
+  Dn.b_s_group_rows = a.D;
+  Dn.bn_out = nmma;
+  Dn.k_chunk = 0;
+  Dn.a_k_mod = 0;
+  Dn.gateup = 0;
+
+  p.offsets = a.offsets;
+  p.status = a.status;
+  p.counters = a.counters;
+  p.nprob = 2;
+  p.E = a.E; p.S = a.S; p.T = a.T;
+  p.rows_r = rows_r;
+  const int tiles_g = mt_upper * ((a.F + half - 1) / half) + a.S * mt_s * ((a.Fs + half - 1) / half);
   const int nt_d = (a.D + nmma - 1) / nmma;
   const int tiles_d = mt_upper * nt_d + a.S * mt_s * nt_d;
-  err = narrow ? launch_one<false, 128>(d, tiles_d, st) : launch_one<false, 256>(d, tiles_d, st);
-  if (err == cudaSuccess && marks) err = cudaEventRecord(static_cast<cudaEvent_t>(marks[1]), st);
-  *nlaunch += 2;
+  cudaError_t err = narrow ? launch_one<128>(p, tiles_g + tiles_d, st)
+                           : launch_one<256>(p, tiles_g + tiles_d, st);
+  if (err == cudaSuccess && marks) err = cudaEventRecord(static_cast<cudaEvent_t>(marks[0]), st);
+  *nlaunch += 1;
   return err;
 }
 

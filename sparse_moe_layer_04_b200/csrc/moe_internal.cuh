@@ -4,6 +4,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <utility>
 
 #include "../../include/moe_b200.h"
 
@@ -45,10 +46,30 @@ cudaError_t noalloc_scratch(int32_t** out);
 
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
 struct WsLayout {
-  size_t status, partials, wr3, idx, w, counts, offsets, perm, inv, blk_base, xperm, act_r,
-      act_s, y, total;
+  size_t status, partials, wr3, idx, w, counts, offsets, perm, inv, blk_base, counters, xperm,
+      act_r, act_s, y, total;
 };
 bool ws_layout(const moe_dims_t& d, WsLayout* out);
+
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while the previous kernel in the stream finishes; every kernel of the
+// library waits (griddepcontrol.wait) before it reads what earlier kernels
+// wrote, and lets its successor launch as soon as it starts.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // --- launchers (return cudaSuccess or the launch error) ---------------------
 cudaError_t launch_router_partials(const uint16_t* h, const float* Wr, int T, int D, int E,
@@ -64,8 +85,9 @@ cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T,
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* blk_base,
                            int* status, cudaStream_t st, int* nlaunch);
+// Also zeroes the expert FFN's per-group counters (`ncounters` ints).
 cudaError_t launch_gather_rows(const uint16_t* h, const int32_t* perm, int rows, int D, int T,
-                               uint16_t* xperm, cudaStream_t st);
+                               uint16_t* xperm, int* counters, int ncounters, cudaStream_t st);
 cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, int T, int D,
                            int k, int S, float* out, int* status, cudaStream_t st);
 
@@ -79,9 +101,10 @@ struct FfnArgs {
   uint16_t* act_s;          // [S*T, Fs]
   float* y;                 // [T*k + S*T, D]
   int* status;
+  int* counters;            // [E + S], zero at launch
   int T, D, E, F, k, S, Fs;
 };
-// `marks` (nullable): two events recorded after the gate/up and the down GEMM.
+// `marks` (nullable): one event recorded after the expert FFN kernel.
 cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch,
                               const char** why, void* const* marks);
 

@@ -14,6 +14,7 @@
 // Batches of at most 256 tokens (one counting block) run all three phases in
 // one launch.  All integer work: exact and deterministic.
 #include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 
@@ -22,6 +23,8 @@ constexpr int kWordsPerBlock = kPermBlockTokens / 32;
 __global__ void __launch_bounds__(kPermBlockTokens) permute_count_kernel(
     const int32_t* __restrict__ idx, int T, int E, int k, int32_t* __restrict__ blk_counts,
     int* __restrict__ status) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
   extern __shared__ int cnt[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -48,6 +51,8 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
                                                             int nblk, int E,
                                                             int32_t* __restrict__ counts,
                                                             int32_t* __restrict__ offsets) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;
   int total = 0;
@@ -91,6 +96,8 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
 __global__ void __launch_bounds__(kPermBlockTokens) permute_scatter_kernel(
     const int32_t* __restrict__ idx, int T, int E, int k, const int32_t* __restrict__ blk_base,
     int32_t* __restrict__ perm, int32_t* __restrict__ inv, int* __restrict__ status) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
   extern __shared__ unsigned mask[];  // [E][kWordsPerBlock]
   for (int i = threadIdx.x; i < E * kWordsPerBlock; i += blockDim.x) mask[i] = 0u;
   __syncthreads();
@@ -130,6 +137,8 @@ __global__ void __launch_bounds__(kPermBlockTokens) permute_single_block_kernel(
     const int32_t* __restrict__ idx, int T, int E, int k, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
     int* __restrict__ status) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
   extern __shared__ int sm[];
   int* cnt = sm;                                          // [E]
   unsigned* mask = reinterpret_cast<unsigned*>(sm + E);   // [E][kWordsPerBlock]
@@ -228,22 +237,20 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
   const int nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
   if (nblk == 1) {
     const size_t smem = (size_t)E * sizeof(int) + (size_t)E * kWordsPerBlock * sizeof(unsigned);
-    permute_single_block_kernel<<<1, kPermBlockTokens, smem, st>>>(idx, T, E, k, counts, offsets,
-                                                                   perm, inv, status);
     *nlaunch += 1;
-    return cudaGetLastError();
+    return launch_pdl(permute_single_block_kernel, dim3(1), dim3(kPermBlockTokens), smem, st, idx,
+                      T, E, k, counts, offsets, perm, inv, status);
   }
-  permute_count_kernel<<<nblk, kPermBlockTokens, E * sizeof(int), st>>>(idx, T, E, k, blk_base,
-                                                                         status);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_pdl(permute_count_kernel, dim3(nblk), dim3(kPermBlockTokens),
+                               E * sizeof(int), st, idx, T, E, k, blk_base, status);
   if (err != cudaSuccess) return err;
-  permute_scan_kernel<<<1, 1024, 0, st>>>(blk_base, nblk, E, counts, offsets);
-  err = cudaGetLastError();
+  err = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, st, blk_base, nblk, E, counts,
+                   offsets);
   if (err != cudaSuccess) return err;
-  permute_scatter_kernel<<<nblk, kPermBlockTokens, E * kWordsPerBlock * sizeof(unsigned), st>>>(
-      idx, T, E, k, blk_base, perm, inv, status);
   *nlaunch += 3;
-  return cudaGetLastError();
+  return launch_pdl(permute_scatter_kernel, dim3(nblk), dim3(kPermBlockTokens),
+                    E * kWordsPerBlock * sizeof(unsigned), st, idx, T, E, k,
+                    static_cast<const int32_t*>(blk_base), perm, inv, status);
 }
 
 // xperm[r] = h[perm[r]] for every grouped row r (16-byte vector copies).  A
@@ -251,7 +258,13 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ h,
                                                           const int32_t* __restrict__ perm,
                                                           int D, int T,
-                                                          uint16_t* __restrict__ xperm) {
+                                                          uint16_t* __restrict__ xperm,
+                                                          int* __restrict__ counters,
+                                                          int ncounters) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < ncounters; i += blockDim.x) counters[i] = 0;
   const int r = blockIdx.x;
   const int t = perm[r];
   uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)r * D);
@@ -264,10 +277,10 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 }
 
 cudaError_t launch_gather_rows(const uint16_t* h, const int32_t* perm, int rows, int D, int T,
-                               uint16_t* xperm, cudaStream_t st) {
+                               uint16_t* xperm, int* counters, int ncounters, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-  gather_rows_kernel<<<rows, 256, 0, st>>>(h, perm, D, T, xperm);
-  return cudaGetLastError();
+  return launch_pdl(gather_rows_kernel, dim3(rows), dim3(256), 0, st, h, perm, D, T, xperm,
+                    counters, ncounters);
 }
 
 }  // namespace moe

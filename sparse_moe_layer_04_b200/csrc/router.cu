@@ -17,6 +17,7 @@
 #include <climits>
 
 #include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 
@@ -57,6 +58,8 @@ RouterSplit router_split(int T, int D, int E) {
 // rounding.
 __global__ void split_router_kernel(const float* __restrict__ Wr, int E, int D,
                                     uint16_t* __restrict__ wr3) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
   const size_t n4 = (size_t)E * D / 4;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -90,8 +93,7 @@ cudaError_t launch_split_router(const float* Wr, int E, int D, uint16_t* wr3, cu
   const size_t n4 = (size_t)E * D / 4;
   size_t blocks = (n4 + 255) / 256;
   if (blocks > 2048) blocks = 2048;
-  split_router_kernel<<<(unsigned)blocks, 256, 0, st>>>(Wr, E, D, wr3);
-  return cudaGetLastError();
+  return launch_pdl(split_router_kernel, dim3((unsigned)blocks), dim3(256), 0, st, Wr, E, D, wr3);
 }
 
 // out[s][t][e] = sum over d in split s of h[t, d] * Wr[e, d], d ascending.
@@ -100,6 +102,8 @@ __global__ void __launch_bounds__(256) router_partials_kernel(const uint16_t* __
                                                               const float* __restrict__ Wr,
                                                               int T, int D, int E, int chunk,
                                                               float* __restrict__ out) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
   __shared__ __align__(16) float hs[kRouterTileD][kRouterTileT + 4];
   __shared__ __align__(16) float wsm[kRouterTileD][kRouterTileE + 4];
   const int tid = threadIdx.x;
@@ -177,6 +181,8 @@ __global__ void __launch_bounds__(256) router_partials_kernel(const uint16_t* __
 
 __global__ void reduce_partials_kernel(const float* __restrict__ p, int nsplit, size_t n,
                                        float* __restrict__ out) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x) {
     float v = p[i];
@@ -189,8 +195,7 @@ cudaError_t launch_router_partials(const uint16_t* h, const float* Wr, int T, in
                                    RouterSplit sp, float* out, cudaStream_t st) {
   dim3 grid((E + kRouterTileE - 1) / kRouterTileE, (T + kRouterTileT - 1) / kRouterTileT,
             sp.nsplit);
-  router_partials_kernel<<<grid, 256, 0, st>>>(h, Wr, T, D, E, sp.chunk, out);
-  return cudaGetLastError();
+  return launch_pdl(router_partials_kernel, grid, dim3(256), 0, st, h, Wr, T, D, E, sp.chunk, out);
 }
 
 cudaError_t launch_reduce_partials(const float* partials, int nsplit, size_t n, float* out,
@@ -199,8 +204,8 @@ cudaError_t launch_reduce_partials(const float* partials, int nsplit, size_t n, 
   size_t blocks = (n + threads - 1) / threads;
   if (blocks > 4096) blocks = 4096;
   if (blocks == 0) return cudaSuccess;
-  reduce_partials_kernel<<<(unsigned)blocks, threads, 0, st>>>(partials, nsplit, n, out);
-  return cudaGetLastError();
+  return launch_pdl(reduce_partials_kernel, dim3((unsigned)blocks), dim3(threads), 0, st, partials,
+                    nsplit, n, out);
 }
 
 // ---------------------------------------------------------------------------
@@ -237,6 +242,8 @@ __global__ void __launch_bounds__(1024) route_kernel(
     const float* __restrict__ src, int nsplit, const float* __restrict__ bias, int T, int E,
     int k, float scale, int32_t* __restrict__ idx, float* __restrict__ w,
     int* __restrict__ status) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
   __shared__ float c_key[kMaxSlots * kMaxSlots];
   __shared__ float c_sc[kMaxSlots * kMaxSlots];
   __shared__ int c_e[kMaxSlots * kMaxSlots];
@@ -318,8 +325,8 @@ __global__ void __launch_bounds__(1024) route_kernel(
 cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T, int E, int k,
                          float scale, int32_t* idx, float* w, int* status, cudaStream_t st) {
   const int threads = (E + 31) / 32 * 32;
-  route_kernel<<<T, threads, 0, st>>>(src, nsplit, bias, T, E, k, scale, idx, w, status);
-  return cudaGetLastError();
+  return launch_pdl(route_kernel, dim3(T), dim3(threads), 0, st, src, nsplit, bias, T, E, k, scale,
+                    idx, w, status);
 }
 
 }  // namespace moe
