@@ -211,8 +211,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     cfg = mi.CONFIGS[args.config]
-    if args.experts:
-        cfg = mi.custom_config(args.config, E=args.experts)
+    if args.experts or args.tokens:
+        cfg = mi.custom_config(args.config, E=args.experts or cfg.E, T=args.tokens or cfg.T)
     inp = mi.layer_weights(cfg, 0, device=dev)
     inp["h"] = mi.hidden(cfg, seed=rank, device=dev)
     d = moe.dims_of(cfg)
@@ -444,6 +444,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (small cases for profiler captures; not a bench line)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (small cases for profiler captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -31,7 +31,7 @@ RouterSplit router_split(int T, int D, int E) {
     const int kblocks = 3 * D / 64;
     const int bn = router_tile_n(T, E);
     const int tiles = ((T + 127) / 128) * ((E + bn - 1) / bn);
-    int want = (kSplitTargetBlocks + tiles - 1) / (tiles > 0 ? tiles : 1);
+    int want = kSplitTargetBlocks / (tiles > 0 ? tiles : 1);  // at most one wave
     want = want < 1 ? 1 : (want > 64 ? 64 : want);
     const int kb_per = (kblocks + want - 1) / want;
     sp.tensor = true;
@@ -322,11 +322,101 @@ __global__ void __launch_bounds__(1024) route_kernel(
   }
 }
 
+// Large batches: one warp per token (four tokens per block), each lane
+// holding the experts lane, lane + 32, ...; the same arithmetic in the same
+// order as route_kernel, so both give identical bits.
+template <int EPL>
+__global__ void __launch_bounds__(128) route_warp_kernel(
+    const float* __restrict__ src, int nsplit, const float* __restrict__ bias, int T, int E,
+    int k, float scale, int32_t* __restrict__ idx, float* __restrict__ w,
+    int* __restrict__ status) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const size_t plane = (size_t)T * E;
+  float key[EPL], sc[EPL];
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      const float* p = src + (size_t)t * E + e;
+      float l = p[0];
+      for (int s0 = 1; s0 < nsplit; s0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = (s0 + q < nsplit) ? p[(s0 + q) * plane] : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (s0 + q < nsplit) l = __fadd_rn(l, v[q]);
+      }
+      const double sd = 1.0 / (1.0 + exp(-(double)l));
+      sc[i] = __double2float_rn(sd);
+      key[i] = __fadd_rn(sc[i], bias[e]);
+      if (!isfinite(l) || !isfinite(key[i])) bad = true;
+    } else {
+      sc[i] = 0.f;
+      key[i] = -INFINITY;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0 && status) atomicOr(status, kStNonFinite);
+
+  unsigned taken = 0u;  // bit i: expert lane + 32 i already selected
+  int my_e = 0;
+  float my_s = 0.f, sum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float bk = -INFINITY, bs = 0.f;
+    int be = INT_MAX;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !(taken & (1u << i)) && precedes(key[i], e, bk, be)) {
+        bk = key[i];
+        be = e;
+        bs = sc[i];
+      }
+    }
+    warp_best(bk, be, bs);
+    if (be != INT_MAX && (be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == j) {
+      my_e = be;
+      my_s = bs;
+    }
+    sum = (j == 0) ? bs : __fadd_rn(sum, bs);
+  }
+  if (lane < k) {
+    idx[(size_t)t * k + lane] = my_e;
+    w[(size_t)t * k + lane] = __fmul_rn(__fdiv_rn(my_s, sum), scale);
+  }
+}
+
+template <int EPL>
+cudaError_t launch_route_warp(const float* src, int nsplit, const float* bias, int T, int E, int k,
+                              float scale, int32_t* idx, float* w, int* status, cudaStream_t st) {
+  return launch_pdl(route_warp_kernel<EPL>, dim3((T + 3) / 4), dim3(128), 0, st, src, nsplit, bias,
+                    T, E, k, scale, idx, w, status);
+}
+
+// Up to 1024 tokens: a block per token (more threads per token, shorter
+// chains); beyond that a warp per token.
+constexpr int kRouteBlockPerTokenMaxT = 1024;
+
 cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T, int E, int k,
                          float scale, int32_t* idx, float* w, int* status, cudaStream_t st) {
-  const int threads = (E + 31) / 32 * 32;
-  return launch_pdl(route_kernel, dim3(T), dim3(threads), 0, st, src, nsplit, bias, T, E, k, scale,
-                    idx, w, status);
+  if (T <= kRouteBlockPerTokenMaxT) {
+    const int threads = (E + 31) / 32 * 32;
+    return launch_pdl(route_kernel, dim3(T), dim3(threads), 0, st, src, nsplit, bias, T, E, k,
+                      scale, idx, w, status);
+  }
+  const int epl = (E + 31) / 32;
+  if (epl <= 1) return launch_route_warp<1>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
+  if (epl <= 2) return launch_route_warp<2>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
+  if (epl <= 4) return launch_route_warp<4>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
+  if (epl <= 8) return launch_route_warp<8>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
+  if (epl <= 16) return launch_route_warp<16>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
+  return launch_route_warp<32>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
 }
 
 }  // namespace moe

@@ -38,6 +38,8 @@ def _ws(moe, d):
 ROUTE_CASES = [
     (1, 8, 2, "normal"), (37, 8, 3, "grid"), (128, 256, 8, "normal"), (1000, 256, 8, "grid"),
     (64, 1024, 32, "normal"), (513, 64, 1, "normal"), (16, 32, 32, "grid"), (200, 40, 6, "normal"),
+    # more than 1024 tokens: the warp-per-token kernel
+    (2000, 256, 8, "grid"), (1500, 64, 6, "normal"), (1100, 1024, 32, "normal"), (1025, 8, 2, "grid"),
 ]
 
 
@@ -137,6 +139,10 @@ FFN_CASES = [
     (300, 1024, 32, 512, 8, 2, 256),   # two shared experts
     (130, 512, 8, 128, 2, 0, 0),       # no shared expert, ragged T
     (1, 136, 4, 64, 4, 1, 64),         # one token, D not a multiple of 64
+    # more than 512 tokens: the 256-wide tiles
+    (700, 256, 16, 192, 4, 1, 320),
+    (900, 384, 12, 320, 3, 2, 192),    # D not a multiple of the 256-wide tile
+    (600, 512, 8, 128, 2, 0, 0),
 ]
 
 
