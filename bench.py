@@ -40,6 +40,35 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ---------------------------------------------------------------------------
+# ranks: one process per GPU, one independent replica per rank
+# ---------------------------------------------------------------------------
+def rank_env():
+    """(rank, world, local_rank) from the torchrun environment (1 process if unset)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def replica_seed(rank: int) -> int:
+    """Seed of a rank's token batch: rank 0 runs the seed-0 workload the tests check."""
+    return rank
+
+
+def max_over_ranks(values, world: int, device="cpu"):
+    """Element-wise max of per-rank floats over all ranks (the slowest rank sets
+    the step time)."""
+    if world <= 1:
+        return list(values)
+    t = torch.tensor(list(values), device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_tokens_per_s(tokens_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's step time."""
+    return world * tokens_per_rank / (max_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # accounting
 # ---------------------------------------------------------------------------
 def layer_bytes_flops(cfg, U: int):
@@ -214,7 +243,7 @@ def run_ours(args, rank, world, local_rank):
     if args.experts or args.tokens:
         cfg = mi.custom_config(args.config, E=args.experts or cfg.E, T=args.tokens or cfg.T)
     inp = mi.layer_weights(cfg, 0, device=dev)
-    inp["h"] = mi.hidden(cfg, seed=rank, device=dev)
+    inp["h"] = mi.hidden(cfg, seed=replica_seed(rank), device=dev)
     d = moe.dims_of(cfg)
     ws = moe.alloc_workspace(d, dev)
     out = torch.empty((cfg.T, cfg.D), dtype=torch.float32, device=dev)
@@ -277,12 +306,7 @@ def run_ours(args, rank, world, local_rank):
     stage_ms = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K))
                 for j, name in enumerate(STAGES)}
     profiled_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][len(STAGES)]) for i in range(K))
-    ms = statistics.mean(step_ms)
-    ffn_ms = stage_ms["expert_ffn"]
-    if world > 1:
-        t = torch.tensor([ms, ffn_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, ffn_ms = t.tolist()
+    ms, ffn_ms = max_over_ranks([statistics.mean(step_ms), stage_ms["expert_ffn"]], world, dev)
 
     counts = torch.bincount(idx.flatten().long(), minlength=cfg.E)
     U = int((counts > 0).sum().item())
@@ -305,11 +329,7 @@ def run_ours(args, rank, world, local_rank):
         b.synchronize()
         if i >= 3:
             e2e_ms.append(a.elapsed_time(b))
-    e2e = statistics.mean(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e = t.item()
+    e2e = max_over_ranks([statistics.mean(e2e_ms)], world, dev)[0]
 
     if rank != 0:
         return None
@@ -340,7 +360,7 @@ def run_ours(args, rank, world, local_rank):
 
     res = {
         "metric": METRIC,
-        "value": world * cfg.T / t_s,
+        "value": aggregate_tokens_per_s(cfg.T, world, ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
@@ -369,7 +389,7 @@ def run_ours(args, rank, world, local_rank):
             "frac": max(t_roof_hbm, t_roof_tc) / t_s,
             "hbm_frac": t_roof_hbm / t_s, "tensor_frac": t_roof_tc / t_s,
             "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "source": peak_src}},
-        "e2e": {"value": world * cfg.T / (e2e / 1e3), "unit": "tokens/s",
+        "e2e": {"value": aggregate_tokens_per_s(cfg.T, world, e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": cfg.T * cfg.D * 2, "d2h_bytes_per_step": cfg.T * cfg.D * 4,
                 "ms_per_step": e2e},
         "gpu_launches": launches_per_step * K,
@@ -450,9 +470,7 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local_rank = rank_env()
 
     if args.impl == "reference":
         if rank != 0:

@@ -184,6 +184,28 @@ int moe_forward(const void* h, const float* Wr, const float* bias, const void* W
                 const void* Ws2, const moe_dims_t* dims, float* out, int32_t* idx_out,
                 float* w_out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Routing statistics of the last moe_forward (or moe_permute) that used
+ * `ws` with these dims: device pointers into the workspace, valid once the
+ * stream has reached the end of that call and until the next call reuses the
+ * workspace (the "Inside GLM" course outline's Sparse execution lesson names
+ * routed-expert utilisation as a quantity to inspect).
+ *   moe_ws_expert_counts   -> int32 [E]: pairs routed to each expert (the
+ *                             per-expert load histogram)
+ *   moe_ws_touched_experts -> int32 [1]: experts with at least one pair
+ * Pointer arithmetic only (no launch, no synchronisation); NULL if ws is NULL
+ * or the dims are invalid. */
+const int32_t* moe_ws_expert_counts(const void* ws, const moe_dims_t* dims);
+const int32_t* moe_ws_touched_experts(const void* ws, const moe_dims_t* dims);
+
+/* Self-test of the bounded device waits (failure detection without a fault):
+ * one kernel waits on an mbarrier that nothing arrives on and on a counter
+ * that nothing increments, using the same bounded-wait code as the layer's
+ * kernels; each wait gives up after about one second.  It records
+ * MOE_ERR_TIMEOUT in the status word at the start of `ws` (read it with
+ * moe_get_device_status) and returns; the CUDA context stays usable.  Takes
+ * about two seconds of GPU time.  `ws` needs at least 256 bytes. */
+int moe_selftest_bounded_wait(void* ws, moe_stream_t stream);
+
 /* Synchronises `stream`, returns the first error recorded in the status word
  * of `ws` (MOE_OK if none) and clears the word. */
 int moe_get_device_status(void* ws, moe_stream_t stream);

@@ -71,6 +71,9 @@ def _load() -> ctypes.CDLL:
         "moe_combine": (I, [P, P, P, D, P, P, P]),
         "moe_forward": (I, [P, P, P, P, P, P, P, P, P, D, P, P, P, P, Z, P]),
         "moe_get_device_status": (I, [P, P]),
+        "moe_selftest_bounded_wait": (I, [P, P]),
+        "moe_ws_expert_counts": (P, [P, D]),
+        "moe_ws_touched_experts": (P, [P, D]),
         "moe_last_error": (ctypes.c_char_p, []),
         "moe_last_launch_count": (I, []),
         "moe_set_profile_events": (I, [ctypes.POINTER(P), I]),
@@ -189,6 +192,30 @@ def moe_forward(h, Wr, bias, W1, W3, W2, Ws1, Ws3, Ws2, d, out, ws, idx_out=None
 def moe_get_device_status(ws, stream=None) -> int:
     """Synchronises the stream; returns (and clears) the first device-side error code."""
     return _lib.moe_get_device_status(_ptr(ws, torch.uint8, "ws"), _stream(stream))
+
+
+def moe_ws_expert_counts(ws, d) -> torch.Tensor:
+    """int32 [E] view of the per-expert load histogram kept in the workspace."""
+    addr = _lib.moe_ws_expert_counts(_ptr(ws, torch.uint8, "ws"), ctypes.byref(d))
+    return _view_int32(ws, addr, d.E)
+
+
+def moe_ws_touched_experts(ws, d) -> torch.Tensor:
+    """int32 [1] view of the touched-expert count kept in the workspace."""
+    addr = _lib.moe_ws_touched_experts(_ptr(ws, torch.uint8, "ws"), ctypes.byref(d))
+    return _view_int32(ws, addr, 1)
+
+
+def _view_int32(ws: torch.Tensor, addr: int, n: int) -> torch.Tensor:
+    if not addr:
+        raise MoeError(MOE_ERR_INVALID_ARG, "invalid workspace or dims")
+    off = addr - ws.data_ptr()
+    return ws[off: off + 4 * n].view(torch.int32)
+
+
+def moe_selftest_bounded_wait(ws, stream=None) -> None:
+    """Runs the bounded-wait self-test; moe_get_device_status then reports MOE_ERR_TIMEOUT."""
+    _check(_lib.moe_selftest_bounded_wait(_ptr(ws, torch.uint8, "ws"), _stream(stream)))
 
 
 def moe_last_error() -> str:

@@ -170,6 +170,7 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
   L->act_r = take(T * k * F * 2);
   L->act_s = take(S * T * Fs * 2);
   L->y = take((T * k + S * T) * D * 4);
+  L->touched = take(4);
   L->total = off;
   return true;
 }
@@ -277,7 +278,8 @@ int moe_permute(const int32_t* idx, const moe_dims_t* dims, int32_t* counts, int
   if ((rc = check_device())) return rc;
   int n = 0;
   cudaError_t e = launch_permute(idx, dims->T, dims->E, dims->k, counts, offsets, perm, inv,
-                                 w.at<int32_t>(w.L.blk_base), w.status(), st, &n);
+                                 w.at<int32_t>(w.L.blk_base), w.status(),
+                                 w.at<int32_t>(w.L.touched), st, &n);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   g_launches = n;
   return MOE_OK;
@@ -311,7 +313,7 @@ int moe_permute_noalloc(const int32_t* idx, const moe_dims_t* dims, int32_t* cou
   if (e != cudaSuccess) return cuda_fail(e, "moe_permute_noalloc: scratch address lookup");
   int n = 0;
   e = launch_permute(idx, dims->T, dims->E, dims->k, counts, offsets, perm, inv, scratch,
-                     nullptr, st, &n);
+                     nullptr, nullptr, st, &n);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   g_launches = n;
   return MOE_OK;
@@ -442,7 +444,7 @@ int moe_forward(const void* h, const float* Wr, const float* bias, const void* W
   if (e != cudaSuccess) return cuda_fail(e, "route launch");
   n += 1;
   e = launch_permute(idx, T, E, k, counts, offsets, perm, inv, w.at<int32_t>(w.L.blk_base),
-                     w.status(), st, &n);
+                     w.status(), w.at<int32_t>(w.L.touched), st, &n);
   if (e == cudaSuccess) e = mark(3, st);
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
@@ -475,6 +477,35 @@ int moe_forward(const void* h, const float* Wr, const float* bias, const void* W
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   n += 1;
   g_launches = n;
+  return MOE_OK;
+}
+
+const int32_t* moe_ws_expert_counts(const void* ws, const moe_dims_t* dims) {
+  if (!ws || check_dims(dims) != MOE_OK) return nullptr;
+  WsLayout L;
+  ws_layout(*dims, &L);
+  return reinterpret_cast<const int32_t*>(static_cast<const uint8_t*>(ws) + L.counts);
+}
+
+const int32_t* moe_ws_touched_experts(const void* ws, const moe_dims_t* dims) {
+  if (!ws || check_dims(dims) != MOE_OK) return nullptr;
+  WsLayout L;
+  ws_layout(*dims, &L);
+  return reinterpret_cast<const int32_t*>(static_cast<const uint8_t*>(ws) + L.touched);
+}
+
+int moe_selftest_bounded_wait(void* ws, moe_stream_t stream) {
+  g_err.clear();
+  g_launches = 0;
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) & 255u)
+    return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  int rc = check_device();
+  if (rc) return rc;
+  cudaError_t e = launch_bounded_wait_selftest(static_cast<int*>(ws),
+                                               reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  g_launches = 1;
   return MOE_OK;
 }
 

@@ -208,21 +208,6 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, volat
   if (!ptx::mbar_wait(bar, parity, &ignore_abort)) *abort = 1;
 }
 
-// Waits until *ctr >= target (acquire), bounded like the mbarrier waits.
-__device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatile int* abort) {
-  if (ptx::ld_acquire_gpu(ctr) >= target) return true;
-  const long long t0 = clock64();
-  for (;;) {
-    __nanosleep(128);
-    if (ptx::ld_acquire_gpu(ctr) >= target) return true;
-    if (*abort) return false;
-    if (clock64() - t0 > ptx::kWaitBudgetCycles) {
-      *abort = 1;
-      return false;
-    }
-  }
-}
-
 template <int MMA_N>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   using Sh = Shape<MMA_N>;
@@ -320,7 +305,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           const int g = ti.shared ? p.E + ti.grp : ti.grp;
           const int nt0 = ti.shared ? col_tiles(p.pr[0].N_s, p.pr[0].bn_out)
                                     : col_tiles(p.pr[0].N_r, p.pr[0].bn_out);
-          if (!wait_counter(p.counters + g, EPI_WARPS * ti.mt * nt0, abort)) break;
+          if (!ptx::counter_wait(p.counters + g, EPI_WARPS * ti.mt * nt0, abort)) break;
           ptx::fence_proxy_async_global();
         }
         const CUtensorMap* amap = ti.shared ? &P.a_s : &P.a_r;

@@ -47,7 +47,7 @@ cudaError_t noalloc_scratch(int32_t** out);
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
 struct WsLayout {
   size_t status, partials, wr3, idx, w, counts, offsets, perm, inv, blk_base, counters, xperm,
-      act_r, act_s, y, total;
+      act_r, act_s, y, touched, total;
 };
 bool ws_layout(const moe_dims_t& d, WsLayout* out);
 
@@ -82,9 +82,10 @@ cudaError_t launch_reduce_partials(const float* partials, int nsplit, size_t n, 
                                    cudaStream_t st);
 cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T, int E, int k,
                          float scale, int32_t* idx, float* w, int* status, cudaStream_t st);
+// `touched` (nullable): number of experts with at least one pair.
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* blk_base,
-                           int* status, cudaStream_t st, int* nlaunch);
+                           int* status, int32_t* touched, cudaStream_t st, int* nlaunch);
 // Also zeroes the expert FFN's per-group counters (`ncounters` ints).
 cudaError_t launch_gather_rows(const uint16_t* h, const int32_t* perm, int rows, int D, int T,
                                uint16_t* xperm, int* counters, int ncounters, cudaStream_t st);
@@ -109,5 +110,7 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch,
                               const char** why, void* const* marks);
 
 int num_sms();
+
+cudaError_t launch_bounded_wait_selftest(int* status, cudaStream_t st);
 
 }  // namespace moe

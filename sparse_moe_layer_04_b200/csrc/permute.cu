@@ -50,7 +50,8 @@ __global__ void __launch_bounds__(kPermBlockTokens) permute_count_kernel(
 __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ blk_base,
                                                             int nblk, int E,
                                                             int32_t* __restrict__ counts,
-                                                            int32_t* __restrict__ offsets) {
+                                                            int32_t* __restrict__ offsets,
+                                                            int32_t* __restrict__ touched) {
   ptx::pdl_launch_dependents();
   ptx::pdl_wait();
   __shared__ int warp_sums[32];
@@ -91,6 +92,8 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
     if (e == E - 1) offsets[E] = excl + total;
     for (int b = 0; b < nblk; ++b) blk_base[(size_t)b * E + e] += excl;
   }
+  const int nz = __syncthreads_count(e < E && total > 0);
+  if (touched && e == 0) *touched = nz;
 }
 
 __global__ void __launch_bounds__(kPermBlockTokens) permute_scatter_kernel(
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(kPermBlockTokens) permute_scatter_kernel(
 __global__ void __launch_bounds__(kPermBlockTokens) permute_single_block_kernel(
     const int32_t* __restrict__ idx, int T, int E, int k, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-    int* __restrict__ status) {
+    int* __restrict__ status, int32_t* __restrict__ touched) {
   ptx::pdl_launch_dependents();
   ptx::pdl_wait();
   extern __shared__ int sm[];
@@ -180,14 +183,24 @@ __global__ void __launch_bounds__(kPermBlockTokens) permute_single_block_kernel(
   int base = incl - local;
   for (int q = 0; q < wid; ++q) base += warp_tot[q];
   __syncthreads();  // everyone has read warp_tot; cnt becomes the offsets
+  int nz = 0;
   for (int e = e0; e < e0 + per && e < E; ++e) {
     const int c = cnt[e];
     counts[e] = c;
     offsets[e] = base;
     cnt[e] = base;
     base += c;
+    nz += c > 0;
   }
   if (threadIdx.x == kPermBlockTokens - 1) offsets[E] = base;  // the last thread ends at the total
+  if (touched) {  // block sum of the per-thread counts of experts with pairs
+    __shared__ int nz_total;
+    if (threadIdx.x == 0) nz_total = 0;
+    __syncthreads();
+    if (nz) atomicAdd(&nz_total, nz);
+    __syncthreads();
+    if (threadIdx.x == 0) *touched = nz_total;
+  }
   __syncthreads();
   if (t < T && !bad) {
     for (int j = 0; j < k; ++j) {
@@ -233,19 +246,19 @@ cudaError_t noalloc_scratch(int32_t** out) {
 
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* blk_base,
-                           int* status, cudaStream_t st, int* nlaunch) {
+                           int* status, int32_t* touched, cudaStream_t st, int* nlaunch) {
   const int nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
   if (nblk == 1) {
     const size_t smem = (size_t)E * sizeof(int) + (size_t)E * kWordsPerBlock * sizeof(unsigned);
     *nlaunch += 1;
     return launch_pdl(permute_single_block_kernel, dim3(1), dim3(kPermBlockTokens), smem, st, idx,
-                      T, E, k, counts, offsets, perm, inv, status);
+                      T, E, k, counts, offsets, perm, inv, status, touched);
   }
   cudaError_t err = launch_pdl(permute_count_kernel, dim3(nblk), dim3(kPermBlockTokens),
                                E * sizeof(int), st, idx, T, E, k, blk_base, status);
   if (err != cudaSuccess) return err;
   err = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, st, blk_base, nblk, E, counts,
-                   offsets);
+                   offsets, touched);
   if (err != cudaSuccess) return err;
   *nlaunch += 3;
   return launch_pdl(permute_scatter_kernel, dim3(nblk), dim3(kPermBlockTokens),

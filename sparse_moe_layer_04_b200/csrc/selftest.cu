@@ -1,0 +1,40 @@
+// Self-test of the bounded device waits.  Every wait in the library's kernels
+// (mbarrier phases inside a CTA, completion counters between CTAs) gives up
+// after a clock budget of about a second, reports MOE_ERR_TIMEOUT through the
+// workspace status word and lets the kernel return, so a lost arrival never
+// hangs the GPU.  This kernel makes both kinds of wait run out on purpose:
+// it waits on an mbarrier that nothing arrives on and on a counter that
+// nothing increments, with the same helpers the kernels use.
+#include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace {
+
+__device__ int g_never_incremented = 0;  // no code ever writes it
+
+__global__ void bounded_wait_selftest_kernel(int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort = 0;
+    ptx::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool got_phase = ptx::mbar_wait(&bar, 0, &abort);  // no arrival will come
+    abort = 0;
+    const bool got_count = ptx::counter_wait(&g_never_incremented, 1, &abort);
+    if (!got_phase && !got_count && status) atomicOr(status, kStTimeout);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bounded_wait_selftest(int* status, cudaStream_t st) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -176,6 +176,22 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   return v;
 }
 
+// Waits until *ctr >= target (acquire), bounded like mbar_wait: gives up when
+// the clock budget runs out (raising *abort) or when *abort is already set.
+__device__ __forceinline__ bool counter_wait(const int* ctr, int target, volatile int* abort) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Descriptors
 // ---------------------------------------------------------------------------

@@ -337,11 +337,15 @@ def test_forward_glm52_full_size(moe, glm52, name, n):
     if name != "skew":
         inp["bias"] = mi.correction_bias(cfg, 0, device="cuda")
     inp["h"] = mi.hidden(cfg, 0, device="cuda")
-    out, idx, _, _ = _forward(moe, cfg, inp)
+    out, idx, _, ws = _forward(moe, cfg, inp)
     assert torch.isfinite(out.float()).all()
     _check_layer(cfg, inp, out, idx, _sample(cfg.T, n, name))
-    # the routed load the workload describes: skew follows the stored Zipf bias
+    # the routed load the workload describes: skew follows the stored Zipf bias;
+    # the histogram kept in the workspace matches the returned indices
     counts = torch.bincount(idx.flatten().long(), minlength=cfg.E).cpu().numpy()
+    d = moe.dims_of(cfg)
+    assert np.array_equal(moe.moe_ws_expert_counts(ws, d).cpu().numpy(), counts)
+    assert int(moe.moe_ws_touched_experts(ws, d).item()) == int((counts > 0).sum())
     if name == "skew":
         assert (counts == 0).sum() >= 16 and counts.max() > 10 * counts.mean()
 
@@ -400,3 +404,16 @@ def test_status_bad_offsets(moe):
     moe.moe_expert_ffn(inp["h"], perm, offsets, inp["W1"], inp["W3"], inp["W2"], None, None, None,
                        d, y, ws)
     assert moe.moe_get_device_status(ws) == moe.MOE_ERR_BOUNDS
+
+
+def test_bounded_wait_times_out_and_the_context_survives(moe):
+    """A wait that can never end gives up after its clock budget and reports
+    MOE_ERR_TIMEOUT; the next layer call on the same context still works."""
+    d = moe.dims(T=4, D=64, E=8, F=64, k=2)
+    ws = _ws(moe, d)
+    moe.moe_selftest_bounded_wait(ws)
+    assert moe.moe_get_device_status(ws) == moe.MOE_ERR_TIMEOUT
+    cfg = mi.CONFIGS["tiny"]
+    inp = layer_on_device(cfg)
+    out, idx, _, _ = _forward(moe, cfg, inp)
+    _check_layer(cfg, inp, out, idx, np.arange(8))
