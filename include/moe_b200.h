@@ -108,6 +108,20 @@ int moe_router_logits(const void* h, const float* Wr, const moe_dims_t* dims, fl
 int moe_route(const float* logits, const float* bias, const moe_dims_t* dims, int32_t* idx,
               float* w, void* ws, moe_stream_t stream);
 
+/* Group-limited routing ("GLM-4.5 Full Forward", How it works: sigmoid group
+ * routing; the pages give neither the rule nor the group counts, so both
+ * are parameters and the rule is the reading documented here).  The E
+ * experts form n_group contiguous groups of E / n_group.  A group's score is
+ * the fp32 sum of its two largest selection keys (its one key for one-expert
+ * groups); the topk_group groups first under (score descending, group index
+ * ascending) are kept; then idx and w are exactly those of moe_route with
+ * the other experts' keys set to -infinity.  n_group = 1 or topk_group =
+ * n_group gives moe_route's result.  Limits: 1 <= n_group <= 32, n_group
+ * divides E, 1 <= topk_group <= n_group, k <= topk_group * E / n_group.
+ * Arguments, layout and errors as moe_route. */
+int moe_route_grouped(const float* logits, const float* bias, const moe_dims_t* dims, int n_group,
+                      int topk_group, int32_t* idx, float* w, void* ws, moe_stream_t stream);
+
 /* Grouping of the (token, slot) pairs by expert (counting sort; the pages
  * call the expert kernels "grouped"):
  *   counts[e]  = number of pairs routed to expert e            [E] int32

@@ -31,6 +31,8 @@ from .moe_oracle import (  # noqa: F401
     select_topk,
     routing_weights,
     route,
+    route_grouped,
+    group_scores,
     routing_alternatives,
     swiglu_expert,
     group_by_expert,

@@ -109,6 +109,49 @@ def route(logits: np.ndarray, bias: np.ndarray, k: int, scale: float
     return idx, routing_weights(s, idx, scale)
 
 
+def group_scores(keys: np.ndarray, n_group: int) -> np.ndarray:
+    """Score of each contiguous expert group: the sum of its two largest
+    selection keys (one fp32 add), or its single key for one-expert groups.
+
+    "GLM-4.5 Full Forward" (How it works) names sigmoid *group* routing
+    without its rule or group counts; this is the reading taken: experts are
+    cut into n_group equal contiguous groups ranked by their two best keys.
+    """
+    keys = np.asarray(keys, F32)
+    T, E = keys.shape
+    if n_group < 1 or E % n_group:
+        raise ValueError("n_group must divide E")
+    g = keys.reshape(T, n_group, E // n_group)
+    if g.shape[2] == 1:
+        return g[:, :, 0].astype(F32)
+    top2 = -np.sort(-g, axis=2)[:, :, :2]
+    return (top2[:, :, 0] + top2[:, :, 1]).astype(F32)
+
+
+def route_grouped(logits: np.ndarray, bias: np.ndarray, k: int, scale: float, n_group: int,
+                  topk_group: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Group-limited routing: keep the topk_group groups that come first under
+    (group score descending, group index ascending), then select the top-k
+    experts inside them exactly as route() does; weights from the un-biased
+    scores.  n_group = 1 (or topk_group = n_group) is plain routing.
+    """
+    s = sigmoid_scores(logits)
+    keys = selection_keys(s, bias)
+    T, E = keys.shape
+    if not 1 <= topk_group <= n_group:
+        raise ValueError("need 1 <= topk_group <= n_group")
+    if k > topk_group * (E // n_group):
+        raise ValueError("k exceeds the experts of the kept groups")
+    gs = group_scores(keys, n_group)
+    keep = np.argsort(-gs, axis=1, kind="stable")[:, :topk_group]
+    allowed = np.zeros((T, n_group), bool)
+    np.put_along_axis(allowed, keep, True, axis=1)
+    mask = np.repeat(allowed, E // n_group, axis=1)
+    masked = np.where(mask, keys, F32(-np.inf)).astype(F32)
+    idx = select_topk(masked, k)
+    return idx, routing_weights(s, idx, scale)
+
+
 def routing_alternatives(logits_row: np.ndarray, bias: np.ndarray, k: int, scale: float,
                          delta: float):
     """Every routing of one token that is correct up to a logit perturbation.

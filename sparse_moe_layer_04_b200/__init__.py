@@ -65,6 +65,7 @@ def _load() -> ctypes.CDLL:
         "moe_workspace_size": (Z, [D]),
         "moe_router_logits": (I, [P, P, D, P, P, Z, P]),
         "moe_route": (I, [P, P, D, P, P, P, P]),
+        "moe_route_grouped": (I, [P, P, D, I, I, P, P, P, P]),
         "moe_permute": (I, [P, D, P, P, P, P, P, Z, P]),
         "moe_permute_noalloc": (I, [P, D, P, P, P, P, P]),
         "moe_expert_ffn": (I, [P, P, P, P, P, P, P, P, P, D, P, P, Z, P]),
@@ -141,6 +142,14 @@ def moe_route(logits, bias, d, idx, w, ws=None, stream=None) -> None:
     _check(_lib.moe_route(_ptr(logits, torch.float32, "logits"), _ptr(bias, torch.float32, "bias"),
                           ctypes.byref(d), _ptr(idx, torch.int32, "idx"),
                           _ptr(w, torch.float32, "w"), wp, _stream(stream)))
+
+
+def moe_route_grouped(logits, bias, d, n_group, topk_group, idx, w, ws=None, stream=None) -> None:
+    wp, _ = _ws(ws)
+    _check(_lib.moe_route_grouped(_ptr(logits, torch.float32, "logits"),
+                                  _ptr(bias, torch.float32, "bias"), ctypes.byref(d), n_group,
+                                  topk_group, _ptr(idx, torch.int32, "idx"),
+                                  _ptr(w, torch.float32, "w"), wp, _stream(stream)))
 
 
 def moe_permute(idx, d, counts, offsets, perm, inv, ws, stream=None) -> None:

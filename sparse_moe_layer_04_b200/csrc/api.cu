@@ -255,6 +255,37 @@ int moe_route(const float* logits, const float* bias, const moe_dims_t* dims, in
   return MOE_OK;
 }
 
+int moe_route_grouped(const float* logits, const float* bias, const moe_dims_t* dims, int n_group,
+                      int topk_group, int32_t* idx, float* w, void* ws, moe_stream_t stream) {
+  int rc = begin(dims);
+  if (rc) return rc;
+  if (n_group < 1 || n_group > 32 || dims->E % n_group)
+    return fail(MOE_ERR_INVALID_ARG, "n_group = %d must divide E = %d and be in [1, 32]", n_group,
+                dims->E);
+  if (topk_group < 1 || topk_group > n_group)
+    return fail(MOE_ERR_INVALID_ARG, "topk_group = %d outside [1, n_group]", topk_group);
+  if ((long long)dims->k > (long long)topk_group * (dims->E / n_group))
+    return fail(MOE_ERR_INVALID_ARG, "k = %d exceeds the %d experts of the kept groups", dims->k,
+                topk_group * (dims->E / n_group));
+  if (dims->T == 0) return MOE_OK;
+  MOE_CHECK_PTR(logits);
+  MOE_CHECK_PTR(bias);
+  MOE_CHECK_PTR(idx);
+  MOE_CHECK_PTR(w);
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  WsLayout L;
+  ws_layout(*dims, &L);
+  int* status = ws ? reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status) : nullptr;
+  if ((rc = check_device())) return rc;
+  cudaError_t e = launch_route_grouped(logits, bias, dims->T, dims->E, dims->k, dims->scale, n_group,
+                                       topk_group, idx, w, status,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "grouped route launch");
+  g_launches = 1;
+  return MOE_OK;
+}
+
 int moe_permute(const int32_t* idx, const moe_dims_t* dims, int32_t* counts, int32_t* offsets,
                 int32_t* perm, int32_t* inv, void* ws, size_t ws_bytes, moe_stream_t stream) {
   int rc = begin(dims);

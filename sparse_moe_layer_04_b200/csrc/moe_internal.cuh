@@ -83,6 +83,9 @@ cudaError_t launch_reduce_partials(const float* partials, int nsplit, size_t n, 
 cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T, int E, int k,
                          float scale, int32_t* idx, float* w, int* status, cudaStream_t st);
 // `touched` (nullable): number of experts with at least one pair.
+cudaError_t launch_route_grouped(const float* logits, const float* bias, int T, int E, int k,
+                                 float scale, int n_group, int topk_group, int32_t* idx, float* w,
+                                 int* status, cudaStream_t st);
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* blk_base,
                            int* status, int32_t* touched, cudaStream_t st, int* nlaunch);

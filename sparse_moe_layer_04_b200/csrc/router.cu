@@ -233,47 +233,18 @@ __device__ __forceinline__ void warp_best(float& bk, int& be, float& bs) {
 
 constexpr int kMaxSlots = 32;
 
-// Thread e sums expert e's partial-sum planes in plane order, takes the
-// sigmoid in fp64 (rounded once to fp32) and adds the bias.  Each warp then
-// extracts its k best (key, index) pairs by warp arg-max rounds; the union
-// of the warps' lists holds the token's top k, which warp 0 extracts the same
-// way, in selection order.  The weights use the un-biased scores.
-__global__ void __launch_bounds__(1024) route_kernel(
-    const float* __restrict__ src, int nsplit, const float* __restrict__ bias, int T, int E,
-    int k, float scale, int32_t* __restrict__ idx, float* __restrict__ w,
-    int* __restrict__ status) {
-  ptx::pdl_launch_dependents();
-  ptx::pdl_wait();
-  __shared__ float c_key[kMaxSlots * kMaxSlots];
-  __shared__ float c_sc[kMaxSlots * kMaxSlots];
-  __shared__ int c_e[kMaxSlots * kMaxSlots];
-  const int t = blockIdx.x;
-  const int e = threadIdx.x;
-  const int lane = e & 31, wid = e >> 5, nw = blockDim.x >> 5;
-  const size_t plane = (size_t)T * E;
-  int bad = 0;
-
-  float key = -INFINITY, sc = 0.f;
-  int me = INT_MAX;
-  if (e < E) {
-    const float* p = src + (size_t)t * E + e;
-    float l = p[0];
-    for (int s0 = 1; s0 < nsplit; s0 += 16) {
-      float v[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) v[q] = (s0 + q < nsplit) ? p[(s0 + q) * plane] : 0.f;
-#pragma unroll
-      for (int q = 0; q < 16; ++q)
-        if (s0 + q < nsplit) l = __fadd_rn(l, v[q]);
-    }
-    const double sd = 1.0 / (1.0 + exp(-(double)l));
-    sc = __double2float_rn(sd);
-    key = __fadd_rn(sc, bias[e]);
-    me = e;
-    bad = !isfinite(l) || !isfinite(key);
-  }
-
-  // per-warp top-k candidates
+// Top-k of one token held one expert per thread (key, score, index; threads
+// past E hold -inf / INT_MAX), in the block's shared candidate arrays: each
+// warp extracts its k best (key, index) pairs by warp arg-max rounds; the
+// union of the warps' lists holds the token's top k, which warp 0 extracts
+// the same way, in selection order, and writes with the renormalised weights
+// (un-biased scores, fp32 sum in slot order, one division and one multiply).
+// Must be called by every thread of the block.
+__device__ __forceinline__ void block_topk_write(float key, float sc, int me, int t, int k,
+                                                 float scale, int32_t* __restrict__ idx,
+                                                 float* __restrict__ w, float* c_key,
+                                                 float* c_sc, int* c_e) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
   bool taken = false;
   for (int j = 0; j < k; ++j) {
     float bk = taken ? -INFINITY : key;
@@ -287,10 +258,8 @@ __global__ void __launch_bounds__(1024) route_kernel(
     }
     if (be == me) taken = true;
   }
-  if (__syncthreads_or(bad) && e == 0 && status) atomicOr(status, kStNonFinite);
+  __syncthreads();
   if (wid != 0) return;
-
-  // warp 0: the token's top k among the nw * k candidates
   const int nc = nw * k;
   unsigned done = 0u;  // bit q: candidate lane + 32 q already selected
   int my_e = 0;
@@ -320,6 +289,108 @@ __global__ void __launch_bounds__(1024) route_kernel(
     idx[(size_t)t * k + lane] = my_e;
     w[(size_t)t * k + lane] = __fmul_rn(__fdiv_rn(my_s, sum), scale);
   }
+}
+
+// Sum of expert e's logit planes in plane order, its sigmoid (fp64, rounded
+// once to fp32) and its selection key.  Returns false for a non-finite value.
+__device__ __forceinline__ bool score_and_key(const float* __restrict__ src, int nsplit,
+                                              size_t plane, size_t at, float b, float* sc,
+                                              float* key) {
+  const float* p = src + at;
+  float l = p[0];
+  for (int s0 = 1; s0 < nsplit; s0 += 16) {
+    float v[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) v[q] = (s0 + q < nsplit) ? p[(s0 + q) * plane] : 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (s0 + q < nsplit) l = __fadd_rn(l, v[q]);
+  }
+  const double sd = 1.0 / (1.0 + exp(-(double)l));
+  *sc = __double2float_rn(sd);
+  *key = __fadd_rn(*sc, b);
+  return isfinite(l) && isfinite(*key);
+}
+
+// Routing with one block per token, one thread per expert.
+__global__ void __launch_bounds__(1024) route_kernel(
+    const float* __restrict__ src, int nsplit, const float* __restrict__ bias, int T, int E,
+    int k, float scale, int32_t* __restrict__ idx, float* __restrict__ w,
+    int* __restrict__ status) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
+  __shared__ float c_key[kMaxSlots * kMaxSlots];
+  __shared__ float c_sc[kMaxSlots * kMaxSlots];
+  __shared__ int c_e[kMaxSlots * kMaxSlots];
+  const int t = blockIdx.x;
+  const int e = threadIdx.x;
+  float key = -INFINITY, sc = 0.f;
+  int me = INT_MAX, bad = 0;
+  if (e < E) {
+    bad = !score_and_key(src, nsplit, (size_t)T * E, (size_t)t * E + e, bias[e], &sc, &key);
+    me = e;
+  }
+  if (__syncthreads_or(bad) && e == 0 && status) atomicOr(status, kStNonFinite);
+  block_topk_write(key, sc, me, t, k, scale, idx, w, c_key, c_sc, c_e);
+}
+
+// Group-limited routing: experts form n_group contiguous groups of E/n_group;
+// a group's score is the sum of its two largest keys (its one key for
+// one-expert groups); the topk_group groups first under (score descending,
+// group index ascending) are kept and the top k is taken among their experts.
+__global__ void __launch_bounds__(1024) route_grouped_kernel(
+    const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
+    float scale, int n_group, int topk_group, int32_t* __restrict__ idx, float* __restrict__ w,
+    int* __restrict__ status) {
+  ptx::pdl_launch_dependents();
+  ptx::pdl_wait();
+  __shared__ float c_key[kMaxSlots * kMaxSlots];
+  __shared__ float c_sc[kMaxSlots * kMaxSlots];
+  __shared__ int c_e[kMaxSlots * kMaxSlots];
+  __shared__ float s_key[1024];
+  __shared__ float g_score[32];
+  __shared__ int g_keep[32];
+  const int t = blockIdx.x;
+  const int e = threadIdx.x;
+  const int lane = e & 31;
+  float key = -INFINITY, sc = 0.f;
+  int me = INT_MAX, bad = 0;
+  if (e < E) {
+    bad = !score_and_key(logits, 1, 0, (size_t)t * E + e, bias[e], &sc, &key);
+    me = e;
+    s_key[e] = key;
+  }
+  if (__syncthreads_or(bad) && e == 0 && status) atomicOr(status, kStNonFinite);
+  const int G = E / n_group;
+  if (e < n_group) {
+    float a = -INFINITY, b = -INFINITY;  // two largest keys of group e
+    for (int i = e * G; i < (e + 1) * G; ++i) {
+      const float v = s_key[i];
+      if (v > a) {
+        b = a;
+        a = v;
+      } else if (v > b) {
+        b = v;
+      }
+    }
+    g_score[e] = (G == 1) ? a : __fadd_rn(a, b);
+    g_keep[e] = 0;
+  }
+  __syncthreads();
+  if (e < 32) {
+    bool taken = false;
+    for (int j = 0; j < topk_group; ++j) {
+      float bk = (lane < n_group && !taken) ? g_score[lane] : -INFINITY;
+      int be = (lane < n_group && !taken) ? lane : INT_MAX;
+      float unused = 0.f;
+      warp_best(bk, be, unused);
+      if (be == lane) taken = true;
+    }
+    if (lane < n_group) g_keep[lane] = taken ? 1 : 0;
+  }
+  __syncthreads();
+  if (e < E && !g_keep[e / G]) key = -INFINITY;
+  block_topk_write(key, sc, me, t, k, scale, idx, w, c_key, c_sc, c_e);
 }
 
 // Large batches: one warp per token (four tokens per block), each lane
@@ -397,6 +468,14 @@ cudaError_t launch_route_warp(const float* src, int nsplit, const float* bias, i
                               float scale, int32_t* idx, float* w, int* status, cudaStream_t st) {
   return launch_pdl(route_warp_kernel<EPL>, dim3((T + 3) / 4), dim3(128), 0, st, src, nsplit, bias,
                     T, E, k, scale, idx, w, status);
+}
+
+cudaError_t launch_route_grouped(const float* logits, const float* bias, int T, int E, int k,
+                                 float scale, int n_group, int topk_group, int32_t* idx, float* w,
+                                 int* status, cudaStream_t st) {
+  const int threads = (E + 31) / 32 * 32;
+  return launch_pdl(route_grouped_kernel, dim3(T), dim3(threads < 32 ? 32 : threads), 0, st,
+                    logits, bias, T, E, k, scale, n_group, topk_group, idx, w, status);
 }
 
 // Up to 1024 tokens: a block per token (more threads per token, shorter

@@ -104,6 +104,15 @@ def test_bad_dims_rejected(mod):
     assert rc == mod.MOE_ERR_INVALID_ARG
 
 
+def test_grouped_route_argument_checks(mod):
+    lib = mod._lib
+    d = mod.dims(T=8, D=128, E=12, F=64, k=4)
+    for n_group, topk_group in [(5, 1), (0, 1), (33, 1), (4, 5), (4, 0), (6, 1)]:
+        rc = lib.moe_route_grouped(FAKE, FAKE, ctypes.byref(d), n_group, topk_group, FAKE, FAKE,
+                                   None, None)
+        assert rc == mod.MOE_ERR_INVALID_ARG, (n_group, topk_group)
+
+
 def test_binding_names_match_the_abi(mod):
     for n in _declared_functions():
         assert hasattr(mod, n), n

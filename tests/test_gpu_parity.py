@@ -62,6 +62,43 @@ def test_route_bit_exact(moe, T, E, k, dist):
     assert np.array_equal(w.cpu().numpy().view(np.uint32), rw.view(np.uint32))
 
 
+GROUPED_CASES = [
+    (128, 256, 8, 8, 4, "normal"), (300, 256, 8, 8, 2, "grid"), (64, 64, 6, 4, 2, "normal"),
+    (77, 160, 4, 32, 3, "grid"), (50, 1024, 32, 32, 16, "normal"), (40, 12, 3, 12, 3, "normal"),  # one-expert groups
+]
+
+
+@pytest.mark.parametrize("T,E,k,n_group,topk_group,dist", GROUPED_CASES)
+def test_route_grouped_bit_exact(moe, T, E, k, n_group, topk_group, dist):
+    name = f"groute{T}x{E}x{n_group}"
+    logits = mi.synthetic_logits(T, E, 1.5, 0, name)
+    bias = mi.normal((E,), 0.1, 0, name + "/bias")
+    if dist == "grid":
+        logits = torch.round(logits * 4) / 4
+        bias = torch.round(bias * 16) / 16
+    d = moe.dims(T=T, D=64, E=E, F=64, k=k, scale=2.5)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    ws = _ws(moe, d)
+    moe.moe_route_grouped(logits.cuda(), bias.cuda(), d, n_group, topk_group, idx, w, ws)
+    assert moe.moe_get_device_status(ws) == 0
+    ridx, rw = orc.route_grouped(logits.numpy(), bias.numpy(), k, 2.5, n_group, topk_group)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.array_equal(w.cpu().numpy().view(np.uint32), rw.view(np.uint32))
+
+
+def test_route_grouped_single_group_equals_route(moe):
+    T, E, k = 200, 256, 8
+    logits = mi.synthetic_logits(T, E, 1.5, 0, "g1").cuda()
+    bias = mi.normal((E,), 0.1, 0, "g1/bias").cuda()
+    d = moe.dims(T=T, D=64, E=E, F=64, k=k)
+    outs = [(torch.empty((T, k), dtype=torch.int32, device="cuda"),
+             torch.empty((T, k), device="cuda")) for _ in range(2)]
+    moe.moe_route(logits, bias, d, *outs[0])
+    moe.moe_route_grouped(logits, bias, d, 1, 1, *outs[1])
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
 def test_route_zero_router_tie(moe):
     T, E, k = 9, 64, 8
     d = moe.dims(T=T, D=64, E=E, F=64, k=k, scale=2.5)

@@ -211,3 +211,59 @@ def test_routing_alternatives_cover_near_ties():
         c = orc.routing_alternatives(lg, b, 4, 2.5, delta=0.0)
         idx, w = orc.route(lg[None, :], b, 4, 2.5)
         assert len(c) == 1 and np.array_equal(c[0][0], idx[0]) and np.array_equal(c[0][1], w[0])
+
+
+# ---------------------------------------------------------------------------
+# group-limited routing
+# ---------------------------------------------------------------------------
+def _brute_grouped(keys_row, k, n_group, topk_group):
+    """Every choice of topk_group groups, ranked by the group scores computed
+    with sorted() on Python floats; the experts by brute-force top-k inside."""
+    E = len(keys_row)
+    G = E // n_group
+    scores = []
+    for g in range(n_group):
+        ks = sorted((float(v) for v in keys_row[g * G:(g + 1) * G]), reverse=True)
+        scores.append(float(F32(ks[0]) + F32(ks[1])) if G > 1 else ks[0])
+    groups = sorted(range(n_group), key=lambda g: (-scores[g], g))[:topk_group]
+    allowed = [e for g in sorted(groups) for e in range(g * G, (g + 1) * G)]
+    sub = [keys_row[e] for e in allowed]
+    picked = _brute_topk(sub, k)
+    return [allowed[i] for i in picked]
+
+
+@pytest.mark.parametrize("E,k,n_group,topk_group", [(8, 2, 4, 2), (12, 3, 3, 1), (8, 4, 2, 2),
+                                                    (16, 4, 8, 3), (6, 2, 6, 4)])
+def test_grouped_routing_matches_brute_force(E, k, n_group, topk_group):
+    rng = np.random.default_rng(50 + E + k)
+    for trial in range(40):
+        if trial % 4 == 0:
+            logits = (rng.integers(-2, 3, size=(1, E)) / 2.0).astype(F32)   # ties
+        else:
+            logits = rng.standard_normal((1, E)).astype(F32)
+        bias = (rng.standard_normal(E) * 0.1).astype(F32)
+        idx, w = orc.route_grouped(logits, bias, k, 2.5, n_group, topk_group)
+        keys = orc.selection_keys(orc.sigmoid_scores(logits), bias)[0].tolist()
+        assert idx[0].tolist() == _brute_grouped(keys, k, n_group, topk_group)
+        assert abs(float(w[0].astype(np.float64).sum()) - 2.5) < 4 * k * 2.4e-7
+
+
+def test_grouped_routing_degenerate_cases_are_plain_routing():
+    rng = np.random.default_rng(77)
+    logits = rng.standard_normal((64, 32)).astype(F32)
+    bias = (rng.standard_normal(32) * 0.1).astype(F32)
+    ref = orc.route(logits, bias, 6, 2.5)
+    for n_group, topk_group in [(1, 1), (4, 4), (32, 32)]:
+        got = orc.route_grouped(logits, bias, 6, 2.5, n_group, topk_group)
+        assert np.array_equal(got[0], ref[0]) and np.array_equal(got[1], ref[1])
+
+
+def test_grouped_routing_keeps_experts_inside_the_best_groups():
+    # group 1 (experts 4..7) has the two best keys; with topk_group = 1 every
+    # selected expert must come from it even though expert 0 has a high key
+    s = np.array([[0.9, 0.1, 0.1, 0.1, 0.8, 0.85, 0.2, 0.3]], F32)
+    logits = np.log(s / (1 - s)).astype(F32)
+    idx, w = orc.route_grouped(logits, np.zeros(8, F32), 2, 1.0, 2, 1)
+    assert sorted(idx[0].tolist()) == [4, 5]
+    idx2, _ = orc.route_grouped(logits, np.zeros(8, F32), 2, 1.0, 2, 2)
+    assert idx2[0].tolist() == [0, 5]
