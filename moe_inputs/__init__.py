@@ -244,3 +244,55 @@ def load_bias_file(path: str, E: int) -> torch.Tensor:
 
 def bias_file_path(cfg: LayerConfig) -> Optional[str]:
     return None if cfg.skew_bias_file is None else os.path.join(_HERE, cfg.skew_bias_file)
+
+
+# ----------------------------------------------------------------------------
+# FP8 weights (E4M3 codes, one power-of-two scale per 128 x 128 block)
+# ----------------------------------------------------------------------------
+FP8_BLOCK = 128
+FP8_MAX = 448.0
+
+
+def quantize_fp8_blocks(w: torch.Tensor):
+    """E4M3 codes and block exponents of a weight matrix [..., rows, K].
+
+    For each 128 x 128 block (ragged at the edges) the exponent e is the
+    smallest integer with max|w| <= 448 * 2**e (0 for an all-zero block); the
+    codes are torch's round-to-nearest-even float8_e4m3fn cast of w * 2**-e.
+    The weight the codes stand for, code * 2**e, is exactly a bf16 value.
+    Returns (codes uint8 [..., rows, K], exps int8 [..., ceil(rows/128), ceil(K/128)]).
+    """
+    *lead, R, K = w.shape
+    RB, KB = -(-R // FP8_BLOCK), -(-K // FP8_BLOCK)
+    wf = w.float()
+    pad = torch.zeros(*lead, RB * FP8_BLOCK, KB * FP8_BLOCK, dtype=torch.float32, device=w.device)
+    pad[..., :R, :K] = wf.abs()
+    amax = pad.reshape(*lead, RB, FP8_BLOCK, KB, FP8_BLOCK).amax(dim=(-3, -1)).double()
+    e = torch.ceil(torch.log2(torch.clamp(amax, min=1e-300) / FP8_MAX))
+    lim = FP8_MAX * torch.pow(2.0, e)
+    e = torch.where(amax > lim, e + 1, e)                       # exact corrections
+    e = torch.where(amax <= FP8_MAX * torch.pow(2.0, e - 1), e - 1, e)
+    e = torch.where(amax == 0, torch.zeros_like(e), e)
+    exps = e.to(torch.int8)
+    scale = torch.pow(2.0, -e).float()
+    full = scale.repeat_interleave(FP8_BLOCK, dim=-2).repeat_interleave(FP8_BLOCK, dim=-1)
+    codes = (wf * full[..., :R, :K]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), exps.contiguous()
+
+
+def fp8_layer_weights(weights: dict) -> dict:
+    """FP8 copies of the expert weights of `layer_weights`: for each of W1,
+    W3, W2, Ws1, Ws3, Ws2 the codes ("W1q" ...) and block exponents ("W1e" ...),
+    on the weights' device.  Quantized one expert at a time, so the
+    temporaries stay the size of one expert matrix."""
+    out = {}
+    for name in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2"):
+        w = weights[name]
+        parts = [quantize_fp8_blocks(w[g]) for g in range(w.shape[0])]
+        R, K = w.shape[-2:]
+        out[name + "q"] = (torch.stack([c for c, _ in parts]) if parts else
+                           torch.empty((0, R, K), dtype=torch.uint8, device=w.device))
+        out[name + "e"] = (torch.stack([e for _, e in parts]) if parts else
+                           torch.empty((0, -(-R // FP8_BLOCK), -(-K // FP8_BLOCK)),
+                                       dtype=torch.int8, device=w.device))
+    return out

@@ -35,6 +35,8 @@ from .moe_oracle import (  # noqa: F401
     group_scores,
     routing_alternatives,
     swiglu_expert,
+    e4m3_value,
+    dequantize_fp8_blocks,
     group_by_expert,
     combine,
     moe_layer,

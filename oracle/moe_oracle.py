@@ -204,6 +204,33 @@ def swiglu_expert(x: np.ndarray, w1: np.ndarray, w3: np.ndarray, w2: np.ndarray)
 
 
 # ----------------------------------------------------------------------------
+# FP8 expert weights
+# ----------------------------------------------------------------------------
+
+def e4m3_value(code: np.ndarray) -> np.ndarray:
+    """Value of an OCP E4M3 (float8_e4m3fn) code, from the format definition:
+    sign bit, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0 is
+    subnormal (m * 2**-9); S.1111.111 is NaN; there is no infinity."""
+    c = np.asarray(code, np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def dequantize_fp8_blocks(codes: np.ndarray, exps: np.ndarray, block: int = 128) -> np.ndarray:
+    """w = e4m3_value(code) * 2**e with one exponent per block x block tile
+    of the last two dimensions (the weights an FP8 layer stands for)."""
+    codes = np.asarray(codes)
+    exps = np.asarray(exps, np.int64)
+    R, K = codes.shape[-2:]
+    scale = np.exp2(np.repeat(np.repeat(exps, block, axis=-2), block, axis=-1)[..., :R, :K])
+    return e4m3_value(codes) * scale
+
+
+# ----------------------------------------------------------------------------
 # grouping by expert and merging
 # ----------------------------------------------------------------------------
 
