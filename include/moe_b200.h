@@ -198,6 +198,63 @@ int moe_forward(const void* h, const float* Wr, const float* bias, const void* W
                 const void* Ws2, const moe_dims_t* dims, float* out, int32_t* idx_out,
                 float* w_out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* ---- FP8 expert weights ------------------------------------------------
+ * The "Inside GLM" course outline names BF16 and FP8 GLM-5.2 artifacts (its
+ * outcomes list and the Release anatomy lesson) but gives no FP8 layout;
+ * this library's is: each expert matrix [rows, K] is stored as
+ * OCP E4M3 (float8_e4m3fn) codes [rows, K] plus one int8 exponent e per
+ * 128 x 128 block ([ceil(rows/128), ceil(K/128)], ragged at the edges), and
+ * stands for the weights  w = e4m3(code) * 2^e.  Every such w is exactly a
+ * bf16 value for e in [-117, 7]; exponents outside that range, and the NaN
+ * codes 0x7F / 0xFF, are outside the format (an exponent outside the range
+ * raises MOE_ERR_BOUNDS in the workspace status word; NaN codes are not
+ * detected).  Activations stay bf16: the FP8 layer computes exactly what the
+ * bf16 layer computes on the decoded weights, with half the weight bytes.
+ *
+ * Code pointers must be 16-byte aligned; exponent pointers have no
+ * alignment rule.  Ws* members may be NULL when S = 0.  The pointed-to
+ * arrays are read only, and owned by the caller. */
+typedef struct moe_fp8_weights {
+  const void* W1;   /* [E, F, D] E4M3 codes */
+  const void* W3;   /* [E, F, D] */
+  const void* W2;   /* [E, D, F] */
+  const void* Ws1;  /* [S, Fs, D] */
+  const void* Ws3;  /* [S, Fs, D] */
+  const void* Ws2;  /* [S, D, Fs] */
+  const int8_t* W1e;   /* [E, ceil(F/128), ceil(D/128)] block exponents */
+  const int8_t* W3e;   /* [E, ceil(F/128), ceil(D/128)] */
+  const int8_t* W2e;   /* [E, ceil(D/128), ceil(F/128)] */
+  const int8_t* Ws1e;  /* [S, ceil(Fs/128), ceil(D/128)] */
+  const int8_t* Ws3e;  /* [S, ceil(Fs/128), ceil(D/128)] */
+  const int8_t* Ws2e;  /* [S, ceil(D/128), ceil(Fs/128)] */
+} moe_fp8_weights_t;
+
+/* moe_expert_ffn with FP8 expert weights (`w8`, device arrays as described
+ * above).  Same rows, outputs, workspace and errors as moe_expert_ffn; in
+ * addition D, F and Fs (when S > 0) must be multiples of 16 (MOE_ERR_INVALID_ARG
+ * otherwise). */
+int moe_expert_ffn_fp8(const void* h, const int32_t* perm, const int32_t* offsets,
+                       const moe_fp8_weights_t* w8, const moe_dims_t* dims, float* y, void* ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward with FP8 expert weights: the same pipeline and outputs, with
+ * moe_expert_ffn_fp8 in place of moe_expert_ffn (router weight Wr stays
+ * fp32).  Same argument rules as moe_forward plus those of
+ * moe_expert_ffn_fp8. */
+int moe_forward_fp8(const void* h, const float* Wr, const float* bias, const moe_fp8_weights_t* w8,
+                    const moe_dims_t* dims, float* out, int32_t* idx_out, float* w_out, void* ws,
+                    size_t ws_bytes, moe_stream_t stream);
+
+/* Decodes FP8 weights to bf16 with the same exact decoding the FP8 layer
+ * uses: codes [G, R, K] (16-byte aligned), exps [G, ceil(R/128), ceil(K/128)]
+ * -> out [G, R, K] bf16 (16-byte aligned), out[g, r, c] = e4m3(code) *
+ * 2^exps[g, r/128, c/128].  K must be a multiple of 16.  An exponent outside
+ * [-117, 7] raises MOE_ERR_BOUNDS in the status word of `ws` (ws may be
+ * NULL: then it is not reported).  G, R, K >= 0; nothing is launched when
+ * one is 0. */
+int moe_fp8_dequantize(const void* codes, const int8_t* exps, int G, int R, int K, void* out,
+                       void* ws, moe_stream_t stream);
+
 /* Routing statistics of the last moe_forward (or moe_permute) that used
  * `ws` with these dims: device pointers into the workspace, valid once the
  * stream has reached the end of that call and until the next call reuses the

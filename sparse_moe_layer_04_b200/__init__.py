@@ -54,6 +54,13 @@ def dims_of(cfg, T: Optional[int] = None) -> moe_dims_t:
                       cfg.scale)
 
 
+class moe_fp8_weights_t(ctypes.Structure):
+    """FP8 expert weights: E4M3 code arrays and int8 block-exponent arrays
+    (device pointers; see moe_fp8_weights_t in include/moe_b200.h)."""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2",
+                                                "W1e", "W3e", "W2e", "Ws1e", "Ws3e", "Ws2e")]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
@@ -61,6 +68,7 @@ def _load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     D = ctypes.POINTER(moe_dims_t)
+    W8 = ctypes.POINTER(moe_fp8_weights_t)
     sig = {
         "moe_workspace_size": (Z, [D]),
         "moe_router_logits": (I, [P, P, D, P, P, Z, P]),
@@ -78,6 +86,9 @@ def _load() -> ctypes.CDLL:
         "moe_last_error": (ctypes.c_char_p, []),
         "moe_last_launch_count": (I, []),
         "moe_set_profile_events": (I, [ctypes.POINTER(P), I]),
+        "moe_expert_ffn_fp8": (I, [P, P, P, W8, D, P, P, Z, P]),
+        "moe_forward_fp8": (I, [P, P, P, W8, D, P, P, P, P, Z, P]),
+        "moe_fp8_dequantize": (I, [P, P, I, I, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -177,6 +188,60 @@ def moe_expert_ffn(h, perm, offsets, W1, W3, W2, Ws1, Ws3, Ws2, d, y, ws, stream
                                _ptr(W3, bf, "W3"), _ptr(W2, bf, "W2"), _ptr(Ws1, bf, "Ws1"),
                                _ptr(Ws3, bf, "Ws3"), _ptr(Ws2, bf, "Ws2"), ctypes.byref(d),
                                _ptr(y, torch.float32, "y"), wp, wn, _stream(stream)))
+
+
+_CODE_DTYPES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _code_ptr(t: Optional[torch.Tensor], name: str) -> Optional[int]:
+    if t is not None and t.dtype not in _CODE_DTYPES:
+        raise TypeError(f"{name}: expected uint8 or float8_e4m3fn codes, got {t.dtype}")
+    return _ptr(t, None, name)
+
+
+def fp8_weights(W1, W3, W2, Ws1, Ws3, Ws2, W1e, W3e, W2e, Ws1e, Ws3e, Ws2e) -> moe_fp8_weights_t:
+    """Packs FP8 code tensors (uint8 or float8_e4m3fn) and their int8 block
+    exponents into the struct the FP8 entry points take.  The struct holds raw
+    pointers: keep the tensors alive while it is in use."""
+    w = moe_fp8_weights_t()
+    for name, t in (("W1", W1), ("W3", W3), ("W2", W2), ("Ws1", Ws1), ("Ws3", Ws3), ("Ws2", Ws2)):
+        setattr(w, name, _code_ptr(t, name))
+    for name, t in (("W1e", W1e), ("W3e", W3e), ("W2e", W2e), ("Ws1e", Ws1e), ("Ws3e", Ws3e),
+                    ("Ws2e", Ws2e)):
+        setattr(w, name, _ptr(t, torch.int8, name))
+    return w
+
+
+def moe_expert_ffn_fp8(h, perm, offsets, w8: moe_fp8_weights_t, d, y, ws, stream=None) -> None:
+    wp, wn = _ws(ws)
+    _check(_lib.moe_expert_ffn_fp8(_ptr(h, torch.bfloat16, "h"), _ptr(perm, torch.int32, "perm"),
+                                   _ptr(offsets, torch.int32, "offsets"), ctypes.byref(w8),
+                                   ctypes.byref(d), _ptr(y, torch.float32, "y"), wp, wn,
+                                   _stream(stream)))
+
+
+def moe_forward_fp8(h, Wr, bias, w8: moe_fp8_weights_t, d, out, ws, idx_out=None, w_out=None,
+                    stream=None) -> None:
+    wp, wn = _ws(ws)
+    _check(_lib.moe_forward_fp8(_ptr(h, torch.bfloat16, "h"), _ptr(Wr, torch.float32, "Wr"),
+                                _ptr(bias, torch.float32, "bias"), ctypes.byref(w8),
+                                ctypes.byref(d), _ptr(out, torch.float32, "out"),
+                                _ptr(idx_out, torch.int32, "idx_out"),
+                                _ptr(w_out, torch.float32, "w_out"), wp, wn, _stream(stream)))
+
+
+def moe_fp8_dequantize(codes, exps, out, ws=None, stream=None) -> None:
+    """codes [G, R, K] (or [R, K]) E4M3, exps [G, ceil(R/128), ceil(K/128)]
+    int8 -> out bf16 of the codes' shape."""
+    if codes.dim() not in (2, 3):
+        raise ValueError("codes: expected [R, K] or [G, R, K]")
+    G, R, K = (1, *codes.shape) if codes.dim() == 2 else tuple(codes.shape)
+    if tuple(out.shape) != tuple(codes.shape):
+        raise ValueError("out: expected the shape of codes")
+    wp, _ = _ws(ws)
+    _check(_lib.moe_fp8_dequantize(_code_ptr(codes, "codes"), _ptr(exps, torch.int8, "exps"),
+                                   G, R, K, _ptr(out, torch.bfloat16, "out"), wp,
+                                   _stream(stream)))
 
 
 def moe_combine(y, w, inv, d, out, ws=None, stream=None) -> None:

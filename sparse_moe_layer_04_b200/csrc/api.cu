@@ -175,6 +175,191 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
   return true;
 }
 
+namespace {
+
+// Expert weights of one call: bf16 matrices, or FP8 codes + exponents.
+struct ExpertWeights {
+  const uint16_t *W1 = nullptr, *W3 = nullptr, *W2 = nullptr, *Ws1 = nullptr, *Ws3 = nullptr,
+                 *Ws2 = nullptr;
+  bool fp8 = false;
+  Fp8Weights f8{};
+};
+
+int check_bf16_weights(const void* W1, const void* W3, const void* W2, const void* Ws1,
+                       const void* Ws3, const void* Ws2, const moe_dims_t* dims,
+                       ExpertWeights* out) {
+  MOE_CHECK_PTR(W1);
+  MOE_CHECK_PTR(W3);
+  MOE_CHECK_PTR(W2);
+  if (dims->S > 0) {
+    MOE_CHECK_PTR(Ws1);
+    MOE_CHECK_PTR(Ws3);
+    MOE_CHECK_PTR(Ws2);
+  }
+  out->W1 = static_cast<const uint16_t*>(W1);
+  out->W3 = static_cast<const uint16_t*>(W3);
+  out->W2 = static_cast<const uint16_t*>(W2);
+  out->Ws1 = static_cast<const uint16_t*>(Ws1);
+  out->Ws3 = static_cast<const uint16_t*>(Ws3);
+  out->Ws2 = static_cast<const uint16_t*>(Ws2);
+  out->fp8 = false;
+  return MOE_OK;
+}
+
+// FP8 weight rows are D, F or Fs bytes long: TMA needs 16-byte row strides.
+int check_fp8_dims(const moe_dims_t* d) {
+  if (d->D % 16) return fail(MOE_ERR_INVALID_ARG, "FP8 weights: D = %d not a multiple of 16", d->D);
+  if (d->F % 16) return fail(MOE_ERR_INVALID_ARG, "FP8 weights: F = %d not a multiple of 16", d->F);
+  if (d->S > 0 && d->Fs % 16)
+    return fail(MOE_ERR_INVALID_ARG, "FP8 weights: Fs = %d not a multiple of 16", d->Fs);
+  return MOE_OK;
+}
+
+#define MOE_CHECK_EXP(p)                                                           \
+  do {                                                                             \
+    if (!(w8->p)) return fail(MOE_ERR_INVALID_ARG, "w8->%s is NULL", #p);          \
+  } while (0)
+
+int check_fp8_weights(const moe_fp8_weights_t* w8, const moe_dims_t* dims, ExpertWeights* out) {
+  if (!w8) return fail(MOE_ERR_INVALID_ARG, "w8 is NULL");
+  const void* W1 = w8->W1;
+  const void* W3 = w8->W3;
+  const void* W2 = w8->W2;
+  MOE_CHECK_PTR(W1);
+  MOE_CHECK_PTR(W3);
+  MOE_CHECK_PTR(W2);
+  MOE_CHECK_EXP(W1e);
+  MOE_CHECK_EXP(W3e);
+  MOE_CHECK_EXP(W2e);
+  const int8_t *W1e = w8->W1e, *W3e = w8->W3e, *W2e = w8->W2e;
+  const void *Ws1 = w8->Ws1, *Ws3 = w8->Ws3, *Ws2 = w8->Ws2;
+  const int8_t *Ws1e = w8->Ws1e, *Ws3e = w8->Ws3e, *Ws2e = w8->Ws2e;
+  if (dims->S > 0) {
+    MOE_CHECK_PTR(Ws1);
+    MOE_CHECK_PTR(Ws3);
+    MOE_CHECK_PTR(Ws2);
+    if (!Ws1e || !Ws3e || !Ws2e) return fail(MOE_ERR_INVALID_ARG, "w8->Ws*e is NULL with S > 0");
+  }
+  out->fp8 = true;
+  out->f8.W1 = static_cast<const uint8_t*>(W1);
+  out->f8.W3 = static_cast<const uint8_t*>(W3);
+  out->f8.W2 = static_cast<const uint8_t*>(W2);
+  out->f8.Ws1 = static_cast<const uint8_t*>(Ws1);
+  out->f8.Ws3 = static_cast<const uint8_t*>(Ws3);
+  out->f8.Ws2 = static_cast<const uint8_t*>(Ws2);
+  out->f8.W1e = W1e; out->f8.W3e = W3e; out->f8.W2e = W2e;
+  out->f8.Ws1e = Ws1e; out->f8.Ws3e = Ws3e; out->f8.Ws2e = Ws2e;
+  return MOE_OK;
+}
+
+FfnArgs ffn_args(const uint16_t* h, const uint16_t* xperm, const int32_t* offsets,
+                 const ExpertWeights& wt, const Ws& w, float* y, int32_t* counters,
+                 const moe_dims_t* d) {
+  FfnArgs a;
+  a.xperm = xperm;
+  a.h = h;
+  a.offsets = offsets;
+  a.W1 = wt.W1; a.W3 = wt.W3; a.W2 = wt.W2;
+  a.Ws1 = wt.Ws1; a.Ws3 = wt.Ws3; a.Ws2 = wt.Ws2;
+  a.act_r = w.at<uint16_t>(w.L.act_r);
+  a.act_s = w.at<uint16_t>(w.L.act_s);
+  a.y = y;
+  a.status = w.status();
+  a.counters = counters;
+  a.T = d->T; a.D = d->D; a.E = d->E; a.F = d->F; a.k = d->k; a.S = d->S; a.Fs = d->Fs;
+  return a;
+}
+
+cudaError_t launch_ffn(const FfnArgs& a, const ExpertWeights& wt, cudaStream_t st, int* n,
+                       const char** why, void* const* marks) {
+  return wt.fp8 ? launch_expert_ffn_fp8(a, wt.f8, st, n, why, marks)
+                : launch_expert_ffn(a, st, n, why, marks);
+}
+
+int expert_ffn_impl(const void* h, const int32_t* perm, const int32_t* offsets,
+                    const ExpertWeights& wt, const moe_dims_t* dims, float* y, void* ws,
+                    size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK_PTR(h);
+  MOE_CHECK_PTR(perm);
+  MOE_CHECK_PTR(offsets);
+  MOE_CHECK_PTR(y);
+  Ws w;
+  int rc;
+  if ((rc = check_ws(dims, ws, ws_bytes, &w))) return rc;
+  if ((rc = check_device())) return rc;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int rows = dims->T * dims->k;
+  const auto* hb = static_cast<const uint16_t*>(h);
+  uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
+  int32_t* counters = w.at<int32_t>(w.L.counters);
+  cudaError_t e = launch_gather_rows(hb, perm, rows, dims->D, dims->T, xperm, counters,
+                                     dims->E + dims->S, st);
+  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  const FfnArgs a = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
+  int n = 1;
+  const char* why = "launch failed";
+  e = launch_ffn(a, wt, st, &n, &why, nullptr);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
+  g_launches = n;
+  return MOE_OK;
+}
+
+int forward_impl(const void* h, const float* Wr, const float* bias, const ExpertWeights& wt,
+                 const moe_dims_t* dims, float* out, int32_t* idx_out, float* w_out, void* ws,
+                 size_t ws_bytes, moe_stream_t stream) {
+  MOE_CHECK_PTR(out);
+  if (idx_out && !aligned16(idx_out)) return fail(MOE_ERR_INVALID_ARG, "idx_out is not 16-byte aligned");
+  if (w_out && !aligned16(w_out)) return fail(MOE_ERR_INVALID_ARG, "w_out is not 16-byte aligned");
+  Ws w;
+  int rc;
+  if ((rc = check_ws(dims, ws, ws_bytes, &w))) return rc;
+  if ((rc = check_device())) return rc;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int T = dims->T, D = dims->D, E = dims->E, k = dims->k;
+  const auto* hb = static_cast<const uint16_t*>(h);
+  int32_t* idx = idx_out ? idx_out : w.at<int32_t>(w.L.idx);
+  float* rw = w_out ? w_out : w.at<float>(w.L.w);
+  int32_t* counts = w.at<int32_t>(w.L.counts);
+  int32_t* offsets = w.at<int32_t>(w.L.offsets);
+  int32_t* perm = w.at<int32_t>(w.L.perm);
+  int32_t* inv = w.at<int32_t>(w.L.inv);
+  float* y = w.at<float>(w.L.y);
+  int n = 0;
+
+  const RouterSplit sp = router_split(T, D, E);
+  float* partials = w.at<float>(w.L.partials);
+  const char* rwhy = "router launch";
+  cudaError_t e = mark(0, st);
+  if (e == cudaSuccess) e = launch_router(hb, Wr, *dims, sp, w, partials, st, &n, &rwhy);
+  if (e == cudaSuccess) e = mark(1, st);
+  if (e != cudaSuccess) return cuda_fail(e, rwhy);
+  e = launch_route(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw, w.status(), st);
+  if (e == cudaSuccess) e = mark(2, st);
+  if (e != cudaSuccess) return cuda_fail(e, "route launch");
+  n += 1;
+  e = launch_permute(idx, T, E, k, counts, offsets, perm, inv, w.at<int32_t>(w.L.blk_base),
+                     w.status(), w.at<int32_t>(w.L.touched), st, &n);
+  if (e == cudaSuccess) e = mark(3, st);
+  if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
+  int32_t* counters = w.at<int32_t>(w.L.counters);
+  e = launch_gather_rows(hb, perm, T * k, D, T, xperm, counters, E + dims->S, st);
+  if (e == cudaSuccess) e = mark(4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  n += 1;
+  const FfnArgs a = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
+  const char* why = "launch failed";
+  e = launch_ffn(a, wt, st, &n, &why, g_prof_events ? g_prof_events + 5 : nullptr);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
+  e = launch_combine(y, rw, inv, T, D, k, dims->S, out, w.status(), st);
+  if (e == cudaSuccess) e = mark(6, st);
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  n += 1;
+  g_launches = n;
+  return MOE_OK;
+}
+
+}  // namespace
 }  // namespace moe
 
 using namespace moe;
@@ -357,51 +542,21 @@ int moe_expert_ffn(const void* h, const int32_t* perm, const int32_t* offsets, c
   int rc = begin(dims);
   if (rc) return rc;
   if (dims->T == 0) return MOE_OK;
-  MOE_CHECK_PTR(h);
-  MOE_CHECK_PTR(perm);
-  MOE_CHECK_PTR(offsets);
-  MOE_CHECK_PTR(W1);
-  MOE_CHECK_PTR(W3);
-  MOE_CHECK_PTR(W2);
-  MOE_CHECK_PTR(y);
-  if (dims->S > 0) {
-    MOE_CHECK_PTR(Ws1);
-    MOE_CHECK_PTR(Ws3);
-    MOE_CHECK_PTR(Ws2);
-  }
-  Ws w;
-  if ((rc = check_ws(dims, ws, ws_bytes, &w))) return rc;
-  if ((rc = check_device())) return rc;
-  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int rows = dims->T * dims->k;
-  uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
-  int32_t* counters = w.at<int32_t>(w.L.counters);
-  cudaError_t e = launch_gather_rows(static_cast<const uint16_t*>(h), perm, rows, dims->D,
-                                     dims->T, xperm, counters, dims->E + dims->S, st);
-  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
-  FfnArgs a;
-  a.xperm = xperm;
-  a.h = static_cast<const uint16_t*>(h);
-  a.offsets = offsets;
-  a.W1 = static_cast<const uint16_t*>(W1);
-  a.W3 = static_cast<const uint16_t*>(W3);
-  a.W2 = static_cast<const uint16_t*>(W2);
-  a.Ws1 = static_cast<const uint16_t*>(Ws1);
-  a.Ws3 = static_cast<const uint16_t*>(Ws3);
-  a.Ws2 = static_cast<const uint16_t*>(Ws2);
-  a.act_r = w.at<uint16_t>(w.L.act_r);
-  a.act_s = w.at<uint16_t>(w.L.act_s);
-  a.y = y;
-  a.status = w.status();
-  a.counters = counters;
-  a.T = dims->T; a.D = dims->D; a.E = dims->E; a.F = dims->F; a.k = dims->k;
-  a.S = dims->S; a.Fs = dims->Fs;
-  int n = 1;
-  const char* why = "launch failed";
-  e = launch_expert_ffn(a, st, &n, &why, nullptr);
-  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
-  g_launches = n;
-  return MOE_OK;
+  ExpertWeights wt;
+  if ((rc = check_bf16_weights(W1, W3, W2, Ws1, Ws3, Ws2, dims, &wt))) return rc;
+  return expert_ffn_impl(h, perm, offsets, wt, dims, y, ws, ws_bytes, stream);
+}
+
+int moe_expert_ffn_fp8(const void* h, const int32_t* perm, const int32_t* offsets,
+                       const moe_fp8_weights_t* w8, const moe_dims_t* dims, float* y, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  int rc = begin(dims);
+  if (rc) return rc;
+  if ((rc = check_fp8_dims(dims))) return rc;
+  if (dims->T == 0) return MOE_OK;
+  ExpertWeights wt;
+  if ((rc = check_fp8_weights(w8, dims, &wt))) return rc;
+  return expert_ffn_impl(h, perm, offsets, wt, dims, y, ws, ws_bytes, stream);
 }
 
 int moe_combine(const float* y, const float* w, const int32_t* inv, const moe_dims_t* dims,
@@ -437,77 +592,46 @@ int moe_forward(const void* h, const float* Wr, const float* bias, const void* W
   MOE_CHECK_PTR(h);
   MOE_CHECK_PTR(Wr);
   MOE_CHECK_PTR(bias);
-  MOE_CHECK_PTR(W1);
-  MOE_CHECK_PTR(W3);
-  MOE_CHECK_PTR(W2);
-  MOE_CHECK_PTR(out);
-  if (dims->S > 0) {
-    MOE_CHECK_PTR(Ws1);
-    MOE_CHECK_PTR(Ws3);
-    MOE_CHECK_PTR(Ws2);
-  }
-  if (idx_out && !aligned16(idx_out)) return fail(MOE_ERR_INVALID_ARG, "idx_out is not 16-byte aligned");
-  if (w_out && !aligned16(w_out)) return fail(MOE_ERR_INVALID_ARG, "w_out is not 16-byte aligned");
-  Ws w;
-  if ((rc = check_ws(dims, ws, ws_bytes, &w))) return rc;
-  if ((rc = check_device())) return rc;
-  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int T = dims->T, D = dims->D, E = dims->E, k = dims->k;
-  const auto* hb = static_cast<const uint16_t*>(h);
-  int32_t* idx = idx_out ? idx_out : w.at<int32_t>(w.L.idx);
-  float* rw = w_out ? w_out : w.at<float>(w.L.w);
-  int32_t* counts = w.at<int32_t>(w.L.counts);
-  int32_t* offsets = w.at<int32_t>(w.L.offsets);
-  int32_t* perm = w.at<int32_t>(w.L.perm);
-  int32_t* inv = w.at<int32_t>(w.L.inv);
-  float* y = w.at<float>(w.L.y);
-  int n = 0;
+  ExpertWeights wt;
+  if ((rc = check_bf16_weights(W1, W3, W2, Ws1, Ws3, Ws2, dims, &wt))) return rc;
+  return forward_impl(h, Wr, bias, wt, dims, out, idx_out, w_out, ws, ws_bytes, stream);
+}
 
-  const RouterSplit sp = router_split(T, D, E);
-  float* partials = w.at<float>(w.L.partials);
-  const char* rwhy = "router launch";
-  cudaError_t e = mark(0, st);
-  if (e == cudaSuccess) e = launch_router(hb, Wr, *dims, sp, w, partials, st, &n, &rwhy);
-  if (e == cudaSuccess) e = mark(1, st);
-  if (e != cudaSuccess) return cuda_fail(e, rwhy);
-  e = launch_route(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw, w.status(), st);
-  if (e == cudaSuccess) e = mark(2, st);
-  if (e != cudaSuccess) return cuda_fail(e, "route launch");
-  n += 1;
-  e = launch_permute(idx, T, E, k, counts, offsets, perm, inv, w.at<int32_t>(w.L.blk_base),
-                     w.status(), w.at<int32_t>(w.L.touched), st, &n);
-  if (e == cudaSuccess) e = mark(3, st);
-  if (e != cudaSuccess) return cuda_fail(e, "permute launch");
-  uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
-  int32_t* counters = w.at<int32_t>(w.L.counters);
-  e = launch_gather_rows(hb, perm, T * k, D, T, xperm, counters, E + dims->S, st);
-  if (e == cudaSuccess) e = mark(4, st);
-  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
-  n += 1;
-  FfnArgs a;
-  a.xperm = xperm;
-  a.h = hb;
-  a.offsets = offsets;
-  a.W1 = static_cast<const uint16_t*>(W1);
-  a.W3 = static_cast<const uint16_t*>(W3);
-  a.W2 = static_cast<const uint16_t*>(W2);
-  a.Ws1 = static_cast<const uint16_t*>(Ws1);
-  a.Ws3 = static_cast<const uint16_t*>(Ws3);
-  a.Ws2 = static_cast<const uint16_t*>(Ws2);
-  a.act_r = w.at<uint16_t>(w.L.act_r);
-  a.act_s = w.at<uint16_t>(w.L.act_s);
-  a.y = y;
-  a.status = w.status();
-  a.counters = counters;
-  a.T = T; a.D = D; a.E = E; a.F = dims->F; a.k = k; a.S = dims->S; a.Fs = dims->Fs;
-  const char* why = "launch failed";
-  e = launch_expert_ffn(a, st, &n, &why, g_prof_events ? g_prof_events + 5 : nullptr);
-  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
-  e = launch_combine(y, rw, inv, T, D, k, dims->S, out, w.status(), st);
-  if (e == cudaSuccess) e = mark(6, st);
-  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
-  n += 1;
-  g_launches = n;
+int moe_forward_fp8(const void* h, const float* Wr, const float* bias, const moe_fp8_weights_t* w8,
+                    const moe_dims_t* dims, float* out, int32_t* idx_out, float* w_out, void* ws,
+                    size_t ws_bytes, moe_stream_t stream) {
+  int rc = begin(dims);
+  if (rc) return rc;
+  if ((rc = check_fp8_dims(dims))) return rc;
+  if (dims->T == 0) return MOE_OK;
+  MOE_CHECK_PTR(h);
+  MOE_CHECK_PTR(Wr);
+  MOE_CHECK_PTR(bias);
+  ExpertWeights wt;
+  if ((rc = check_fp8_weights(w8, dims, &wt))) return rc;
+  return forward_impl(h, Wr, bias, wt, dims, out, idx_out, w_out, ws, ws_bytes, stream);
+}
+
+int moe_fp8_dequantize(const void* codes, const int8_t* exps, int G, int R, int K, void* out,
+                       void* ws, moe_stream_t stream) {
+  g_err.clear();
+  g_launches = 0;
+  if (G < 0 || R < 0 || K < 0) return fail(MOE_ERR_INVALID_ARG, "G, R, K must be >= 0");
+  if (K % 16) return fail(MOE_ERR_INVALID_ARG, "K = %d is not a multiple of 16", K);
+  if ((long long)G * R * K >= (1ll << 40)) return fail(MOE_ERR_UNSUPPORTED, "G*R*K >= 2^40");
+  if ((long long)G * R * K == 0) return MOE_OK;
+  MOE_CHECK_PTR(codes);
+  MOE_CHECK_PTR(out);
+  if (!exps) return fail(MOE_ERR_INVALID_ARG, "exps is NULL");
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  int rc = check_device();
+  if (rc) return rc;
+  cudaError_t e = launch_fp8_dequantize(static_cast<const uint8_t*>(codes), exps, G, R, K,
+                                        static_cast<uint16_t*>(out), static_cast<int*>(ws),
+                                        reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  g_launches = 1;
   return MOE_OK;
 }
 

@@ -45,20 +45,16 @@
 //               lanes 32*(w%4) .. +31), fused activation, global stores.
 #include <cuda_bf16.h>
 
-#include "moe_internal.cuh"
-#include "sm100_ptx.cuh"
+#include "ffn_common.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BK = 64;                    // one 128-byte swizzle row of bf16
+using namespace ffn;
+
 constexpr int THREADS = 192;
-constexpr int A_BYTES = BM * BK * 2;      // 16 KiB
-constexpr int MAX_E = 1024;
 constexpr int RING_BYTES = 192 * 1024;    // operand ring budget
 constexpr int MAX_STAGES = 6;
-constexpr int EPI_WARPS = 4;              // each releases its rows of a gate/up tile
 
 template <int MMA_N>
 struct Shape {
@@ -70,39 +66,6 @@ struct Shape {
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, MMA_N);
 };
 
-// One grouped GEMM.  Routed group e has rows [off[e], off[e+1]) of the routed
-// A / output matrices; shared group s has rows s*T .. s*T + T - 1 of the
-// shared output (its A rows start at s * a_s_group_stride).
-struct alignas(64) Problem {
-  CUtensorMap a_r;   // routed A  [rows_r, K_r]
-  CUtensorMap a_s;   // shared A
-  CUtensorMap b0_r;  // W1 [E*F, D] (gate/up) | W2 [E*D, F] (down)
-  CUtensorMap b1_r;  // W3 [E*F, D] (gate/up only)
-  CUtensorMap b0_s;  // Ws1 | Ws2
-  CUtensorMap b1_s;  // Ws3
-  void* out_r;
-  void* out_s;
-  int K_r, K_s;              // reduction lengths
-  int N_r, N_s;              // output columns (= output row strides)
-  int a_s_group_stride;      // rows between shared groups' A blocks (0 or T)
-  int b_r_group_rows;        // B rows per routed expert (F or D)
-  int b_s_group_rows;        // B rows per shared expert (Fs, D or 0)
-  int bn_out;                // output columns per tile (N or N/2)
-  int k_chunk;               // > 0: shared group g covers K range [g*k_chunk, (g+1)*k_chunk)
-  int a_k_mod;               // > 0: the A operand's K coordinate wraps modulo this
-  int gateup;                // epilogue: 1 = SiLU gate -> bf16, 0 = fp32 store
-};
-
-struct GemmParams {
-  Problem pr[2];
-  const int32_t* offsets;    // [E+1] routed group row offsets (E > 0)
-  int* status;
-  int* counters;             // [E+S] gate/up tiles stored per group (two problems)
-  int nprob;                 // 1 or 2
-  int E, S, T;
-  int rows_r;                // T * k
-};
-
 struct SharedState {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
@@ -111,102 +74,8 @@ struct SharedState {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  int mt_total;              // routed row tiles over all experts
-  int off[MAX_E + 1];        // group row offsets
-  int mt_prefix[MAX_E + 1];  // routed row-tile prefix per expert
+  TileMap tm;
 };
-
-struct TileInfo {
-  int prob;
-  bool shared;
-  int grp;      // expert (routed) or shared expert index
-  int m0;       // first row within the group
-  int n0;       // first output column
-  int rows;     // rows in the group
-  int row0;     // group's first row in the output (and routed A) matrix
-  int mt;       // row tiles of the group
-};
-
-__device__ __forceinline__ int col_tiles(int N, int bn) { return (N + bn - 1) / bn; }
-
-__device__ __forceinline__ int problem_tiles(const Problem& P, const SharedState& ss,
-                                             const GemmParams& p) {
-  const int mt_s = (p.T + BM - 1) / BM;
-  return ss.mt_total * col_tiles(P.N_r, P.bn_out) + p.S * mt_s * col_tiles(P.N_s, P.bn_out);
-}
-
-__device__ __forceinline__ TileInfo decode_tile(int tile, const SharedState& ss,
-                                                const GemmParams& p, int tiles0) {
-  TileInfo ti;
-  ti.prob = (tile >= tiles0) ? 1 : 0;
-  const Problem& P = p.pr[ti.prob];
-  const int lt = tile - (ti.prob ? tiles0 : 0);
-  const int nt_r = col_tiles(P.N_r, P.bn_out);
-  const int routed = ss.mt_total * nt_r;
-  if (lt < routed) {
-    // expert e: largest with mt_prefix[e] * nt_r <= lt
-    const int q = lt / nt_r;
-    int lo = 0, hi = p.E - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (ss.mt_prefix[mid] <= q) lo = mid; else hi = mid - 1;
-    }
-    const int e = lo;
-    const int rows = ss.off[e + 1] - ss.off[e];
-    const int mt = (rows + BM - 1) / BM;
-    const int local = lt - ss.mt_prefix[e] * nt_r;
-    ti.shared = false;
-    ti.grp = e;
-    ti.m0 = (local % mt) * BM;
-    ti.n0 = (local / mt) * P.bn_out;
-    ti.rows = rows;
-    ti.row0 = ss.off[e];
-    ti.mt = mt;
-  } else {
-    const int ls = lt - routed;
-    const int mt = (p.T + BM - 1) / BM;
-    const int nt = col_tiles(P.N_s, P.bn_out);
-    const int s = ls / (mt * nt);
-    const int rem = ls - s * mt * nt;
-    ti.shared = true;
-    ti.grp = s;
-    ti.m0 = (rem % mt) * BM;
-    ti.n0 = (rem / mt) * P.bn_out;
-    ti.rows = p.T;
-    ti.row0 = s * p.T;
-    ti.mt = mt;
-  }
-  return ti;
-}
-
-// K range of a tile: the whole reduction, or one chunk of it when the shared
-// groups split K (the router's split-K partial sums).
-__device__ __forceinline__ void tile_k_range(const TileInfo& ti, const Problem& P, int* kbeg,
-                                             int* K) {
-  if (ti.shared && P.k_chunk > 0) {
-    *kbeg = ti.grp * P.k_chunk;
-    *K = min(P.k_chunk, P.K_s - *kbeg);
-  } else {
-    *kbeg = 0;
-    *K = ti.shared ? P.K_s : P.K_r;
-  }
-}
-
-__device__ __forceinline__ float silu_times(float g, float u) {
-  return g / (1.0f + __expf(-g)) * u;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Waits for in-flight async work even after an abort (bounded by the same
-// clock budget); a timeout here raises the CTA's abort flag too.
-__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  int ignore_abort = 0;
-  if (!ptx::mbar_wait(bar, parity, &ignore_abort)) *abort = 1;
-}
 
 template <int MMA_N>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
@@ -252,43 +121,15 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   // everything below reads what earlier kernels in the stream wrote
   ptx::pdl_wait();
 
-  // Routed row-tile prefix from the group offsets (warp 2 scans 32 experts at a time).
-  if (warp == 2) {
-    int carry = 0;
-    bool bad = false;
-    for (int base = 0; base < p.E; base += 32) {
-      const int e = base + lane;
-      int cnt = 0;
-      if (e < p.E) {
-        const int a = p.offsets[e], b = p.offsets[e + 1];
-        ss.off[e] = a;
-        if (e == p.E - 1) ss.off[p.E] = b;
-        if (a < 0 || b < a || b > p.rows_r || (e == 0 && a != 0)) bad = true;
-        cnt = b >= a ? (b - a + BM - 1) / BM : 0;
-      }
-      int incl = cnt;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      if (e < p.E) ss.mt_prefix[e] = carry + incl - cnt;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    bad = __any_sync(0xffffffffu, bad);
-    if (lane == 0) {
-      ss.mt_prefix[p.E] = carry;
-      ss.mt_total = bad ? 0 : carry;
-      if (bad && p.status) atomicOr(p.status, kStBounds);
-    }
-  }
+  // Routed row-tile map from the group offsets.
+  if (warp == 2) build_tile_map(ss.tm, p, lane);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
 
   const uint32_t tmem_base = ss.tmem_base;
-  const int tiles0 = problem_tiles(p.pr[0], ss, p);
-  const int total = tiles0 + (p.nprob > 1 ? problem_tiles(p.pr[1], ss, p) : 0);
+  const int tiles0 = problem_tiles(p.pr[0], ss.tm, p);
+  const int total = tiles0 + (p.nprob > 1 ? problem_tiles(p.pr[1], ss.tm, p) : 0);
   volatile int* abort = &ss.abort;
 
   if (warp == 0) {
@@ -298,14 +139,12 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       uint32_t phase = 0;
       uint32_t issued_mask = 0, last_parity = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(tile, ss, p, tiles0);
+        const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
         const Problem& P = p.pr[ti.prob];
         if (ti.prob == 1) {
           // the activations of this group come from problem 0's epilogues
           const int g = ti.shared ? p.E + ti.grp : ti.grp;
-          const int nt0 = ti.shared ? col_tiles(p.pr[0].N_s, p.pr[0].bn_out)
-                                    : col_tiles(p.pr[0].N_r, p.pr[0].bn_out);
-          if (!ptx::counter_wait(p.counters + g, EPI_WARPS * ti.mt * nt0, abort)) break;
+          if (!ptx::counter_wait(p.counters + g, rows_ready_target(p, ti), abort)) break;
           ptx::fence_proxy_async_global();
         }
         const CUtensorMap* amap = ti.shared ? &P.a_s : &P.a_r;
@@ -349,7 +188,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(tile, ss, p, tiles0);
+        const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
         int kbeg, K;
         tile_k_range(ti, p.pr[ti.prob], &kbeg, &K);
         const int nk = (K + BK - 1) / BK;
@@ -384,68 +223,17 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const TileInfo ti = decode_tile(tile, ss, p, tiles0);
+      const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
       const Problem& P = p.pr[ti.prob];
       if (!ptx::mbar_wait(&ss.tmem_full[acc], acc_phase, abort)) break;
       ptx::tc_fence_after();
-      const int r = ti.m0 + q * 32 + lane;       // row within the group
-      const bool row_ok = r < ti.rows;
-      const int N = ti.shared ? P.N_s : P.N_r;
-      const size_t out_row = (size_t)ti.row0 + r;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * ACC_COLS;
-      if (P.gateup) {
-        uint16_t* out = static_cast<uint16_t*>(ti.shared ? P.out_s : P.out_r);
-#pragma unroll 1
-        for (int c = 0; c < HALF; c += 16) {
-          uint32_t g[16], u[16];
-          ptx::tmem_ld_x16(taddr + c, g);
-          ptx::tmem_ld_x16(taddr + HALF + c, u);
-          ptx::tmem_wait_ld();
-          const int col = ti.n0 + c;
-          if (row_ok && col < N) {
-            uint32_t pk[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              pk[i] = pack_bf16(silu_times(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
-                                silu_times(__uint_as_float(g[2 * i + 1]),
-                                           __uint_as_float(u[2 * i + 1])));
-            uint4* dst = reinterpret_cast<uint4*>(out + out_row * N + col);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            if (col + 8 < N) dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          }
-        }
-      } else {
-        float* out = static_cast<float*>(ti.shared ? P.out_s : P.out_r);
-#pragma unroll 1
-        for (int c = 0; c < MMA_N; c += 16) {
-          uint32_t v[16];
-          ptx::tmem_ld_x16(taddr + c, v);
-          ptx::tmem_wait_ld();
-          const int col = ti.n0 + c;
-          if (row_ok && col < N) {
-            uint4* dst = reinterpret_cast<uint4*>(out + out_row * N + col);
-            dst[0] = make_uint4(v[0], v[1], v[2], v[3]);
-            dst[1] = make_uint4(v[4], v[5], v[6], v[7]);
-            if (col + 8 < N) {
-              dst[2] = make_uint4(v[8], v[9], v[10], v[11]);
-              dst[3] = make_uint4(v[12], v[13], v[14], v[15]);
-            }
-          }
-        }
-      }
+      store_tile<MMA_N>(ti, P, taddr, q, lane);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ss.tmem_empty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-      if (p.nprob > 1 && ti.prob == 0) {
-        // release this warp's rows of the tile to the down tiles of its
-        // group: make the stores visible to the async proxy and to the whole
-        // GPU, then count them (four counts per tile, one per epilogue warp)
-        ptx::fence_proxy_async_global();
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) atomicAdd(p.counters + (ti.shared ? p.E + ti.grp : ti.grp), 1);
-      }
+      if (p.nprob > 1 && ti.prob == 0) release_rows(p, ti, lane);
     }
   }
 
@@ -461,36 +249,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// bf16 row-major [rows, cols] matrix, box = box_rows x 64 columns, 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {BK, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_tensor_map(m, base, rows, cols, box_rows, BK, 2, 128);
 }
 
 template <int MMA_N>
@@ -520,6 +280,42 @@ cudaError_t launch_one(const GemmParams& p, int tiles_upper, cudaStream_t st) {
 }
 
 }  // namespace
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+bool make_tensor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                     uint32_t box_rows, uint32_t box_cols, int elem_bytes, int swizzle_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * (cuuint64_t)elem_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+            : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                  : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 // Router logits on the tensor cores.  The fp32 router weight is split exactly
 // into three bf16 pieces (hi + mid + lo, each the bf16 rounding of what the

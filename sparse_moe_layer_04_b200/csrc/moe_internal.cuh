@@ -112,6 +112,20 @@ struct FfnArgs {
 cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch,
                               const char** why, void* const* marks);
 
+// FP8 expert weights: E4M3 codes and int8 block exponents (one per 128 x 128
+// block of each expert's [rows, K] matrix).
+struct Fp8Weights {
+  const uint8_t *W1, *W3, *W2, *Ws1, *Ws3, *Ws2;
+  const int8_t *W1e, *W3e, *W2e, *Ws1e, *Ws3e, *Ws2e;
+};
+// The expert MLPs of FfnArgs (whose bf16 weight pointers are unused) with FP8
+// weights.
+cudaError_t launch_expert_ffn_fp8(const FfnArgs& a, const Fp8Weights& w, cudaStream_t st,
+                                  int* nlaunch, const char** why, void* const* marks);
+// codes [G, R, K] + exps [G, ceil(R/128), ceil(K/128)] -> bf16 [G, R, K]; K % 16 == 0.
+cudaError_t launch_fp8_dequantize(const uint8_t* codes, const int8_t* exps, int G, int R, int K,
+                                  uint16_t* out, int* status, cudaStream_t st);
+
 int num_sms();
 
 cudaError_t launch_bounded_wait_selftest(int* status, cudaStream_t st);

@@ -116,3 +116,62 @@ def test_grouped_route_argument_checks(mod):
 def test_binding_names_match_the_abi(mod):
     for n in _declared_functions():
         assert hasattr(mod, n), n
+
+
+def _w8(mod, **over):
+    w = mod.moe_fp8_weights_t()
+    for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2", "W1e", "W3e", "W2e", "Ws1e", "Ws3e", "Ws2e"):
+        setattr(w, n, over.get(n, FAKE))
+    return w
+
+
+def test_fp8_argument_checks(mod):
+    lib = mod._lib
+    d = mod.dims(T=8, D=128, E=8, F=64, k=2)
+    ws_n = mod.moe_workspace_size(d)
+    ok = _w8(mod)
+    # D, F, Fs must be multiples of 16 for FP8 rows (TMA strides)
+    for bad in (dict(D=136), dict(F=72), dict(Fs=40)):
+        db = mod.dims(**{**dict(T=8, D=128, E=8, F=64, k=2), **bad})
+        rc = lib.moe_expert_ffn_fp8(FAKE, FAKE, FAKE, ctypes.byref(ok), ctypes.byref(db), FAKE,
+                                    FAKE, 1 << 40, None)
+        assert rc == mod.MOE_ERR_INVALID_ARG and "multiple of 16" in mod.moe_last_error(), bad
+    rc = lib.moe_expert_ffn_fp8(FAKE, FAKE, FAKE, None, ctypes.byref(d), FAKE, FAKE, ws_n, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "w8" in mod.moe_last_error()
+    rc = lib.moe_expert_ffn_fp8(FAKE, FAKE, FAKE, ctypes.byref(_w8(mod, W2e=None)), ctypes.byref(d),
+                                FAKE, FAKE, ws_n, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "W2e" in mod.moe_last_error()
+    rc = lib.moe_expert_ffn_fp8(FAKE, FAKE, FAKE, ctypes.byref(_w8(mod, W3=FAKE + 8)),
+                                ctypes.byref(d), FAKE, FAKE, ws_n, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "aligned" in mod.moe_last_error()
+    rc = lib.moe_expert_ffn_fp8(FAKE, FAKE, FAKE, ctypes.byref(_w8(mod, Ws2e=None)),
+                                ctypes.byref(d), FAKE, FAKE, ws_n, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "Ws" in mod.moe_last_error()
+    # S = 0: shared members may be NULL (then the workspace check is reached)
+    d0 = mod.dims(T=8, D=128, E=8, F=64, k=2, S=0, Fs=8)
+    rc = lib.moe_expert_ffn_fp8(FAKE, FAKE, FAKE,
+                                ctypes.byref(_w8(mod, Ws1=None, Ws3=None, Ws2=None, Ws1e=None,
+                                                 Ws3e=None, Ws2e=None)),
+                                ctypes.byref(d0), FAKE, FAKE, 0, None)
+    assert rc == mod.MOE_ERR_WORKSPACE
+    rc = lib.moe_forward_fp8(FAKE, FAKE, None, ctypes.byref(ok), ctypes.byref(d), FAKE, None, None,
+                             FAKE, ws_n, None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "bias" in mod.moe_last_error()
+    rc = lib.moe_forward_fp8(FAKE, FAKE, FAKE, ctypes.byref(ok), ctypes.byref(d), FAKE, None, None,
+                             FAKE, ws_n - 256, None)
+    assert rc == mod.MOE_ERR_WORKSPACE
+    # T = 0 is a no-op that launches nothing
+    dz = mod.dims(T=0, D=128, E=8, F=64, k=2)
+    assert lib.moe_forward_fp8(None, None, None, None, ctypes.byref(dz), None, None, None, None, 0,
+                               None) == mod.MOE_OK
+
+
+def test_fp8_dequantize_argument_checks(mod):
+    lib = mod._lib
+    assert lib.moe_fp8_dequantize(FAKE, FAKE, 1, 4, 24, FAKE, None, None) == mod.MOE_ERR_INVALID_ARG
+    assert "multiple of 16" in mod.moe_last_error()
+    assert lib.moe_fp8_dequantize(FAKE, FAKE, -1, 4, 16, FAKE, None, None) == mod.MOE_ERR_INVALID_ARG
+    assert lib.moe_fp8_dequantize(FAKE, None, 1, 4, 16, FAKE, None, None) == mod.MOE_ERR_INVALID_ARG
+    assert lib.moe_fp8_dequantize(FAKE + 1, FAKE, 1, 4, 16, FAKE, None, None) == mod.MOE_ERR_INVALID_ARG
+    assert lib.moe_fp8_dequantize(FAKE, FAKE, 1, 4, 16, FAKE, FAKE + 16, None) == mod.MOE_ERR_WORKSPACE
+    assert lib.moe_fp8_dequantize(None, None, 0, 4, 16, None, None, None) == mod.MOE_OK
