@@ -64,7 +64,8 @@ class moe_fp8_weights_t(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m sparse_moe_layer_04_b200.build`")
+                          "`python sparse_moe_layer_04_b200/build.py` (or "
+                          "`python __graft_entry__.py`)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     D = ctypes.POINTER(moe_dims_t)
