@@ -71,26 +71,34 @@ def aggregate_tokens_per_s(tokens_per_rank: int, world: int, max_ms: float) -> f
 # ---------------------------------------------------------------------------
 # accounting
 # ---------------------------------------------------------------------------
-def layer_bytes_flops(cfg, U: int):
+def expert_weight_bytes(rows: int, K: int, weights: str) -> int:
+    """Bytes of one expert matrix [rows, K]: bf16, or FP8 codes plus one int8
+    exponent per 128 x 128 block."""
+    if weights == "fp8":
+        return rows * K + -(-rows // 128) * -(-K // 128)
+    return rows * K * 2
+
+
+def layer_bytes_flops(cfg, U: int, weights: str = "bf16"):
     """Algorithmic bytes and flops of one layer pass (touched experts only):
     expert weights of the touched routed experts and of the shared experts, the
     router weight and bias, the bf16 input, the fp32 output, the routing."""
     T, D, E, F, k, S, Fs = cfg.T, cfg.D, cfg.E, cfg.F, cfg.k, cfg.S, cfg.Fs
-    B = (U * 3 * D * F * 2 + S * 3 * D * Fs * 2 + E * D * 4 + E * 4 + T * D * 2 + T * D * 4
-         + T * k * 8)
+    wb = 3 * (U * expert_weight_bytes(F, D, weights) + S * expert_weight_bytes(Fs, D, weights))
+    B = wb + E * D * 4 + E * 4 + T * D * 2 + T * D * 4 + T * k * 8
     FL = 2 * T * D * E + 6 * D * F * T * k + 6 * D * Fs * T * S
     return B, FL
 
 
-def ffn_bytes(cfg, U: int):
+def ffn_bytes(cfg, U: int, weights: str = "bf16"):
     """Algorithmic bytes of one expert-FFN launch (gate/up and down GEMMs in one
     kernel): W1, W3 and W2 of the touched routed experts and of the shared
     experts, the gathered bf16 input rows, and the fp32 expert outputs written.
     The gated activations stay inside the kernel's working set and are not
     counted."""
     T, D, F, k, S, Fs = cfg.T, cfg.D, cfg.F, cfg.k, cfg.S, cfg.Fs
-    return (U * 3 * F * D * 2 + S * 3 * Fs * D * 2 + (T * k + S * T) * D * 2
-            + (T * k + S * T) * D * 4)
+    wb = 3 * (U * expert_weight_bytes(F, D, weights) + S * expert_weight_bytes(Fs, D, weights))
+    return wb + (T * k + S * T) * D * 2 + (T * k + S * T) * D * 4
 
 
 def ffn_flops(cfg):
@@ -211,18 +219,27 @@ def time_oracle(run, n_tokens: int, min_s: float, max_s: float):
     return n_tokens * reps / el, reps, el
 
 
-def cpu_baseline_from_device(cfg, inp, n_tokens: int):
+def cpu_baseline_from_device(cfg, inp, n_tokens: int, fp8=None):
+    """The oracle on the first tokens of the batch; with `fp8` (codes and
+    exponents) the experts are the oracle's decoding of the FP8 weights."""
+    from oracle import moe_oracle as orc
+
     h = inp["h"][:n_tokens].float().cpu().numpy()
     Wr = inp["Wr"].cpu().numpy()
     bias = inp["bias"].cpu().numpy()
     cache = {}
 
+    def matrices(names, g):
+        if fp8 is None:
+            return tuple(inp[n][g].cpu().double().numpy() for n in names)
+        return tuple(orc.dequantize_fp8_blocks(fp8[n + "q"][g].cpu().numpy(),
+                                               fp8[n + "e"][g].cpu().numpy()) for n in names)
+
     def expert(e):
         if e not in cache:
-            cache[e] = tuple(x[e].cpu().double().numpy() for x in (inp["W1"], inp["W3"], inp["W2"]))
+            cache[e] = matrices(("W1", "W3", "W2"), e)
         return cache[e]
-    shared = [tuple(x[s].cpu().double().numpy() for x in (inp["Ws1"], inp["Ws3"], inp["Ws2"]))
-              for s in range(cfg.S)]
+    shared = [matrices(("Ws1", "Ws3", "Ws2"), s) for s in range(cfg.S)]
     run = oracle_sample_runner(cfg, h, Wr, bias, expert, shared)
     tps, reps, el = time_oracle(run, n_tokens, 10.0, 30.0)
     return {"value": tps, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
@@ -244,6 +261,15 @@ def run_ours(args, rank, world, local_rank):
         cfg = mi.custom_config(args.config, E=args.experts or cfg.E, T=args.tokens or cfg.T)
     inp = mi.layer_weights(cfg, 0, device=dev)
     inp["h"] = mi.hidden(cfg, seed=replica_seed(rank), device=dev)
+    fp8 = None
+    if args.weights == "fp8":
+        # the FP8 layer stores only codes and block exponents
+        fp8 = mi.fp8_layer_weights(inp)
+        for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2"):
+            del inp[n]
+        torch.cuda.empty_cache()
+        w8 = moe.fp8_weights(*(fp8[n + "q"] for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2")),
+                             *(fp8[n + "e"] for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2")))
     d = moe.dims_of(cfg)
     ws = moe.alloc_workspace(d, dev)
     out = torch.empty((cfg.T, cfg.D), dtype=torch.float32, device=dev)
@@ -251,9 +277,15 @@ def run_ours(args, rank, world, local_rank):
     wgt = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
+    def forward(h, o, i=None, w=None):
+        if fp8 is not None:
+            moe.moe_forward_fp8(h, inp["Wr"], inp["bias"], w8, d, o, ws, i, w)
+        else:
+            moe.moe_forward(h, inp["Wr"], inp["bias"], inp["W1"], inp["W3"], inp["W2"],
+                            inp["Ws1"], inp["Ws3"], inp["Ws2"], d, o, ws, i, w)
+
     def step():
-        moe.moe_forward(inp["h"], inp["Wr"], inp["bias"], inp["W1"], inp["W3"], inp["W2"],
-                        inp["Ws1"], inp["Ws3"], inp["Ws2"], d, out, ws, idx, wgt)
+        forward(inp["h"], out, idx, wgt)
 
     sampler = ClockSampler(local_rank)
     for _ in range(args.warmup):
@@ -322,8 +354,7 @@ def run_ours(args, rank, world, local_rank):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         h_dev.copy_(h_pin, non_blocking=True)
-        moe.moe_forward(h_dev, inp["Wr"], inp["bias"], inp["W1"], inp["W3"], inp["W2"],
-                        inp["Ws1"], inp["Ws3"], inp["Ws2"], d, out, ws)
+        forward(h_dev, out)
         out_pin.copy_(out, non_blocking=True)
         b.record()
         b.synchronize()
@@ -337,11 +368,11 @@ def run_ours(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     hbm = float(peaks["hbm_gbs"])
     bf16 = float(peaks["bf16_tflops"])
-    B, FL = layer_bytes_flops(cfg, U)
+    B, FL = layer_bytes_flops(cfg, U, args.weights)
     t_s = ms / 1e3
     t_roof_hbm = B / (hbm * 1e9)
     t_roof_tc = FL / (bf16 * 1e12)
-    f_bytes = ffn_bytes(cfg, U)
+    f_bytes = ffn_bytes(cfg, U, args.weights)
     f_flops = ffn_flops(cfg)
     f_gbs = f_bytes / (ffn_ms / 1e3) / 1e9
     f_tfs = f_flops / (ffn_ms / 1e3) / 1e12
@@ -352,8 +383,10 @@ def run_ours(args, rank, world, local_rank):
     else:
         roof = {"bound": "tensor", "achieved": f_tfs, "peak": bf16, "unit": "TFLOP/s",
                 "frac": f_tfs / bf16}
-    roof.update({"traffic": stored_traffic(f"expert_ffn/{cfg.name}"),
-                 "kernel": "grouped_gemm_kernel (fused gate/up + down expert FFN)", "ms": ffn_ms,
+    traffic_key = ("expert_ffn_fp8/" if fp8 is not None else "expert_ffn/") + cfg.name
+    kernel = ("ffn_fp8_kernel (fused gate/up + down expert FFN, FP8 weights decoded into TMEM)"
+              if fp8 is not None else "grouped_gemm_kernel (fused gate/up + down expert FFN)")
+    roof.update({"traffic": stored_traffic(traffic_key), "kernel": kernel, "ms": ffn_ms,
                  "algorithmic_bytes": f_bytes, "algorithmic_flops": f_flops,
                  "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured"
                  else "fallback (profiling recipe)"})
@@ -378,6 +411,8 @@ def run_ours(args, rank, world, local_rank):
                                f"E={cfg.E} k={cfg.k} F={cfg.F} S={cfg.S} Fs={cfg.Fs} "
                                f"scale={cfg.scale}",
                    "T": cfg.T, "touched_experts": U, "global_batch": world * cfg.T,
+                   "weights": ("fp8 e4m3 codes + power-of-two 128x128 block exponents, decoded "
+                               "exactly to bf16 in the kernel" if fp8 is not None else "bf16"),
                    "parallelism": f"replicas x{world} (token-parallel, no exchange)",
                    "l2": "flushed: 256 MiB memset before every timed step, outside its events",
                    "ms_p10_p90": [float(np.percentile(step_ms, 10)), float(np.percentile(step_ms, 90))],
@@ -397,7 +432,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline_from_device(cfg, inp, min(cfg.T, args.cpu_tokens))
+        res["cpu_baseline"] = cpu_baseline_from_device(cfg, inp, min(cfg.T, args.cpu_tokens), fp8)
     return res
 
 
@@ -414,12 +449,17 @@ def run_reference(args):
     bias = mi.correction_bias(cfg, 0).numpy()
     cache = {}
 
+    def matrices(ws):
+        if args.weights == "fp8":   # the weights the FP8 codes stand for
+            return tuple(orc.dequantize_fp8_blocks(*(t.numpy() for t in mi.quantize_fp8_blocks(x)))
+                         for x in ws)
+        return tuple(x.double().numpy() for x in ws)
+
     def expert(e):
         if e not in cache:
-            cache[e] = tuple(x.double().numpy() for x in mi.expert_weights(cfg, e, 0))
+            cache[e] = matrices(mi.expert_weights(cfg, e, 0))
         return cache[e]
-    shared = [tuple(x.double().numpy() for x in mi.expert_weights(cfg, s, 0, shared=True))
-              for s in range(cfg.S)]
+    shared = [matrices(mi.expert_weights(cfg, s, 0, shared=True)) for s in range(cfg.S)]
 
     def step():
         return orc.moe_layer_tokens(h, Wr, bias, cfg.k, cfg.scale, expert, shared)
@@ -444,7 +484,7 @@ def run_reference(args):
         "data": "synthetic (seeded counter-based generator)",
         "config": {"workload": f"{cfg.name}: T={cfg.T} D={cfg.D} E={cfg.E} k={cfg.k} F={cfg.F} "
                                f"S={cfg.S} Fs={cfg.Fs} scale={cfg.scale}", "T": cfg.T,
-                   "sample_tokens": n},
+                   "sample_tokens": n, "weights": args.weights},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -462,6 +502,9 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=128,
                     help="tokens of the batch the CPU oracle processes per pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
+                    help="expert weight storage: bf16 (the headline layer) or FP8 E4M3 with "
+                         "128x128 block scales")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (small cases for profiler captures; not a bench line)")
     ap.add_argument("--tokens", type=int, default=None,

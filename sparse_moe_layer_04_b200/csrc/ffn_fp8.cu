@@ -27,17 +27,26 @@
 // Ordering and the gate/up -> down hand-off (per-group counters, bounded
 // acquire waits) are those of the bf16 kernel.
 //
-// CTA (320 threads, one per SM):
-//   warp 0      TMA producer: token tiles (bf16, 128-byte swizzle, boxes of 64
-//               rows) and FP8 weight tiles (64-byte swizzle) on two rings.
-//   warp 1      TMEM allocator (512 columns) and single-thread MMA issuer,
+// CTA (512 threads, one per SM):
+//   warp 0      token producer: TMA of token tiles (bf16, 128-byte swizzle,
+//               boxes of 64 rows); waits for the gate/up -> down hand-off.
+//   warp 10     weight producer: TMA of FP8 weight tiles (64-byte swizzle) on
+//               a 12-stage ring of its own, running ahead of the tokens.
+//   warps 1,11  MMA issuers (warp 1 also allocates the 512 TMEM columns):
 //               tcgen05.mma.cta_group::1.kind::f16, M = 128, N <= NT, K = 16.
-//   warps 2-5   epilogue (tcgen05.ld, SiLU gate or fp32 store).
-//   warps 6-9   decoders: each reads its 32 weight rows of a stage (one row
-//               per thread, 64 codes), decodes, and stores them to its TMEM
-//               lane quarter; four weight stages live in TMEM.
+//               One issuing thread manages one tcgen05.mma per ~100 cycles,
+//               more than an M = 128, N = 128 MMA takes to execute, so for
+//               NT = 128 two warps take alternate K-blocks into two
+//               accumulators; one commit per K-block frees both the token
+//               stage and the decoded-weight stage.
+//   warps 2-5   epilogue (tcgen05.ld of both accumulators, SiLU gate or fp32
+//               store).
+//   warps 6-9,  decoders, two sets of four taking alternate stages: each warp
+//   12-15       reads its 32 weight rows of a stage (one row per thread, 64
+//               codes), decodes, and stores them to its TMEM lane quarter.
+//               One set alone needs about as long per stage as the MMAs.
 // TMEM columns: accumulators [0, 256) (two of 128 for NT = 128, one of 256
-// for NT = 256), weight stages [256, 384).
+// for NT = 256), decoded-weight stages from column 256 (32 columns each).
 #include <cuda_bf16.h>
 
 #include "ffn_common.cuh"
@@ -53,29 +62,49 @@ constexpr int GU_FEATS = 64;                     // gate/up tile: 64 W1 + 64 W3 
 constexpr int TOK_BOX = 64;                      // token rows per TMA box
 constexpr int TOK_BOX_BYTES = TOK_BOX * BK * 2;  // 8 KiB
 constexpr int W8_BYTES = W_ROWS * BK;            // 8 KiB of codes per stage
-constexpr int W8_STAGES = 8;
-constexpr int A_STAGES = 4;                      // weight stages in TMEM
 constexpr uint32_t A_STAGE_COLS = BK / 2;        // 128 lanes x 64 bf16
-constexpr uint32_t A_COL0 = 256;
+constexpr uint32_t A_COL0 = 256;                 // weight stages follow the accumulators
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int THREADS = 320;
-constexpr int DEC_WARP0 = 6;
+constexpr int TPROD_WARP = 0;                    // token producer
+constexpr int MMA_WARP0 = 1;                     // MMA issuer (and TMEM allocator)
+constexpr int DEC_WARP0 = 6;                     // decoder set 0: warps 6..9
+constexpr int WPROD_WARP = 10;                   // weight producer
+constexpr int MMA_WARP1 = 11;                    // second MMA issuer (NT = 128)
+constexpr int DEC_WARP1 = 12;                    // decoder set 1: warps 12..15
+constexpr int THREADS = 512;
 constexpr int DEC_THREADS = 128;
-constexpr int MAX_TOK_STAGES = 6;
+constexpr int MAX_STAGES = 6;
+constexpr int MAX_W8_STAGES = 12;
 
+// Per-NT configuration.
+//   STAGES     depth of the token ring and of the decoded-weight ring in TMEM;
+//              the two advance together (one stage per K-block) and share
+//              their "empty" barrier, so one tcgen05.commit per K-block
+//              releases both.
+//   W8_STAGES  depth of the FP8 code ring (HBM latency is the longest).
+//   MMA_WARPS  a single thread issues a tcgen05.mma every ~100 cycles at best,
+//              far slower than an M = 128, N <= 128 MMA executes, so NT = 128
+//              blocks split each tile's K-blocks between two issuing warps with
+//              an accumulator each (even K-blocks -> D0, odd -> D1); the
+//              epilogue adds the two.  NT = 256 MMAs are long enough for one.
 template <int NT>
 struct Cfg {
   static constexpr int TOK_STAGE_BYTES = NT * BK * 2;
-  static constexpr int TOK_STAGES = NT == 128 ? 6 : 4;
-  static constexpr int ACC_BUFS = NT == 128 ? 2 : 1;
+  static constexpr int STAGES = NT == 128 ? 6 : 3;
+  static constexpr int W8_STAGES = 12;
+  static constexpr int MMA_WARPS = NT == 128 ? 2 : 1;
+  static_assert(STAGES <= MAX_STAGES && W8_STAGES <= MAX_W8_STAGES, "ring sizes");
+  static_assert(MMA_WARPS * NT <= (int)A_COL0, "accumulators fit below the weight stages");
+  static_assert(A_COL0 + STAGES * A_STAGE_COLS <= TMEM_COLS, "weight stages fit in TMEM");
 };
 
 struct SharedState8 {
-  uint64_t tok_full[MAX_TOK_STAGES], tok_empty[MAX_TOK_STAGES];
-  uint64_t w8_full[W8_STAGES], w8_empty[W8_STAGES];
-  uint64_t a_full[A_STAGES], a_empty[A_STAGES];
-  uint64_t tmem_full[2], tmem_empty[2];
-  uint64_t drain;
+  uint64_t tok_full[MAX_STAGES];      // token tile landed (TMA transaction bytes)
+  uint64_t a_full[MAX_STAGES];        // decoded weights stored in TMEM (decoder threads)
+  uint64_t stage_empty[MAX_STAGES];   // the K-block's MMAs completed (tcgen05.commit)
+  uint64_t w8_full[MAX_W8_STAGES], w8_empty[MAX_W8_STAGES];
+  uint64_t tmem_full, tmem_empty;
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
   TileMap tm;
@@ -92,12 +121,28 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
+// 16 accumulator columns of this warp's lane quarter: D0, plus D1 when the
+// tile's K-blocks were split between two accumulators.
+__device__ __forceinline__ void load_acc(uint32_t taddr, uint32_t d1_off, bool two,
+                                         uint32_t (&v)[16]) {
+  ptx::tmem_ld_x16(taddr, v);
+  if (two) {
+    uint32_t u[16];
+    ptx::tmem_ld_x16(taddr + d1_off, u);
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(u[j]));
+  } else {
+    ptx::tmem_wait_ld();
+  }
+}
+
 // Gate/up epilogue of one warp: lane i < 16 holds the gate row of feature
 // n0 + 16q + i, lane i + 16 the up row of the same feature; columns are the
 // block's tokens.  Per 16 tokens the low lanes finish tokens 0-7 and the high
 // lanes tokens 8-15, each taking the missing half from its partner lane.
 __device__ __forceinline__ void store_gateup(const TileInfo& ti, const Problem& P, uint32_t taddr,
-                                             int n, int q, int lane) {
+                                             uint32_t d1_off, bool two, int n, int q, int lane) {
   const int Nout = ti.shared ? P.N_s : P.N_r;
   const int f = ti.n0 + q * 16 + (lane & 15);
   const bool hi = lane >= 16;
@@ -106,8 +151,7 @@ __device__ __forceinline__ void store_gateup(const TileInfo& ti, const Problem& 
 #pragma unroll 1
   for (int c = 0; c < n; c += 16) {
     uint32_t v[16];
-    ptx::tmem_ld_x16(taddr + c, v);
-    ptx::tmem_wait_ld();
+    load_acc(taddr + c, d1_off, two, v);
     const int t0 = ti.m0 + c + (hi ? 8 : 0);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -123,7 +167,7 @@ __device__ __forceinline__ void store_gateup(const TileInfo& ti, const Problem& 
 
 // Down epilogue of one warp: lane i holds output column n0 + 32q + i.
 __device__ __forceinline__ void store_down(const TileInfo& ti, const Problem& P, uint32_t taddr,
-                                           int n, int q, int lane) {
+                                           uint32_t d1_off, bool two, int n, int q, int lane) {
   const int Nout = ti.shared ? P.N_s : P.N_r;
   const int d = ti.n0 + q * 32 + lane;
   const bool d_ok = d < Nout;
@@ -131,8 +175,7 @@ __device__ __forceinline__ void store_down(const TileInfo& ti, const Problem& P,
 #pragma unroll 1
   for (int c = 0; c < n; c += 16) {
     uint32_t v[16];
-    ptx::tmem_ld_x16(taddr + c, v);
-    ptx::tmem_wait_ld();
+    load_acc(taddr + c, d1_off, two, v);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int t = ti.m0 + c + j;
@@ -141,46 +184,49 @@ __device__ __forceinline__ void store_down(const TileInfo& ti, const Problem& P,
   }
 }
 
+__device__ __forceinline__ int tile_k_blocks(const TileInfo& ti, const Problem& P) {
+  const int K = ti.shared ? P.K_s : P.K_r;
+  return (K + BK - 1) / BK;
+}
+
 template <int NT>
 __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<NT>;
-  constexpr int TS = C::TOK_STAGES;
+  constexpr int S = C::STAGES;
+  constexpr int W8S = C::W8_STAGES;
+  constexpr int MW = C::MMA_WARPS;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_addr(smem_raw);
   uint8_t* tok_ring = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint8_t* w8_ring = tok_ring + TS * C::TOK_STAGE_BYTES;
-  SharedState8& ss = *reinterpret_cast<SharedState8*>(w8_ring + W8_STAGES * W8_BYTES);
+  uint8_t* w8_ring = tok_ring + S * C::TOK_STAGE_BYTES;
+  SharedState8& ss = *reinterpret_cast<SharedState8*>(w8_ring + W8S * W8_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   ptx::pdl_launch_dependents();
-  if (warp == 1) {
+  if (warp == MMA_WARP0) {
     ptx::tmem_alloc(&ss.tmem_base, TMEM_COLS);
     ptx::tmem_relinquish();
   }
   if (threadIdx.x == 0) {
-    for (int i = 0; i < TS; ++i) {
+    for (int i = 0; i < S; ++i) {
       ptx::mbar_init(&ss.tok_full[i], 1);
-      ptx::mbar_init(&ss.tok_empty[i], 1);
+      ptx::mbar_init(&ss.a_full[i], DEC_THREADS);
+      ptx::mbar_init(&ss.stage_empty[i], 1);
     }
-    for (int i = 0; i < W8_STAGES; ++i) {
+    for (int i = 0; i < W8S; ++i) {
       ptx::mbar_init(&ss.w8_full[i], 1);
       ptx::mbar_init(&ss.w8_empty[i], DEC_THREADS);
     }
-    for (int i = 0; i < A_STAGES; ++i) {
-      ptx::mbar_init(&ss.a_full[i], DEC_THREADS);
-      ptx::mbar_init(&ss.a_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(&ss.tmem_full[i], 1);
-      ptx::mbar_init(&ss.tmem_empty[i], EPI_WARPS);
-    }
-    ptx::mbar_init(&ss.drain, 1);
+    ptx::mbar_init(&ss.tmem_full, MW);
+    ptx::mbar_init(&ss.tmem_empty, EPI_WARPS);
+    ptx::mbar_init(&ss.drain[0], 1);
+    ptx::mbar_init(&ss.drain[1], 1);
     ss.abort = 0;
     ptx::fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == TPROD_WARP && lane == 0) {
     ptx::tma_prefetch_desc(&p.pr[0].a_r);
     ptx::tma_prefetch_desc(&p.pr[0].b0_r);
     ptx::tma_prefetch_desc(&p.pr[0].b1_r);
@@ -199,12 +245,12 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
   volatile int* abort = &ss.abort;
   bool bad_exp = false;
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
+  if (warp == TPROD_WARP) {
+    // ---------------- token producer ----------------
     if (lane == 0) {
-      int ts = 0, ws = 0;
-      uint32_t tph = 0, wph = 0;
-      uint32_t tok_issued = 0, tok_par = 0, w8_issued = 0, w8_par = 0;
+      int ts = 0;
+      uint32_t tph = 0;
+      uint32_t issued = 0, par = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
         const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
         const Problem& P = p.pr[ti.prob];
@@ -215,113 +261,138 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
           ptx::fence_proxy_async_global();
         }
         const CUtensorMap* amap = ti.shared ? &P.a_s : &P.a_r;
-        const CUtensorMap* w0 = ti.shared ? &P.b0_s : &P.b0_r;
-        const CUtensorMap* w1 = ti.shared ? &P.b1_s : &P.b1_r;
         const int a_row = ti.shared ? ti.grp * P.a_s_group_stride + ti.m0 : ti.row0 + ti.m0;
-        const int w_row = ti.grp * (ti.shared ? P.b_s_group_rows : P.b_r_group_rows) + ti.n0;
-        const int K = ti.shared ? P.K_s : P.K_r;
-        const int nk = (K + BK - 1) / BK;
+        const int nk = tile_k_blocks(ti, P);
         const int nbox = (block_n<NT>(ti.rows - ti.m0) + TOK_BOX - 1) / TOK_BOX;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
-          const int x = kb * BK;
-          if (!ptx::mbar_wait(&ss.tok_empty[ts], tph ^ 1u, abort)) { ok = false; break; }
+          if (!ptx::mbar_wait(&ss.stage_empty[ts], tph ^ 1u, abort)) { ok = false; break; }
           uint8_t* st = tok_ring + ts * C::TOK_STAGE_BYTES;
           ptx::mbar_arrive_expect_tx(&ss.tok_full[ts], nbox * TOK_BOX_BYTES);
           for (int b = 0; b < nbox; ++b)
-            ptx::tma_load_2d(st + b * TOK_BOX_BYTES, amap, &ss.tok_full[ts], x, a_row + b * TOK_BOX);
-          tok_issued |= 1u << ts;
-          tok_par = (tok_par & ~(1u << ts)) | (tph << ts);
-          if (++ts == TS) { ts = 0; tph ^= 1u; }
-
-          if (!ptx::mbar_wait(&ss.w8_empty[ws], wph ^ 1u, abort)) { ok = false; break; }
-          uint8_t* sw = w8_ring + ws * W8_BYTES;
-          ptx::mbar_arrive_expect_tx(&ss.w8_full[ws], W8_BYTES);
-          ptx::tma_load_2d(sw, w0, &ss.w8_full[ws], x, w_row);
-          if (P.gateup) ptx::tma_load_2d(sw + W8_BYTES / 2, w1, &ss.w8_full[ws], x, w_row);
-          w8_issued |= 1u << ws;
-          w8_par = (w8_par & ~(1u << ws)) | (wph << ws);
-          if (++ws == W8_STAGES) { ws = 0; wph ^= 1u; }
+            ptx::tma_load_2d(st + b * TOK_BOX_BYTES, amap, &ss.tok_full[ts], kb * BK,
+                             a_row + b * TOK_BOX);
+          issued |= 1u << ts;
+          par = (par & ~(1u << ts)) | (tph << ts);
+          if (++ts == S) { ts = 0; tph ^= 1u; }
         }
         if (!ok) break;
       }
       // every issued load has landed before the CTA may retire
-      for (int s = 0; s < TS; ++s)
-        if (tok_issued & (1u << s)) wait_drain(&ss.tok_full[s], (tok_par >> s) & 1u, abort);
-      for (int s = 0; s < W8_STAGES; ++s)
-        if (w8_issued & (1u << s)) wait_drain(&ss.w8_full[s], (w8_par >> s) & 1u, abort);
+      for (int s = 0; s < S; ++s)
+        if (issued & (1u << s)) wait_drain(&ss.tok_full[s], (par >> s) & 1u, abort);
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == WPROD_WARP) {
+    // ---------------- weight producer ----------------
+    // Weights depend on nothing the kernel writes, so this warp runs ahead of
+    // the token producer (which may wait on the gate/up -> down hand-off) as
+    // far as the code ring allows.
     if (lane == 0) {
-      int ts = 0, as = 0, acc = 0;
-      uint32_t tph = 0, aph = 0, acc_phase = 0;
+      int ws = 0;
+      uint32_t wph = 0;
+      uint32_t issued = 0, par = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
         const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
         const Problem& P = p.pr[ti.prob];
-        const int K = ti.shared ? P.K_s : P.K_r;
-        const int nk = (K + BK - 1) / BK;
-        const uint32_t idesc = ptx::idesc_bf16_f32(W_ROWS, block_n<NT>(ti.rows - ti.m0));
-        if (!ptx::mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1u, abort)) break;
-        ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * NT;
+        const CUtensorMap* w0 = ti.shared ? &P.b0_s : &P.b0_r;
+        const CUtensorMap* w1 = ti.shared ? &P.b1_s : &P.b1_r;
+        const int w_row = ti.grp * (ti.shared ? P.b_s_group_rows : P.b_r_group_rows) + ti.n0;
+        const int nk = tile_k_blocks(ti, P);
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!ptx::mbar_wait(&ss.a_full[as], aph, abort) ||
-              !ptx::mbar_wait(&ss.tok_full[ts], tph, abort)) {
+          if (!ptx::mbar_wait(&ss.w8_empty[ws], wph ^ 1u, abort)) { ok = false; break; }
+          uint8_t* sw = w8_ring + ws * W8_BYTES;
+          ptx::mbar_arrive_expect_tx(&ss.w8_full[ws], W8_BYTES);
+          ptx::tma_load_2d(sw, w0, &ss.w8_full[ws], kb * BK, w_row);
+          if (P.gateup) ptx::tma_load_2d(sw + W8_BYTES / 2, w1, &ss.w8_full[ws], kb * BK, w_row);
+          issued |= 1u << ws;
+          par = (par & ~(1u << ws)) | (wph << ws);
+          if (++ws == W8S) { ws = 0; wph ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      for (int s = 0; s < W8S; ++s)
+        if (issued & (1u << s)) wait_drain(&ss.w8_full[s], (par >> s) & 1u, abort);
+    }
+  } else if (warp == MMA_WARP0 || (MW > 1 && warp == MMA_WARP1)) {
+    // ---------------- MMA issuers ----------------
+    // Issuer m takes the K-blocks kb with kb % MW == m of every tile into
+    // accumulator D_m; all issuers walk the same stage sequence.
+    const int m = warp == MMA_WARP0 ? 0 : 1;
+    if (lane == 0) {
+      int st = 0;
+      uint32_t sph = 0, acc_phase = 0;
+      const uint32_t d_tmem = tmem_base + m * NT;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
+        const Problem& P = p.pr[ti.prob];
+        const int nk = tile_k_blocks(ti, P);
+        const uint32_t idesc = ptx::idesc_bf16_f32(W_ROWS, block_n<NT>(ti.rows - ti.m0));
+        if (!ptx::mbar_wait(&ss.tmem_empty, acc_phase ^ 1u, abort)) break;
+        ptx::tc_fence_after();
+        bool ok = true;
+        uint32_t accumulate = 0;
+        for (int kb = 0; kb < nk; ++kb) {
+          const int cur = st;
+          const uint32_t cur_ph = sph;
+          if (++st == S) { st = 0; sph ^= 1u; }
+          if (kb % MW != m) continue;
+          if (!ptx::mbar_wait(&ss.a_full[cur], cur_ph, abort) ||
+              !ptx::mbar_wait(&ss.tok_full[cur], cur_ph, abort)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t a_tmem = tmem_base + A_COL0 + as * A_STAGE_COLS;
-          const uint32_t sb = ptx::smem_addr(tok_ring + ts * C::TOK_STAGE_BYTES);
+          const uint32_t a_tmem = tmem_base + A_COL0 + cur * A_STAGE_COLS;
+          // descriptor start-address field counts 16-byte units: +2 per K step
+          const uint64_t b_desc = ptx::smem_desc_sw128(ptx::smem_addr(tok_ring + cur * C::TOK_STAGE_BYTES));
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            ptx::mma_f16_ts(d_tmem, a_tmem + kk * 8, ptx::smem_desc_sw128(sb + kk * 32), idesc,
-                            (kb > 0 || kk > 0) ? 1u : 0u);
-          ptx::mma_commit(&ss.a_empty[as]);    // weight stage free when these MMAs finish
-          ptx::mma_commit(&ss.tok_empty[ts]);  // token stage likewise
-          if (++as == A_STAGES) { as = 0; aph ^= 1u; }
-          if (++ts == TS) { ts = 0; tph ^= 1u; }
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            ptx::mma_f16_ts(d_tmem, a_tmem + kk * 8, b_desc + 2 * kk, idesc, accumulate);
+            accumulate = 1;
+          }
+          ptx::mma_commit(&ss.stage_empty[cur]);   // token and weight stage free
         }
         if (!ok) break;
-        ptx::mma_commit(&ss.tmem_full[acc]);
-        if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
+        ptx::mma_commit(&ss.tmem_full);
+        acc_phase ^= 1u;
       }
-      ptx::mma_commit(&ss.drain);
-      wait_drain(&ss.drain, 0, abort);
+      ptx::mma_commit(&ss.drain[m]);
+      wait_drain(&ss.drain[m], 0, abort);
     }
-  } else if (warp < DEC_WARP0) {
+  } else if (warp >= 2 && warp < DEC_WARP0) {
     // ---------------- epilogue (warps 2..5) ----------------
     const int q = warp & 3;
-    int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
       const Problem& P = p.pr[ti.prob];
       const int n = block_n<NT>(ti.rows - ti.m0);
-      if (!ptx::mbar_wait(&ss.tmem_full[acc], acc_phase, abort)) break;
+      const bool two = MW > 1 && tile_k_blocks(ti, P) > 1;
+      if (!ptx::mbar_wait(&ss.tmem_full, acc_phase, abort)) break;
       ptx::tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * NT;
-      if (P.gateup) store_gateup(ti, P, taddr, n, q, lane);
-      else store_down(ti, P, taddr, n, q, lane);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      if (P.gateup) store_gateup(ti, P, taddr, NT, two, n, q, lane);
+      else store_down(ti, P, taddr, NT, two, n, q, lane);
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&ss.tmem_empty[acc]);
-      if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
+      if (lane == 0) ptx::mbar_arrive(&ss.tmem_empty);
+      acc_phase ^= 1u;
       if (p.nprob > 1 && ti.prob == 0) release_rows(p, ti, lane);
     }
-  } else {
-    // ---------------- weight decoders (warps 6..9) ----------------
+  } else if ((warp >= DEC_WARP0 && warp < DEC_WARP0 + 4) || warp >= DEC_WARP1) {
+    // ---------------- weight decoders (warps 6..9 and 12..15) ----------------
+    // Two sets of four warps take alternate stages; each warp decodes the 32
+    // weight rows of its TMEM lane quarter.
     const int q = warp & 3;
+    const int set = warp >= DEC_WARP1 ? 1 : 0;
     const uint32_t t_lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + A_COL0;
-    int ws = 0, as = 0;
+    int ws = 0, as = 0, seq = 0;
     uint32_t wph = 0, aph = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
       const Problem& P = p.pr[ti.prob];
-      const int K = ti.shared ? P.K_s : P.K_r;
-      const int nk = (K + BK - 1) / BK;
+      const int nk = tile_k_blocks(ti, P);
       // this thread's weight row: gate/up stacks the W1 box (64 rows) and the
       // W3 box; lanes 0-15 of quarter q take W1 rows 16q.., lanes 16-31 the
       // W3 rows of the same features; down takes row 32q + lane of one box
@@ -335,15 +406,20 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       const int8_t* ex_row = ex + ((size_t)ti.grp * rbn + ti.n0 / fp8::kBlock) * kbn;
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
-        if (!ptx::mbar_wait(&ss.w8_full[ws], wph, abort)) { ok = false; break; }
-        const uint8_t* rowp = w8_ring + ws * W8_BYTES + row_off;
+        const int my_ws = ws, my_as = as;
+        const uint32_t my_wph = wph, my_aph = aph;
+        if (++ws == W8S) { ws = 0; wph ^= 1u; }
+        if (++as == S) { as = 0; aph ^= 1u; }
+        if ((seq++ & 1) != set) continue;
+        // the exponent load goes out first; the stage wait hides its latency
+        const int e = ex_row[(kb * BK) / fp8::kBlock];
+        if (!ptx::mbar_wait(&ss.w8_full[my_ws], my_wph, abort)) { ok = false; break; }
+        const uint8_t* rowp = w8_ring + my_ws * W8_BYTES + row_off;
         uint4 c4[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           c4[c] = *reinterpret_cast<const uint4*>(rowp + ((c ^ swz) << 4));
-        ptx::mbar_arrive(&ss.w8_empty[ws]);
-        if (++ws == W8_STAGES) { ws = 0; wph ^= 1u; }
-        const int e = ex_row[(kb * BK) / fp8::kBlock];
+        ptx::mbar_arrive(&ss.w8_empty[my_ws]);
         bad_exp |= !fp8::exp_ok(e);
         const uint32_t s2 = fp8::scale_pair(e);
         uint32_t w[32];
@@ -354,13 +430,13 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
           fp8::decode4(c4[c].z, s2, w[8 * c + 4], w[8 * c + 5]);
           fp8::decode4(c4[c].w, s2, w[8 * c + 6], w[8 * c + 7]);
         }
-        if (!ptx::mbar_wait(&ss.a_empty[as], aph ^ 1u, abort)) { ok = false; break; }
+        // the stage's previous K-block has been read by its MMAs
+        if (!ptx::mbar_wait(&ss.stage_empty[my_as], my_aph ^ 1u, abort)) { ok = false; break; }
         ptx::tc_fence_after();
-        ptx::tmem_st_x32(t_lanes + as * A_STAGE_COLS, w);
+        ptx::tmem_st_x32(t_lanes + my_as * A_STAGE_COLS, w);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&ss.a_full[as]);
-        if (++as == A_STAGES) { as = 0; aph ^= 1u; }
+        ptx::mbar_arrive(&ss.a_full[my_as]);
       }
       if (!ok) break;
     }
@@ -369,7 +445,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
   if (bad_exp && p.status) atomicOr(p.status, kStBounds);
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == MMA_WARP0) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, TMEM_COLS);
   }
@@ -378,7 +454,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
 
 template <int NT>
 constexpr size_t smem_bytes8() {
-  return 1024 + Cfg<NT>::TOK_STAGES * Cfg<NT>::TOK_STAGE_BYTES + W8_STAGES * W8_BYTES +
+  return 1024 + Cfg<NT>::STAGES * Cfg<NT>::TOK_STAGE_BYTES + Cfg<NT>::W8_STAGES * W8_BYTES +
          sizeof(SharedState8);
 }
 static_assert(smem_bytes8<256>() <= 227 * 1024 && smem_bytes8<128>() <= 227 * 1024,
@@ -409,8 +485,8 @@ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 }  // namespace
 
-// Batches of at most 128 tokens fit every group in one 128-token block and
-// double-buffer the accumulator; larger batches use 256-token blocks.
+// Batches of at most 128 tokens fit every group in one 128-token block (two
+// MMA issuers); larger batches use 256-token blocks.
 cudaError_t launch_expert_ffn_fp8(const FfnArgs& a, const Fp8Weights& w, cudaStream_t st,
                                   int* nlaunch, const char** why, void* const* marks) {
   const bool small = a.T <= 128;
