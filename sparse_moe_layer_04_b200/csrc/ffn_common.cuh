@@ -195,13 +195,32 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, volat
   if (!ptx::mbar_wait(bar, parity, &ignore_abort)) *abort = 1;
 }
 
+// 16 accumulator columns of this warp's lane quarter: D0, plus D1 (d1_off
+// columns further) when the tile's K-blocks were split between two
+// accumulators.
+__device__ __forceinline__ void load_acc16(uint32_t taddr, uint32_t d1_off, bool two,
+                                           uint32_t (&v)[16]) {
+  ptx::tmem_ld_x16(taddr, v);
+  if (two) {
+    uint32_t u[16];
+    ptx::tmem_ld_x16(taddr + d1_off, u);
+    ptx::tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(u[j]));
+  } else {
+    ptx::tmem_wait_ld();
+  }
+}
+
 // Epilogue of one accumulator tile (warp quarter q of the four epilogue
 // warps): gate/up tiles apply the SiLU gate (gate in TMEM columns [0, HALF),
 // up in [HALF, 2 HALF)) and store bf16; down tiles store fp32.  `taddr` is the
-// warp's TMEM lane quarter at the accumulator's first column.
+// warp's TMEM lane quarter at the accumulator's first column; with `two` the
+// tile is the sum of that accumulator and the one d1_off columns further.
 template <int MMA_N>
 __device__ __forceinline__ void store_tile(const TileInfo& ti, const Problem& P, uint32_t taddr,
-                                           int q, int lane) {
+                                           uint32_t d1_off, bool two, int q, int lane) {
   constexpr int HALF = MMA_N / 2;
   const int r = ti.m0 + q * 32 + lane;       // row within the group
   const bool row_ok = r < ti.rows;
@@ -212,9 +231,8 @@ __device__ __forceinline__ void store_tile(const TileInfo& ti, const Problem& P,
 #pragma unroll 1
     for (int c = 0; c < HALF; c += 16) {
       uint32_t g[16], u[16];
-      ptx::tmem_ld_x16(taddr + c, g);
-      ptx::tmem_ld_x16(taddr + HALF + c, u);
-      ptx::tmem_wait_ld();
+      load_acc16(taddr + c, d1_off, two, g);
+      load_acc16(taddr + HALF + c, d1_off, two, u);
       const int col = ti.n0 + c;
       if (row_ok && col < N) {
         uint32_t pk[8];
@@ -233,8 +251,7 @@ __device__ __forceinline__ void store_tile(const TileInfo& ti, const Problem& P,
 #pragma unroll 1
     for (int c = 0; c < MMA_N; c += 16) {
       uint32_t v[16];
-      ptx::tmem_ld_x16(taddr + c, v);
-      ptx::tmem_wait_ld();
+      load_acc16(taddr + c, d1_off, two, v);
       const int col = ti.n0 + c;
       if (row_ok && col < N) {
         uint4* dst = reinterpret_cast<uint4*>(out + out_row * N + col);

@@ -33,15 +33,19 @@
 // finer to keep all 148 SMs busy.  The same kernel also computes the router
 // logits as a dense split-K GEMM (one problem, one shared group per K chunk).
 //
-// CTA structure (192 threads, one CTA per SM):
+// CTA structure (224 threads, one CTA per SM):
 //   warp 0      TMA producer: ring of (A 128x64, B Nx64) bf16 tiles (4 stages
 //               for N = 256, 6 for N = 128), 128-byte swizzled, completion
 //               counted on "full" mbarriers.
-//   warp 1      TMEM allocator and single-thread MMA issuer:
+//   warp 1      TMEM allocator (512 columns) and MMA issuer:
 //               tcgen05.mma.cta_group::1.kind::f16, M = 128, N, K = 16,
 //               fp32 accumulators in TMEM, two accumulator buffers so the
 //               epilogue of tile i overlaps the main loop of tile i+1.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//   warp 6      second MMA issuer for N = 128: a thread issues one
+//               tcgen05.mma per ~100 cycles at best, longer than an N = 128
+//               MMA runs, so warps 1 and 6 take alternate K-blocks of a tile
+//               into two accumulators of its buffer (idle for N = 256).
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator(s) (warp w reads TMEM
 //               lanes 32*(w%4) .. +31), fused activation, global stores.
 #include <cuda_bf16.h>
 
@@ -52,7 +56,8 @@ namespace {
 
 using namespace ffn;
 
-constexpr int THREADS = 192;
+constexpr int THREADS = 224;             // warps 0-5 and the second MMA issuer (warp 6)
+constexpr int MMA_WARP1 = 6;
 constexpr int RING_BYTES = 192 * 1024;    // operand ring budget
 constexpr int MAX_STAGES = 6;
 
@@ -62,7 +67,13 @@ struct Shape {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = RING_BYTES / STAGE_BYTES;    // 4 (N=256) or 6 (N=128)
   static constexpr int ACC_COLS = MMA_N;                     // fp32 TMEM columns per accumulator
-  static constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;        // double buffered
+  // One thread issues a tcgen05.mma every ~100 cycles at best, longer than an
+  // N = 128 MMA executes: N = 128 tiles split their K-blocks between two
+  // issuing warps with an accumulator each (the epilogue adds them).
+  static constexpr int MMA_WARPS = MMA_N == 128 ? 2 : 1;
+  static constexpr int BUF_COLS = MMA_WARPS * ACC_COLS;      // one accumulator buffer
+  static constexpr uint32_t TMEM_COLS = 2 * BUF_COLS;        // double buffered
+  static_assert(TMEM_COLS <= 512, "TMEM columns");
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, MMA_N);
 };
 
@@ -71,7 +82,7 @@ struct SharedState {
   uint64_t empty[MAX_STAGES];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
   TileMap tm;
@@ -85,6 +96,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   constexpr int ACC_COLS = Sh::ACC_COLS;
   constexpr uint32_t TMEM_COLS = Sh::TMEM_COLS;
   constexpr uint32_t IDESC = Sh::IDESC;
+  constexpr int MW = Sh::MMA_WARPS;
+  constexpr int BUF_COLS = Sh::BUF_COLS;
   constexpr int HALF = MMA_N / 2;  // gate/up: W1 rows [0, HALF), W3 rows [HALF, MMA_N)
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned operand ring (128-byte swizzle atoms span 1024 bytes)
@@ -106,10 +119,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       ptx::mbar_init(&ss.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(&ss.tmem_full[i], 1);
+      ptx::mbar_init(&ss.tmem_full[i], MW);
       ptx::mbar_init(&ss.tmem_empty[i], 4);
     }
-    ptx::mbar_init(&ss.drain, 1);
+    ptx::mbar_init(&ss.drain[0], 1);
+    ptx::mbar_init(&ss.drain[1], 1);
     ss.abort = 0;
     ptx::fence_barrier_init();
   }
@@ -180,8 +194,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       for (int s = 0; s < STAGES; ++s)
         if (issued_mask & (1u << s)) wait_drain(&ss.full[s], (last_parity >> s) & 1u, abort);
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == 1 || (MW > 1 && warp == MMA_WARP1)) {
+    // ---------------- MMA issuers ----------------
+    // Issuer m takes the K-blocks kb with kb % MW == m of every tile into
+    // accumulator m of the tile's buffer; all issuers walk the same stages.
+    const int m = warp == 1 ? 0 : 1;
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -194,30 +211,35 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         const int nk = (K + BK - 1) / BK;
         if (!ptx::mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1u, abort)) break;
         ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        const uint32_t d_tmem = tmem_base + acc * BUF_COLS + m * ACC_COLS;
         bool ok = true;
+        uint32_t accumulate = 0;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!ptx::mbar_wait(&ss.full[stage], phase, abort)) { ok = false; break; }
+          const int cur = stage;
+          const uint32_t cur_phase = phase;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (kb % MW != m) continue;
+          if (!ptx::mbar_wait(&ss.full[cur], cur_phase, abort)) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t sa = ptx::smem_addr(ring + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_BYTES;
+          const uint32_t sa = ptx::smem_addr(ring + cur * STAGE_BYTES);
+          // descriptor start-address fields count 16-byte units: +2 per K step
+          const uint64_t a_desc = ptx::smem_desc_sw128(sa);
+          const uint64_t b_desc = ptx::smem_desc_sw128(sa + A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            ptx::mma_f16_ss(d_tmem, ptx::smem_desc_sw128(sa + kk * 32),
-                            ptx::smem_desc_sw128(sb + kk * 32), IDESC,
-                            (kb > 0 || kk > 0) ? 1u : 0u);
+            ptx::mma_f16_ss(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, IDESC, accumulate);
+            accumulate = 1;
           }
-          ptx::mma_commit(&ss.empty[stage]);   // frees the smem stage when these MMAs finish
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          ptx::mma_commit(&ss.empty[cur]);     // frees the smem stage when these MMAs finish
         }
         if (!ok) break;
         ptx::mma_commit(&ss.tmem_full[acc]);   // accumulator ready for the epilogue
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
-      ptx::mma_commit(&ss.drain);
-      wait_drain(&ss.drain, 0, abort);
+      ptx::mma_commit(&ss.drain[m]);
+      wait_drain(&ss.drain[m], 0, abort);
     }
-  } else {
+  } else if (warp >= 2 && warp < 6) {
     // ---------------- epilogue (warps 2..5) ----------------
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
@@ -225,10 +247,13 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
       const Problem& P = p.pr[ti.prob];
+      int kbeg, K;
+      tile_k_range(ti, P, &kbeg, &K);
+      const bool two = MW > 1 && K > BK;   // the second accumulator holds K-blocks
       if (!ptx::mbar_wait(&ss.tmem_full[acc], acc_phase, abort)) break;
       ptx::tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * ACC_COLS;
-      store_tile<MMA_N>(ti, P, taddr, q, lane);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BUF_COLS;
+      store_tile<MMA_N>(ti, P, taddr, ACC_COLS, two, q, lane);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ss.tmem_empty[acc]);
