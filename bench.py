@@ -114,9 +114,19 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def source_digest(paths) -> str:
+    """First 16 hex digits of the SHA-256 of the given source files, concatenated."""
+    import hashlib
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def stored_traffic(kernel_key: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+    the current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -124,13 +134,11 @@ def stored_traffic(kernel_key: str):
         rec = json.load(f).get(kernel_key)
     if not rec:
         return None
-    import hashlib
-    src = os.path.join(ROOT, rec["source"])
-    if not os.path.exists(src):
+    srcs = rec["sources"]
+    if not all(os.path.exists(os.path.join(ROOT, s)) for s in srcs):
         return None
-    with open(src, "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest()[:16] != rec["source_sha256_16"]:
-            return None
+    if source_digest(srcs) != rec["sources_sha256_16"]:
+        return None
     return rec["dram_bytes_per_launch"]
 
 
