@@ -172,6 +172,7 @@ class ClockSampler:
             self.proc.kill()
             out, _ = self.proc.communicate()
         mhz, maxs, reasons = [], [], set()
+        capped = 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
@@ -185,10 +186,12 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
+            capped += parts[8].lower() == "active"
         if not mhz:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxs),
-                "reasons": sorted(reasons), "samples": len(mhz)}
+                "reasons": sorted(reasons), "samples": len(mhz),
+                "power_cap_fraction": capped / len(mhz)}
 
 
 # ---------------------------------------------------------------------------
@@ -375,7 +378,16 @@ def run_ours(args, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     hbm = float(peaks["hbm_gbs"])
-    bf16 = float(peaks["bf16_tflops"])
+    bf16_burst = float(peaks["bf16_tflops"])
+    bf16_sust = float(peaks.get("bf16_tflops_sustained", bf16_burst))
+    # The tensor denominator: the burst figure for a step the power cap left
+    # alone, the sustained one when the clock record of the run shows the power
+    # cap active in at least a quarter of the samples (long tensor-heavy steps
+    # run at the capped clock).  Both fractions are reported.
+    capped = bool(clocks) and clocks.get("power_cap_fraction", 0.0) >= 0.25
+    bf16 = bf16_sust if capped else bf16_burst
+    tc_peak_choice = ("sustained (sw_power_cap active in >= 25% of the clock samples)" if capped
+                      else "burst (power cap active in < 25% of the clock samples)")
     B, FL = layer_bytes_flops(cfg, U, args.weights)
     t_s = ms / 1e3
     t_roof_hbm = B / (hbm * 1e9)
@@ -396,6 +408,8 @@ def run_ours(args, rank, world, local_rank):
               if fp8 is not None else "grouped_gemm_kernel (fused gate/up + down expert FFN)")
     roof.update({"traffic": stored_traffic(traffic_key), "kernel": kernel, "ms": ffn_ms,
                  "algorithmic_bytes": f_bytes, "algorithmic_flops": f_flops,
+                 "tensor_peak": tc_peak_choice,
+                 "tensor_frac_burst": f_tfs / bf16_burst, "tensor_frac_sustained": f_tfs / bf16_sust,
                  "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured"
                  else "fallback (profiling recipe)"})
 
@@ -431,7 +445,11 @@ def run_ours(args, rank, world, local_rank):
             "binding": "hbm" if t_roof_hbm >= t_roof_tc else "tensor",
             "frac": max(t_roof_hbm, t_roof_tc) / t_s,
             "hbm_frac": t_roof_hbm / t_s, "tensor_frac": t_roof_tc / t_s,
-            "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "source": peak_src}},
+            "tensor_frac_burst": FL / (bf16_burst * 1e12) / t_s,
+            "tensor_frac_sustained": FL / (bf16_sust * 1e12) / t_s,
+            "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "bf16_tflops_burst": bf16_burst,
+                      "bf16_tflops_sustained": bf16_sust, "tensor_peak": tc_peak_choice,
+                      "source": peak_src}},
         "e2e": {"value": aggregate_tokens_per_s(cfg.T, world, e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": cfg.T * cfg.D * 2, "d2h_bytes_per_step": cfg.T * cfg.D * 4,
                 "ms_per_step": e2e},
