@@ -255,6 +255,17 @@ int moe_forward_fp8(const void* h, const float* Wr, const float* bias, const moe
 int moe_fp8_dequantize(const void* codes, const int8_t* exps, int G, int R, int K, void* out,
                        void* ws, moe_stream_t stream);
 
+/* Row gather, the data movement around the expert-parallel exchange (each
+ * rank owns a block of experts; the pages' default multi-GPU layout is expert
+ * parallelism, "GLM-5.2" PocketLLM, Implemented execution path):
+ *   dst[i] = src[idx[i]],  i < n,
+ * rows of row_bytes bytes (a positive multiple of 16), src [src_rows, row_bytes]
+ * and dst [n, row_bytes] device buffers (16-byte aligned), idx [n] int32.  An
+ * index outside [0, src_rows) zero-fills its row and raises MOE_ERR_BOUNDS in
+ * the status word of ws (ws may be NULL: then it is not reported). */
+int moe_gather_rows(const void* src, int src_rows, const int32_t* idx, int n, int row_bytes,
+                    void* dst, void* ws, moe_stream_t stream);
+
 /* Routing statistics of the last moe_forward (or moe_permute) that used
  * `ws` with these dims: device pointers into the workspace, valid once the
  * stream has reached the end of that call and until the next call reuses the

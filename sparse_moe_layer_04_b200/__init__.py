@@ -90,6 +90,7 @@ def _load() -> ctypes.CDLL:
         "moe_expert_ffn_fp8": (I, [P, P, P, W8, D, P, P, Z, P]),
         "moe_forward_fp8": (I, [P, P, P, W8, D, P, P, P, P, Z, P]),
         "moe_fp8_dequantize": (I, [P, P, I, I, I, P, P, P]),
+        "moe_gather_rows": (I, [P, I, P, I, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -243,6 +244,19 @@ def moe_fp8_dequantize(codes, exps, out, ws=None, stream=None) -> None:
     _check(_lib.moe_fp8_dequantize(_code_ptr(codes, "codes"), _ptr(exps, torch.int8, "exps"),
                                    G, R, K, _ptr(out, torch.bfloat16, "out"), wp,
                                    _stream(stream)))
+
+
+def moe_gather_rows(src, idx, dst, ws=None, stream=None) -> None:
+    """dst[i] = src[idx[i]] (rows of any dtype, a multiple of 16 bytes wide)."""
+    if src.dim() != 2 or dst.dim() != 2 or src.shape[1] != dst.shape[1] or src.dtype != dst.dtype:
+        raise ValueError("src [rows, W] and dst [n, W] with one dtype expected")
+    if idx.numel() != dst.shape[0]:
+        raise ValueError("idx must have one entry per dst row")
+    wp, _ = _ws(ws)
+    row_bytes = src.shape[1] * src.element_size()
+    _check(_lib.moe_gather_rows(_ptr(src, None, "src"), src.shape[0], _ptr(idx, torch.int32, "idx"),
+                                idx.numel(), row_bytes, _ptr(dst, None, "dst"), wp,
+                                _stream(stream)))
 
 
 def moe_combine(y, w, inv, d, out, ws=None, stream=None) -> None:

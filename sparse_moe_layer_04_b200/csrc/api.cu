@@ -635,6 +635,28 @@ int moe_fp8_dequantize(const void* codes, const int8_t* exps, int G, int R, int 
   return MOE_OK;
 }
 
+int moe_gather_rows(const void* src, int src_rows, const int32_t* idx, int n, int row_bytes,
+                    void* dst, void* ws, moe_stream_t stream) {
+  g_err.clear();
+  g_launches = 0;
+  if (src_rows < 0 || n < 0) return fail(MOE_ERR_INVALID_ARG, "src_rows and n must be >= 0");
+  if (row_bytes <= 0 || row_bytes % 16)
+    return fail(MOE_ERR_INVALID_ARG, "row_bytes = %d is not a positive multiple of 16", row_bytes);
+  if (n == 0) return MOE_OK;
+  MOE_CHECK_PTR(src);
+  MOE_CHECK_PTR(idx);
+  MOE_CHECK_PTR(dst);
+  if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return fail(MOE_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  int rc = check_device();
+  if (rc) return rc;
+  cudaError_t e = launch_gather_bytes(src, src_rows, idx, n, row_bytes, dst, static_cast<int*>(ws),
+                                      reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  g_launches = 1;
+  return MOE_OK;
+}
+
 const int32_t* moe_ws_expert_counts(const void* ws, const moe_dims_t* dims) {
   if (!ws || check_dims(dims) != MOE_OK) return nullptr;
   WsLayout L;

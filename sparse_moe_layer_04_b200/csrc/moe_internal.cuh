@@ -126,6 +126,10 @@ cudaError_t launch_expert_ffn_fp8(const FfnArgs& a, const Fp8Weights& w, cudaStr
 cudaError_t launch_fp8_dequantize(const uint8_t* codes, const int8_t* exps, int G, int R, int K,
                                   uint16_t* out, int* status, cudaStream_t st);
 
+// dst[i] = src[idx[i]] for n rows of row_bytes (a multiple of 16) bytes.
+cudaError_t launch_gather_bytes(const void* src, int src_rows, const int32_t* idx, int n,
+                                int row_bytes, void* dst, int* status, cudaStream_t st);
+
 int num_sms();
 
 cudaError_t launch_bounded_wait_selftest(int* status, cudaStream_t st);

@@ -175,3 +175,14 @@ def test_fp8_dequantize_argument_checks(mod):
     assert lib.moe_fp8_dequantize(FAKE + 1, FAKE, 1, 4, 16, FAKE, None, None) == mod.MOE_ERR_INVALID_ARG
     assert lib.moe_fp8_dequantize(FAKE, FAKE, 1, 4, 16, FAKE, FAKE + 16, None) == mod.MOE_ERR_WORKSPACE
     assert lib.moe_fp8_dequantize(None, None, 0, 4, 16, None, None, None) == mod.MOE_OK
+
+
+def test_gather_rows_argument_checks(mod):
+    lib = mod._lib
+    assert lib.moe_gather_rows(FAKE, 10, FAKE, 4, 24, FAKE, None, None) == mod.MOE_ERR_INVALID_ARG
+    assert "multiple of 16" in mod.moe_last_error()
+    assert lib.moe_gather_rows(FAKE, -1, FAKE, 4, 32, FAKE, None, None) == mod.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather_rows(FAKE + 8, 10, FAKE, 4, 32, FAKE, None, None) == mod.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather_rows(FAKE, 10, None, 4, 32, FAKE, None, None) == mod.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather_rows(FAKE, 10, FAKE, 4, 32, FAKE, FAKE + 16, None) == mod.MOE_ERR_WORKSPACE
+    assert lib.moe_gather_rows(None, 0, None, 0, 32, None, None, None) == mod.MOE_OK
