@@ -165,7 +165,7 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
   L->perm = take(T * k * 4);
   L->inv = take(T * k * 4);
   L->blk_base = take(nblk * E * 4);
-  L->counters = take((E + S) * 4);
+  L->counters = take((E + S + 1) * 4);   // per-group counters + the tile claim counter
   L->xperm = take(T * k * D * 2);
   L->act_r = take(T * k * F * 2);
   L->act_s = take(S * T * Fs * 2);
@@ -293,7 +293,7 @@ int expert_ffn_impl(const void* h, const int32_t* perm, const int32_t* offsets,
   uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
   int32_t* counters = w.at<int32_t>(w.L.counters);
   cudaError_t e = launch_gather_rows(hb, perm, rows, dims->D, dims->T, xperm, counters,
-                                     dims->E + dims->S, st);
+                                     dims->E + dims->S + 1, st);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   const FfnArgs a = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
   int n = 1;
@@ -343,7 +343,7 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
   if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
   int32_t* counters = w.at<int32_t>(w.L.counters);
-  e = launch_gather_rows(hb, perm, T * k, D, T, xperm, counters, E + dims->S, st);
+  e = launch_gather_rows(hb, perm, T * k, D, T, xperm, counters, E + dims->S + 1, st);
   if (e == cudaSuccess) e = mark(4, st);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   n += 1;

@@ -53,6 +53,7 @@ struct GemmParams {
   const int32_t* offsets;    // [E+1] routed group row offsets (E > 0)
   int* status;
   int* counters;             // [E+S] gate/up tiles stored per group (two problems)
+  int* sched;                // tile claim counter, zero at launch; nullptr: static round-robin
   int nprob;                 // 1 or 2
   int E, S, T;
   int rows_r;                // T * k
@@ -178,6 +179,18 @@ __device__ __forceinline__ void tile_k_range(const TileInfo& ti, const Problem& 
     *K = ti.shared ? P.K_s : P.K_r;
   }
 }
+
+// Tile scheduling.  CTA c starts with tile c; later tiles are claimed in
+// increasing order from a global counter (the first claim returns gridDim.x),
+// so CTAs that finish early take more tiles; without a counter, CTA c takes
+// c, c + gridDim.x, ...  Either way every tile below a claimed one has been
+// taken by a running CTA, which the gate/up -> down hand-off relies on.
+__device__ __forceinline__ int claim_tile(const GemmParams& p, int tile) {
+  return p.sched ? (int)gridDim.x + atomicAdd(p.sched, 1) : tile + (int)gridDim.x;
+}
+
+// Queue of claimed tiles from the producer to the other roles of the CTA.
+constexpr int TILE_Q = 4;
 
 __device__ __forceinline__ float silu_times(float g, float u) {
   return g / (1.0f + __expf(-g)) * u;

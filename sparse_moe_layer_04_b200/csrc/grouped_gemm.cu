@@ -19,14 +19,20 @@
 // Tiles are numbered problem 0 first, then problem 1; within a problem routed
 // experts first (expert, column tile, row tile with the row tile fastest, so
 // CTAs running at the same time share each weight tile through L2), then the
-// shared experts.  CTA c takes tiles c, c + gridDim.x, ...  A down tile of an
+// shared experts.  CTA c takes tile c first and then claims further tiles in
+// increasing order from a counter in the workspace (zeroed by the row-gather
+// kernel), so CTAs that finish early take more tiles; the producer passes each
+// claimed tile to the MMA and epilogue warps through a small shared-memory
+// queue (the router GEMM, which has no such counter, takes c, c + gridDim.x,
+// ...).  A down tile of an
 // expert waits until every gate/up tile of that expert has been stored: each
 // gate/up epilogue warp releases a per-expert counter after a proxy fence, and
 // the producer acquires it before its TMA loads read the activations.  Down tiles
 // therefore fill the SMs that the tail of the gate/up tiles leaves idle.
-// Because every CTA takes its tiles in increasing order and all CTAs are
-// resident (one per SM), every counter a CTA waits on is advanced by tiles that
-// precede it, so the waits always end; they are bounded all the same.
+// Because tiles are taken in increasing order and all CTAs are resident (one
+// per SM), every counter a CTA waits on is advanced by tiles that precede it
+// and are held by running CTAs, so the waits always end; they are bounded all
+// the same.
 //
 // N (the MMA width) is 256 for large batches and 128 for small ones, where
 // each expert has only a row tile or two and the weight stream must be cut
@@ -80,6 +86,8 @@ struct Shape {
 struct SharedState {
   uint64_t full[MAX_STAGES];
   uint64_t empty[MAX_STAGES];
+  uint64_t tq_full[TILE_Q], tq_empty[TILE_Q];
+  int tq_tile[TILE_Q];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t drain[2];
@@ -124,6 +132,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     }
     ptx::mbar_init(&ss.drain[0], 1);
     ptx::mbar_init(&ss.drain[1], 1);
+    for (int i = 0; i < TILE_Q; ++i) {
+      ptx::mbar_init(&ss.tq_full[i], 1);
+      ptx::mbar_init(&ss.tq_empty[i], MW + EPI_WARPS);
+    }
     ss.abort = 0;
     ptx::fence_barrier_init();
   }
@@ -152,7 +164,17 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued_mask = 0, last_parity = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int qslot = 0;
+      uint32_t qphase = 0;
+      int tile = blockIdx.x;
+      int next = tile < total ? claim_tile(p, tile) : total;
+      for (;;) {
+        // hand the tile (or the end mark) to the MMA and epilogue warps
+        if (!ptx::mbar_wait(&ss.tq_empty[qslot], qphase ^ 1u, abort)) break;
+        ss.tq_tile[qslot] = tile < total ? tile : -1;
+        ptx::mbar_arrive(&ss.tq_full[qslot]);
+        if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+        if (tile >= total) break;
         const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
         const Problem& P = p.pr[ti.prob];
         if (ti.prob == 1) {
@@ -189,6 +211,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
+        tile = next;
+        next = tile < total ? claim_tile(p, tile) : total;
       }
       // every issued load has landed before the CTA may retire
       for (int s = 0; s < STAGES; ++s)
@@ -204,7 +228,14 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int qslot = 0;
+      uint32_t qphase = 0;
+      for (;;) {
+        if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
+        const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
+        ptx::mbar_arrive(&ss.tq_empty[qslot]);
+        if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+        if (tile < 0) break;
         const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
         int kbeg, K;
         tile_k_range(ti, p.pr[ti.prob], &kbeg, &K);
@@ -244,7 +275,15 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    int qslot = 0;
+    uint32_t qphase = 0;
+    for (;;) {
+      if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
+      const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&ss.tq_empty[qslot]);
+      if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+      if (tile < 0) break;
       const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
       const Problem& P = p.pr[ti.prob];
       int kbeg, K;
@@ -447,6 +486,7 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, c
   p.offsets = a.offsets;
   p.status = a.status;
   p.counters = a.counters;
+  p.sched = a.counters + a.E + a.S;   // zeroed with the group counters
   p.nprob = 2;
   p.E = a.E; p.S = a.S; p.T = a.T;
   p.rows_r = rows_r;

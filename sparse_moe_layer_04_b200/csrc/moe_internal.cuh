@@ -89,7 +89,8 @@ cudaError_t launch_route_grouped(const float* logits, const float* bias, int T, 
 cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* blk_base,
                            int* status, int32_t* touched, cudaStream_t st, int* nlaunch);
-// Also zeroes the expert FFN's per-group counters (`ncounters` ints).
+// Also zeroes the expert FFN's per-group counters and tile claim counter
+// (`ncounters` ints).
 cudaError_t launch_gather_rows(const uint16_t* h, const int32_t* perm, int rows, int D, int T,
                                uint16_t* xperm, int* counters, int ncounters, cudaStream_t st);
 cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, int T, int D,
@@ -105,7 +106,7 @@ struct FfnArgs {
   uint16_t* act_s;          // [S*T, Fs]
   float* y;                 // [T*k + S*T, D]
   int* status;
-  int* counters;            // [E + S], zero at launch
+  int* counters;            // [E + S + 1], zero at launch (group counters, tile claims)
   int T, D, E, F, k, S, Fs;
 };
 // `marks` (nullable): one event recorded after the expert FFN kernel.
