@@ -192,6 +192,11 @@ __device__ __forceinline__ int claim_tile(const GemmParams& p, int tile) {
 // Queue of claimed tiles from the producer to the other roles of the CTA.
 constexpr int TILE_Q = 4;
 
+// K-blocks of a tile padded to whole rounds of `m` issuers: the padding
+// stages go through the ring's barriers with no data and no MMA, so every
+// tile starts on stage 0 of a round and stage s always meets issuer s % m.
+__device__ __forceinline__ int round_up(int n, int m) { return (n + m - 1) / m * m; }
+
 __device__ __forceinline__ float silu_times(float g, float u) {
   return g / (1.0f + __expf(-g)) * u;
 }

@@ -31,22 +31,23 @@
 //   warp 0      token producer: TMA of token tiles (bf16, 128-byte swizzle,
 //               boxes of 64 rows); waits for the gate/up -> down hand-off.
 //   warp 10     weight producer: TMA of FP8 weight tiles (64-byte swizzle) on
-//               a 12-stage ring of its own, running ahead of the tokens.
+//               a ring of its own (12 stages for NT = 128, 8 for NT = 256),
+//               running ahead of the tokens.
 //   warps 1,11  MMA issuers (warp 1 also allocates the 512 TMEM columns):
 //               tcgen05.mma.cta_group::1.kind::f16, M = 128, N <= NT, K = 16.
-//               One issuing thread manages one tcgen05.mma per ~100 cycles,
-//               more than an M = 128, N = 128 MMA takes to execute, so for
-//               NT = 128 two warps take alternate K-blocks into two
-//               accumulators; one commit per K-block frees both the token
-//               stage and the decoded-weight stage.
-//   warps 2-5   epilogue (tcgen05.ld of both accumulators, SiLU gate or fp32
+//               The weights are bf16 in the MMA, so a stage of 8 KB of codes
+//               costs as many MMAs as 16 KB of bf16 weights, and one thread
+//               issues a tcgen05.mma only every ~100+ cycles at N <= 128: for
+//               NT = 128 two warps take alternate K-blocks into an accumulator
+//               each (the epilogue adds them); one commit per K-block frees
+//               both the token and the decoded-weight stage.
+//   warps 2-5   epilogue (tcgen05.ld of the accumulators, SiLU gate or fp32
 //               store).
-//   warps 6-9,  decoders, two sets of four taking alternate stages: each warp
-//   12-15       reads its 32 weight rows of a stage (one row per thread, 64
-//               codes), decodes, and stores them to its TMEM lane quarter.
-//               One set alone needs about as long per stage as the MMAs.
-// TMEM columns: accumulators [0, 256) (two of 128 for NT = 128, one of 256
-// for NT = 256), decoded-weight stages from column 256 (32 columns each).
+//   warps 6-9,  decoders, two sets of four taking alternate stages: each
+//   12-15       warp reads its 32 weight rows of a stage (one row per thread,
+//               64 codes), decodes, and stores them to its TMEM lane quarter.
+// TMEM columns: accumulators first (two of 128 for NT = 128, one of 256 for
+// NT = 256), then the decoded-weight stages (32 columns each).
 #include <cuda_bf16.h>
 
 #include "ffn_common.cuh"
@@ -63,18 +64,25 @@ constexpr int TOK_BOX = 64;                      // token rows per TMA box
 constexpr int TOK_BOX_BYTES = TOK_BOX * BK * 2;  // 8 KiB
 constexpr int W8_BYTES = W_ROWS * BK;            // 8 KiB of codes per stage
 constexpr uint32_t A_STAGE_COLS = BK / 2;        // 128 lanes x 64 bf16
-constexpr uint32_t A_COL0 = 256;                 // weight stages follow the accumulators
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int TPROD_WARP = 0;                    // token producer
 constexpr int MMA_WARP0 = 1;                     // MMA issuer (and TMEM allocator)
-constexpr int DEC_WARP0 = 6;                     // decoder set 0: warps 6..9
 constexpr int WPROD_WARP = 10;                   // weight producer
-constexpr int MMA_WARP1 = 11;                    // second MMA issuer (NT = 128)
-constexpr int DEC_WARP1 = 12;                    // decoder set 1: warps 12..15
-constexpr int THREADS = 512;
+constexpr int MMA_WARP1 = 11;                    // further MMA issuers (NT = 128)
+constexpr int MAX_MMA_WARPS = 2;
+constexpr int DEC_SETS = 2;                      // decoder sets: warps 6-9, 12-15
+constexpr int THREADS = 16 * 32;
 constexpr int DEC_THREADS = 128;
 constexpr int MAX_STAGES = 6;
-constexpr int MAX_W8_STAGES = 12;
+constexpr int MAX_W8_STAGES = 16;
+
+// Role of a warp: MMA issuer index (or -1) and decoder set (or -1).
+__device__ __forceinline__ int mma_index(int warp) {
+  return warp == MMA_WARP0 ? 0 : warp == MMA_WARP1 ? 1 : -1;
+}
+__device__ __forceinline__ int decoder_set(int warp) {
+  return (warp >= 6 && warp < 10) ? 0 : (warp >= 12 && warp < 16) ? 1 : -1;
+}
 
 // Per-NT configuration.
 //   STAGES     depth of the token ring and of the decoded-weight ring in TMEM;
@@ -85,16 +93,23 @@ constexpr int MAX_W8_STAGES = 12;
 //   MMA_WARPS  a single thread issues a tcgen05.mma every ~100 cycles at best,
 //              far slower than an M = 128, N <= 128 MMA executes, so NT = 128
 //              blocks split each tile's K-blocks between two issuing warps with
-//              an accumulator each (even K-blocks -> D0, odd -> D1); the
-//              epilogue adds the two.  NT = 256 MMAs are long enough for one.
+//              an accumulator each (K-block kb -> D_{kb mod 2}); the epilogue
+//              adds them.  NT = 256 MMAs are long enough for one.
 template <int NT>
 struct Cfg {
   static constexpr int TOK_STAGE_BYTES = NT * BK * 2;
-  static constexpr int STAGES = NT == 128 ? 6 : 3;
-  static constexpr int W8_STAGES = 12;
   static constexpr int MMA_WARPS = NT == 128 ? 2 : 1;
+  static constexpr uint32_t A_COL0 = MMA_WARPS * NT;      // weight stages follow the accumulators
+  static constexpr int STAGES = NT == 128 ? 6 : 4;
+  static constexpr int W8_STAGES = NT == 128 ? 12 : 8;
   static_assert(STAGES <= MAX_STAGES && W8_STAGES <= MAX_W8_STAGES, "ring sizes");
-  static_assert(MMA_WARPS * NT <= (int)A_COL0, "accumulators fit below the weight stages");
+  static_assert(MMA_WARPS <= MAX_MMA_WARPS, "one drain barrier per MMA issuer");
+  // Every stage must always meet the same MMA issuer and the same decoder set:
+  // mbarrier waits tell phases apart only modulo 2, so a warp may never skip a
+  // use of a stage it waits on.  Ring depths are multiples of the issuer and
+  // set counts, and every tile's K-blocks are padded to whole issuer rounds.
+  static_assert(STAGES % MMA_WARPS == 0 && STAGES % DEC_SETS == 0, "stages pair with warps");
+  static_assert(W8_STAGES % DEC_SETS == 0, "code stages pair with decoder sets");
   static_assert(A_COL0 + STAGES * A_STAGE_COLS <= TMEM_COLS, "weight stages fit in TMEM");
 };
 
@@ -104,7 +119,7 @@ struct SharedState8 {
   uint64_t stage_empty[MAX_STAGES];   // the K-block's MMAs completed (tcgen05.commit)
   uint64_t w8_full[MAX_W8_STAGES], w8_empty[MAX_W8_STAGES];
   uint64_t tmem_full, tmem_empty;
-  uint64_t drain[2];
+  uint64_t drain[MAX_MMA_WARPS];      // one per MMA issuer: its last MMAs completed
   uint32_t tmem_base;
   int abort;
   TileMap tm;
@@ -121,19 +136,20 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
-// 16 accumulator columns of this warp's lane quarter: D0, plus D1 when the
-// tile's K-blocks were split between two accumulators.
-__device__ __forceinline__ void load_acc(uint32_t taddr, uint32_t d1_off, bool two,
+// 16 accumulator columns of this warp's lane quarter: the sum of the tile's
+// `nacc` accumulators (its K-blocks split between the MMA issuers), `stride`
+// columns apart, added in issuer order.
+__device__ __forceinline__ void load_acc(uint32_t taddr, uint32_t stride, int nacc,
                                          uint32_t (&v)[16]) {
   ptx::tmem_ld_x16(taddr, v);
-  if (two) {
+  ptx::tmem_wait_ld();
+  for (int a = 1; a < nacc; ++a) {
     uint32_t u[16];
-    ptx::tmem_ld_x16(taddr + d1_off, u);
+    ptx::tmem_ld_x16(taddr + a * stride, u);
     ptx::tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(u[j]));
-  } else {
-    ptx::tmem_wait_ld();
+    for (int j = 0; j < 16; ++j)
+      v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(u[j]));
   }
 }
 
@@ -142,7 +158,7 @@ __device__ __forceinline__ void load_acc(uint32_t taddr, uint32_t d1_off, bool t
 // block's tokens.  Per 16 tokens the low lanes finish tokens 0-7 and the high
 // lanes tokens 8-15, each taking the missing half from its partner lane.
 __device__ __forceinline__ void store_gateup(const TileInfo& ti, const Problem& P, uint32_t taddr,
-                                             uint32_t d1_off, bool two, int n, int q, int lane) {
+                                             uint32_t stride, int nacc, int n, int q, int lane) {
   const int Nout = ti.shared ? P.N_s : P.N_r;
   const int f = ti.n0 + q * 16 + (lane & 15);
   const bool hi = lane >= 16;
@@ -151,7 +167,7 @@ __device__ __forceinline__ void store_gateup(const TileInfo& ti, const Problem& 
 #pragma unroll 1
   for (int c = 0; c < n; c += 16) {
     uint32_t v[16];
-    load_acc(taddr + c, d1_off, two, v);
+    load_acc(taddr + c, stride, nacc, v);
     const int t0 = ti.m0 + c + (hi ? 8 : 0);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -167,7 +183,7 @@ __device__ __forceinline__ void store_gateup(const TileInfo& ti, const Problem& 
 
 // Down epilogue of one warp: lane i holds output column n0 + 32q + i.
 __device__ __forceinline__ void store_down(const TileInfo& ti, const Problem& P, uint32_t taddr,
-                                           uint32_t d1_off, bool two, int n, int q, int lane) {
+                                           uint32_t stride, int nacc, int n, int q, int lane) {
   const int Nout = ti.shared ? P.N_s : P.N_r;
   const int d = ti.n0 + q * 32 + lane;
   const bool d_ok = d < Nout;
@@ -175,7 +191,7 @@ __device__ __forceinline__ void store_down(const TileInfo& ti, const Problem& P,
 #pragma unroll 1
   for (int c = 0; c < n; c += 16) {
     uint32_t v[16];
-    load_acc(taddr + c, d1_off, two, v);
+    load_acc(taddr + c, stride, nacc, v);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int t = ti.m0 + c + j;
@@ -221,8 +237,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     }
     ptx::mbar_init(&ss.tmem_full, MW);
     ptx::mbar_init(&ss.tmem_empty, EPI_WARPS);
-    ptx::mbar_init(&ss.drain[0], 1);
-    ptx::mbar_init(&ss.drain[1], 1);
+    for (int i = 0; i < MAX_MMA_WARPS; ++i) ptx::mbar_init(&ss.drain[i], 1);
     ss.abort = 0;
     ptx::fence_barrier_init();
   }
@@ -265,13 +280,17 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
         const int nk = tile_k_blocks(ti, P);
         const int nbox = (block_n<NT>(ti.rows - ti.m0) + TOK_BOX - 1) / TOK_BOX;
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < round_up(nk, MW); ++kb) {
           if (!ptx::mbar_wait(&ss.stage_empty[ts], tph ^ 1u, abort)) { ok = false; break; }
-          uint8_t* st = tok_ring + ts * C::TOK_STAGE_BYTES;
-          ptx::mbar_arrive_expect_tx(&ss.tok_full[ts], nbox * TOK_BOX_BYTES);
-          for (int b = 0; b < nbox; ++b)
-            ptx::tma_load_2d(st + b * TOK_BOX_BYTES, amap, &ss.tok_full[ts], kb * BK,
-                             a_row + b * TOK_BOX);
+          if (kb >= nk) {
+            ptx::mbar_arrive(&ss.tok_full[ts]);   // padding stage: no data
+          } else {
+            uint8_t* st = tok_ring + ts * C::TOK_STAGE_BYTES;
+            ptx::mbar_arrive_expect_tx(&ss.tok_full[ts], nbox * TOK_BOX_BYTES);
+            for (int b = 0; b < nbox; ++b)
+              ptx::tma_load_2d(st + b * TOK_BOX_BYTES, amap, &ss.tok_full[ts], kb * BK,
+                               a_row + b * TOK_BOX);
+          }
           issued |= 1u << ts;
           par = (par & ~(1u << ts)) | (tph << ts);
           if (++ts == S) { ts = 0; tph ^= 1u; }
@@ -299,12 +318,17 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
         const int w_row = ti.grp * (ti.shared ? P.b_s_group_rows : P.b_r_group_rows) + ti.n0;
         const int nk = tile_k_blocks(ti, P);
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < round_up(nk, MW); ++kb) {
           if (!ptx::mbar_wait(&ss.w8_empty[ws], wph ^ 1u, abort)) { ok = false; break; }
-          uint8_t* sw = w8_ring + ws * W8_BYTES;
-          ptx::mbar_arrive_expect_tx(&ss.w8_full[ws], W8_BYTES);
-          ptx::tma_load_2d(sw, w0, &ss.w8_full[ws], kb * BK, w_row);
-          if (P.gateup) ptx::tma_load_2d(sw + W8_BYTES / 2, w1, &ss.w8_full[ws], kb * BK, w_row);
+          if (kb >= nk) {
+            ptx::mbar_arrive(&ss.w8_full[ws]);    // padding stage: no data
+          } else {
+            uint8_t* sw = w8_ring + ws * W8_BYTES;
+            ptx::mbar_arrive_expect_tx(&ss.w8_full[ws], W8_BYTES);
+            ptx::tma_load_2d(sw, w0, &ss.w8_full[ws], kb * BK, w_row);
+            if (P.gateup)
+              ptx::tma_load_2d(sw + W8_BYTES / 2, w1, &ss.w8_full[ws], kb * BK, w_row);
+          }
           issued |= 1u << ws;
           par = (par & ~(1u << ws)) | (wph << ws);
           if (++ws == W8S) { ws = 0; wph ^= 1u; }
@@ -314,11 +338,11 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       for (int s = 0; s < W8S; ++s)
         if (issued & (1u << s)) wait_drain(&ss.w8_full[s], (par >> s) & 1u, abort);
     }
-  } else if (warp == MMA_WARP0 || (MW > 1 && warp == MMA_WARP1)) {
+  } else if (mma_index(warp) >= 0 && mma_index(warp) < MW) {
     // ---------------- MMA issuers ----------------
     // Issuer m takes the K-blocks kb with kb % MW == m of every tile into
     // accumulator D_m; all issuers walk the same stage sequence.
-    const int m = warp == MMA_WARP0 ? 0 : 1;
+    const int m = mma_index(warp);
     if (lane == 0) {
       int st = 0;
       uint32_t sph = 0, acc_phase = 0;
@@ -332,7 +356,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
         ptx::tc_fence_after();
         bool ok = true;
         uint32_t accumulate = 0;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < round_up(nk, MW); ++kb) {
           const int cur = st;
           const uint32_t cur_ph = sph;
           if (++st == S) { st = 0; sph ^= 1u; }
@@ -342,14 +366,17 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
             ok = false;
             break;
           }
-          ptx::tc_fence_after();
-          const uint32_t a_tmem = tmem_base + A_COL0 + cur * A_STAGE_COLS;
-          // descriptor start-address field counts 16-byte units: +2 per K step
-          const uint64_t b_desc = ptx::smem_desc_sw128(ptx::smem_addr(tok_ring + cur * C::TOK_STAGE_BYTES));
+          if (kb < nk) {
+            ptx::tc_fence_after();
+            const uint32_t a_tmem = tmem_base + C::A_COL0 + cur * A_STAGE_COLS;
+            // descriptor start-address field counts 16-byte units: +2 per K step
+            const uint64_t b_desc =
+                ptx::smem_desc_sw128(ptx::smem_addr(tok_ring + cur * C::TOK_STAGE_BYTES));
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            ptx::mma_f16_ts(d_tmem, a_tmem + kk * 8, b_desc + 2 * kk, idesc, accumulate);
-            accumulate = 1;
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              ptx::mma_f16_ts(d_tmem, a_tmem + kk * 8, b_desc + 2 * kk, idesc, accumulate);
+              accumulate = 1;
+            }
           }
           ptx::mma_commit(&ss.stage_empty[cur]);   // token and weight stage free
         }
@@ -360,7 +387,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       ptx::mma_commit(&ss.drain[m]);
       wait_drain(&ss.drain[m], 0, abort);
     }
-  } else if (warp >= 2 && warp < DEC_WARP0) {
+  } else if (warp >= 2 && warp < 6) {
     // ---------------- epilogue (warps 2..5) ----------------
     const int q = warp & 3;
     uint32_t acc_phase = 0;
@@ -368,25 +395,25 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
       const Problem& P = p.pr[ti.prob];
       const int n = block_n<NT>(ti.rows - ti.m0);
-      const bool two = MW > 1 && tile_k_blocks(ti, P) > 1;
+      const int nacc = min(MW, tile_k_blocks(ti, P));
       if (!ptx::mbar_wait(&ss.tmem_full, acc_phase, abort)) break;
       ptx::tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      if (P.gateup) store_gateup(ti, P, taddr, NT, two, n, q, lane);
-      else store_down(ti, P, taddr, NT, two, n, q, lane);
+      if (P.gateup) store_gateup(ti, P, taddr, NT, nacc, n, q, lane);
+      else store_down(ti, P, taddr, NT, nacc, n, q, lane);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ss.tmem_empty);
       acc_phase ^= 1u;
       if (p.nprob > 1 && ti.prob == 0) release_rows(p, ti, lane);
     }
-  } else if ((warp >= DEC_WARP0 && warp < DEC_WARP0 + 4) || warp >= DEC_WARP1) {
+  } else if (decoder_set(warp) >= 0) {
     // ---------------- weight decoders (warps 6..9 and 12..15) ----------------
     // Two sets of four warps take alternate stages; each warp decodes the 32
     // weight rows of its TMEM lane quarter.
     const int q = warp & 3;
-    const int set = warp >= DEC_WARP1 ? 1 : 0;
-    const uint32_t t_lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + A_COL0;
+    const int set = decoder_set(warp);
+    const uint32_t t_lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::A_COL0;
     int ws = 0, as = 0, seq = 0;
     uint32_t wph = 0, aph = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -405,12 +432,20 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       const int kbn = ti.shared ? P.kb_s : P.kb_r;
       const int8_t* ex_row = ex + ((size_t)ti.grp * rbn + ti.n0 / fp8::kBlock) * kbn;
       bool ok = true;
-      for (int kb = 0; kb < nk; ++kb) {
+      for (int kb = 0; kb < round_up(nk, MW); ++kb) {
         const int my_ws = ws, my_as = as;
         const uint32_t my_wph = wph, my_aph = aph;
         if (++ws == W8S) { ws = 0; wph ^= 1u; }
         if (++as == S) { as = 0; aph ^= 1u; }
-        if ((seq++ & 1) != set) continue;
+        if (seq++ % DEC_SETS != set) continue;
+        if (kb >= nk) {
+          // padding stage: pass it through both rings with no data
+          if (!ptx::mbar_wait(&ss.w8_full[my_ws], my_wph, abort)) { ok = false; break; }
+          ptx::mbar_arrive(&ss.w8_empty[my_ws]);
+          if (!ptx::mbar_wait(&ss.stage_empty[my_as], my_aph ^ 1u, abort)) { ok = false; break; }
+          ptx::mbar_arrive(&ss.a_full[my_as]);
+          continue;
+        }
         // the exponent load goes out first; the stage wait hides its latency
         const int e = ex_row[(kb * BK) / fp8::kBlock];
         if (!ptx::mbar_wait(&ss.w8_full[my_ws], my_wph, abort)) { ok = false; break; }

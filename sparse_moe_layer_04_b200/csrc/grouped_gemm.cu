@@ -80,6 +80,13 @@ struct Shape {
   static constexpr int BUF_COLS = MMA_WARPS * ACC_COLS;      // one accumulator buffer
   static constexpr uint32_t TMEM_COLS = 2 * BUF_COLS;        // double buffered
   static_assert(TMEM_COLS <= 512, "TMEM columns");
+  static_assert(MMA_WARPS <= 2, "one drain barrier per MMA issuer (SharedState::drain)");
+  // Each stage must always be consumed by the same issuer (stage s by issuer
+  // s % MMA_WARPS): mbarrier waits tell phases apart only modulo 2, so a warp
+  // may never skip a use of a stage it waits on.  With the ring a multiple of
+  // the issuer count and every tile's K-blocks padded to whole rounds, stage
+  // and issuer stay paired.
+  static_assert(STAGES % MMA_WARPS == 0, "stages pair with issuers");
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, MMA_N);
 };
 
@@ -192,19 +199,23 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         tile_k_range(ti, P, &kbeg, &K);
         const int nk = (K + BK - 1) / BK;
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < round_up(nk, MW); ++kb) {
           if (!ptx::mbar_wait(&ss.empty[stage], phase ^ 1u, abort)) { ok = false; break; }
-          uint8_t* sa = ring + stage * STAGE_BYTES;
-          uint8_t* sb = sa + A_BYTES;
-          const int xb = kbeg + kb * BK;
-          const int xa = P.a_k_mod > 0 ? xb % P.a_k_mod : xb;
-          ptx::mbar_arrive_expect_tx(&ss.full[stage], STAGE_BYTES);
-          ptx::tma_load_2d(sa, amap, &ss.full[stage], xa, a_row);
-          if (P.gateup) {
-            ptx::tma_load_2d(sb, b0, &ss.full[stage], xb, b_row);
-            ptx::tma_load_2d(sb + HALF * BK * 2, b1, &ss.full[stage], xb, b_row);
+          if (kb >= nk) {
+            ptx::mbar_arrive(&ss.full[stage]);   // padding stage: no data
           } else {
-            ptx::tma_load_2d(sb, b0, &ss.full[stage], xb, b_row);
+            uint8_t* sa = ring + stage * STAGE_BYTES;
+            uint8_t* sb = sa + A_BYTES;
+            const int xb = kbeg + kb * BK;
+            const int xa = P.a_k_mod > 0 ? xb % P.a_k_mod : xb;
+            ptx::mbar_arrive_expect_tx(&ss.full[stage], STAGE_BYTES);
+            ptx::tma_load_2d(sa, amap, &ss.full[stage], xa, a_row);
+            if (P.gateup) {
+              ptx::tma_load_2d(sb, b0, &ss.full[stage], xb, b_row);
+              ptx::tma_load_2d(sb + HALF * BK * 2, b1, &ss.full[stage], xb, b_row);
+            } else {
+              ptx::tma_load_2d(sb, b0, &ss.full[stage], xb, b_row);
+            }
           }
           issued_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -245,21 +256,23 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         const uint32_t d_tmem = tmem_base + acc * BUF_COLS + m * ACC_COLS;
         bool ok = true;
         uint32_t accumulate = 0;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < round_up(nk, MW); ++kb) {
           const int cur = stage;
           const uint32_t cur_phase = phase;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           if (kb % MW != m) continue;
           if (!ptx::mbar_wait(&ss.full[cur], cur_phase, abort)) { ok = false; break; }
-          ptx::tc_fence_after();
-          const uint32_t sa = ptx::smem_addr(ring + cur * STAGE_BYTES);
-          // descriptor start-address fields count 16-byte units: +2 per K step
-          const uint64_t a_desc = ptx::smem_desc_sw128(sa);
-          const uint64_t b_desc = ptx::smem_desc_sw128(sa + A_BYTES);
+          if (kb < nk) {
+            ptx::tc_fence_after();
+            const uint32_t sa = ptx::smem_addr(ring + cur * STAGE_BYTES);
+            // descriptor start-address fields count 16-byte units: +2 per K step
+            const uint64_t a_desc = ptx::smem_desc_sw128(sa);
+            const uint64_t b_desc = ptx::smem_desc_sw128(sa + A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            ptx::mma_f16_ss(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, IDESC, accumulate);
-            accumulate = 1;
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              ptx::mma_f16_ss(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, IDESC, accumulate);
+              accumulate = 1;
+            }
           }
           ptx::mma_commit(&ss.empty[cur]);     // frees the smem stage when these MMAs finish
         }
