@@ -121,9 +121,12 @@ class CudaOps:
         self._ws = {}
 
     def _workspace(self, d):
-        key = (d.T, d.D, d.E, d.F, d.k, d.S, d.Fs)
+        """One workspace per call shape apart from T, grown when a larger T
+        needs more (the received row count changes from pass to pass)."""
+        key = (d.D, d.E, d.F, d.k, d.S, d.Fs)
+        need = self.moe.moe_workspace_size(d)
         ws = self._ws.get(key)
-        if ws is None:
+        if ws is None or ws.numel() < need:
             ws = self.moe.alloc_workspace(d)
             self._ws[key] = ws
         return ws
