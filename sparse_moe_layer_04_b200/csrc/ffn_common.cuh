@@ -54,6 +54,8 @@ struct GemmParams {
   int* status;
   int* counters;             // [E+S] gate/up tiles stored per group (two problems)
   int* sched;                // tile claim counter, zero at launch; nullptr: static round-robin
+  int weights_once;          // 1: weight tiles are read by about one row tile each, so
+                             // they are loaded with an L2 evict-first policy
   int nprob;                 // 1 or 2
   int E, S, T;
   int rows_r;                // T * k

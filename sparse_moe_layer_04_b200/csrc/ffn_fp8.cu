@@ -307,6 +307,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     // the token producer (which may wait on the gate/up -> down hand-off) as
     // far as the code ring allows.
     if (lane == 0) {
+      const uint64_t w_policy = ptx::l2_policy_evict_first();
       int ws = 0;
       uint32_t wph = 0;
       uint32_t issued = 0, par = 0;
@@ -325,9 +326,18 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
           } else {
             uint8_t* sw = w8_ring + ws * W8_BYTES;
             ptx::mbar_arrive_expect_tx(&ss.w8_full[ws], W8_BYTES);
-            ptx::tma_load_2d(sw, w0, &ss.w8_full[ws], kb * BK, w_row);
-            if (P.gateup)
-              ptx::tma_load_2d(sw + W8_BYTES / 2, w1, &ss.w8_full[ws], kb * BK, w_row);
+            if (p.weights_once) {
+              // codes read once: evict them first, keeping tokens and
+              // activations in L2
+              ptx::tma_load_2d_hint(sw, w0, &ss.w8_full[ws], kb * BK, w_row, w_policy);
+              if (P.gateup)
+                ptx::tma_load_2d_hint(sw + W8_BYTES / 2, w1, &ss.w8_full[ws], kb * BK, w_row,
+                                      w_policy);
+            } else {
+              ptx::tma_load_2d(sw, w0, &ss.w8_full[ws], kb * BK, w_row);
+              if (P.gateup)
+                ptx::tma_load_2d(sw + W8_BYTES / 2, w1, &ss.w8_full[ws], kb * BK, w_row);
+            }
           }
           issued |= 1u << ws;
           par = (par & ~(1u << ws)) | (wph << ws);
@@ -583,6 +593,7 @@ cudaError_t launch_expert_ffn_fp8(const FfnArgs& a, const Fp8Weights& w, cudaStr
   p.nprob = 2;
   p.E = a.E; p.S = a.S; p.T = a.T;
   p.rows_r = rows_r;
+  p.weights_once = small ? 1 : 0;   // one 128-token block per group: codes read once
   const int tiles_g = mt_upper * cdiv(a.F, GU_FEATS) + a.S * mt_s * cdiv(a.Fs, GU_FEATS);
   const int tiles_d = (mt_upper + a.S * mt_s) * cdiv(a.D, W_ROWS);
   cudaError_t err = small ? launch_one8<128>(p, tiles_g + tiles_d, st)
