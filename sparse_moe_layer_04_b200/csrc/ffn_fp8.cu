@@ -24,8 +24,8 @@
 //            (lanes 0-15) and up rows (lanes 16-31) of the same 16 features,
 //            and the epilogue warp pairs them with one lane shuffle;
 //   down     one group x 128 output columns x a token block.
-// Ordering and the gate/up -> down hand-off (per-group counters, bounded
-// acquire waits) are those of the bf16 kernel.
+// Ordering, dynamic tile claiming and the gate/up -> down hand-off (per-group
+// counters, bounded acquire waits) are those of the bf16 kernel.
 //
 // CTA (512 threads, one per SM):
 //   warp 0      token producer: TMA of token tiles (bf16, 128-byte swizzle,
@@ -120,6 +120,8 @@ struct SharedState8 {
   uint64_t w8_full[MAX_W8_STAGES], w8_empty[MAX_W8_STAGES];
   uint64_t tmem_full, tmem_empty;
   uint64_t drain[MAX_MMA_WARPS];      // one per MMA issuer: its last MMAs completed
+  uint64_t tq_full[TILE_Q], tq_empty[TILE_Q];   // claimed tiles, weight producer -> the rest
+  int tq_tile[TILE_Q];
   uint32_t tmem_base;
   int abort;
   TileMap tm;
@@ -238,6 +240,12 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     ptx::mbar_init(&ss.tmem_full, MW);
     ptx::mbar_init(&ss.tmem_empty, EPI_WARPS);
     for (int i = 0; i < MAX_MMA_WARPS; ++i) ptx::mbar_init(&ss.drain[i], 1);
+    // readers of the tile queue: token producer, MMA issuers, 4 epilogue and
+    // 8 decoder warps
+    for (int i = 0; i < TILE_Q; ++i) {
+      ptx::mbar_init(&ss.tq_full[i], 1);
+      ptx::mbar_init(&ss.tq_empty[i], 1 + MW + EPI_WARPS + 4 * DEC_SETS);
+    }
     ss.abort = 0;
     ptx::fence_barrier_init();
   }
@@ -266,7 +274,14 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       int ts = 0;
       uint32_t tph = 0;
       uint32_t issued = 0, par = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int qslot = 0;
+      uint32_t qphase = 0;
+      for (;;) {
+        if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
+        const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
+        ptx::mbar_arrive(&ss.tq_empty[qslot]);
+        if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+        if (tile < 0) break;
         const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
         const Problem& P = p.pr[ti.prob];
         if (ti.prob == 1) {
@@ -305,13 +320,25 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     // ---------------- weight producer ----------------
     // Weights depend on nothing the kernel writes, so this warp runs ahead of
     // the token producer (which may wait on the gate/up -> down hand-off) as
-    // far as the code ring allows.
+    // far as the code ring allows.  It also claims the CTA's tiles (in
+    // increasing order, see claim_tile) and publishes each one to the other
+    // warps through the tile queue before loading it.
     if (lane == 0) {
       const uint64_t w_policy = ptx::l2_policy_evict_first();
       int ws = 0;
       uint32_t wph = 0;
       uint32_t issued = 0, par = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int qslot = 0;
+      uint32_t qphase = 0;
+      int tile = blockIdx.x;
+      int next = tile < total ? claim_tile(p, tile) : total;
+      for (;;) {
+        // hand the tile (or the end mark) to the other roles
+        if (!ptx::mbar_wait(&ss.tq_empty[qslot], qphase ^ 1u, abort)) break;
+        ss.tq_tile[qslot] = tile < total ? tile : -1;
+        ptx::mbar_arrive(&ss.tq_full[qslot]);
+        if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+        if (tile >= total) break;
         const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
         const Problem& P = p.pr[ti.prob];
         const CUtensorMap* w0 = ti.shared ? &P.b0_s : &P.b0_r;
@@ -344,6 +371,8 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
           if (++ws == W8S) { ws = 0; wph ^= 1u; }
         }
         if (!ok) break;
+        tile = next;
+        next = tile < total ? claim_tile(p, tile) : total;
       }
       for (int s = 0; s < W8S; ++s)
         if (issued & (1u << s)) wait_drain(&ss.w8_full[s], (par >> s) & 1u, abort);
@@ -357,7 +386,14 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       int st = 0;
       uint32_t sph = 0, acc_phase = 0;
       const uint32_t d_tmem = tmem_base + m * NT;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int qslot = 0;
+      uint32_t qphase = 0;
+      for (;;) {
+        if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
+        const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
+        ptx::mbar_arrive(&ss.tq_empty[qslot]);
+        if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+        if (tile < 0) break;
         const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
         const Problem& P = p.pr[ti.prob];
         const int nk = tile_k_blocks(ti, P);
@@ -401,7 +437,15 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     // ---------------- epilogue (warps 2..5) ----------------
     const int q = warp & 3;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    int qslot = 0;
+    uint32_t qphase = 0;
+    for (;;) {
+      if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
+      const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&ss.tq_empty[qslot]);
+      if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+      if (tile < 0) break;
       const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
       const Problem& P = p.pr[ti.prob];
       const int n = block_n<NT>(ti.rows - ti.m0);
@@ -426,7 +470,15 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     const uint32_t t_lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::A_COL0;
     int ws = 0, as = 0, seq = 0;
     uint32_t wph = 0, aph = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    int qslot = 0;
+    uint32_t qphase = 0;
+    for (;;) {
+      if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
+      const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&ss.tq_empty[qslot]);
+      if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+      if (tile < 0) break;
       const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
       const Problem& P = p.pr[ti.prob];
       const int nk = tile_k_blocks(ti, P);
@@ -594,6 +646,7 @@ cudaError_t launch_expert_ffn_fp8(const FfnArgs& a, const Fp8Weights& w, cudaStr
   p.E = a.E; p.S = a.S; p.T = a.T;
   p.rows_r = rows_r;
   p.weights_once = small ? 1 : 0;   // one 128-token block per group: codes read once
+  p.sched = a.counters + a.E + a.S; // tile claims, zeroed with the group counters
   const int tiles_g = mt_upper * cdiv(a.F, GU_FEATS) + a.S * mt_s * cdiv(a.Fs, GU_FEATS);
   const int tiles_d = (mt_upper + a.S * mt_s) * cdiv(a.D, W_ROWS);
   cudaError_t err = small ? launch_one8<128>(p, tiles_g + tiles_d, st)
