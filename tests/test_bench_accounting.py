@@ -1,0 +1,64 @@
+"""The benchmark's accounting on the CPU: algorithmic bytes and flops of the
+layer and of the expert-FFN launch (the roofline numerators), FP8 weight
+bytes, whole-job throughput, and the traffic record keyed by kernel sources."""
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import moe_inputs as mi  # noqa: E402
+
+
+def test_expert_weight_bytes():
+    assert bench.expert_weight_bytes(2048, 6144, "bf16") == 2048 * 6144 * 2
+    # codes + one exponent per 128 x 128 block (ragged blocks count whole)
+    assert bench.expert_weight_bytes(2048, 6144, "fp8") == 2048 * 6144 + 16 * 48
+    assert bench.expert_weight_bytes(200, 136, "fp8") == 200 * 136 + 2 * 2
+
+
+def test_decode_ffn_bytes_and_flops():
+    cfg = mi.CONFIGS["decode"]
+    T, D, F, k = cfg.T, cfg.D, cfg.F, cfg.k
+    rows = T * k + T                                   # routed rows + shared rows
+    weights = 11 * 3 * F * D * 2                       # 10 touched + 1 shared expert
+    assert bench.ffn_bytes(cfg, 10) == weights + rows * D * 2 + rows * D * 4 == 872939520
+    assert bench.ffn_bytes(cfg, 10, "fp8") == 457728768
+    assert bench.ffn_flops(cfg) == 6 * D * F * (T * k + T)
+    B, FL = bench.layer_bytes_flops(cfg, 10)
+    assert B == weights + cfg.E * D * 4 + cfg.E * 4 + T * D * 2 + T * D * 4 + T * k * 8
+    assert FL == 2 * T * D * cfg.E + bench.ffn_flops(cfg)
+
+
+def test_throughput_counts_every_rank():
+    assert bench.aggregate_tokens_per_s(128, 1, 0.2) == pytest.approx(128 / 2e-4)
+    assert bench.aggregate_tokens_per_s(128, 8, 0.2) == pytest.approx(8 * 128 / 2e-4)
+    assert bench.max_over_ranks([1.0, 2.0], 1) == [1.0, 2.0]
+
+
+def test_traffic_record_follows_the_kernel_sources(tmp_path, monkeypatch):
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        recs = json.load(f)
+    for key, rec in recs.items():
+        for src in rec["sources"]:
+            assert os.path.exists(os.path.join(ROOT, src)), src
+        assert rec["dram_bytes_per_launch"] > 0
+    assert bench.stored_traffic("no_such_kernel/decode") is None
+    # a record taken on other sources is not reported
+    fake = tmp_path / "profiles"
+    fake.mkdir()
+    rec = dict(recs["expert_ffn/decode"], sources_sha256_16="0" * 16)
+    (fake / "traffic.json").write_text(json.dumps({"expert_ffn/decode": rec}))
+    for src in rec["sources"]:
+        dst = tmp_path / src
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        dst.write_bytes(open(os.path.join(ROOT, src), "rb").read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.stored_traffic("expert_ffn/decode") is None
+    rec["sources_sha256_16"] = bench.source_digest(rec["sources"])
+    (fake / "traffic.json").write_text(json.dumps({"expert_ffn/decode": rec}))
+    assert bench.stored_traffic("expert_ffn/decode") == rec["dram_bytes_per_launch"]
