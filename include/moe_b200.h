@@ -266,6 +266,56 @@ int moe_fp8_dequantize(const void* codes, const int8_t* exps, int G, int R, int 
 int moe_gather_rows(const void* src, int src_rows, const int32_t* idx, int n, int row_bytes,
                     void* dst, void* ws, moe_stream_t stream);
 
+/* ---- Host-buffer pipeline ----------------------------------------------
+ * The layer forward from page-locked host memory to page-locked host memory,
+ * for callers whose hidden states live on the host (the pages' own runtime
+ * stages activations between host and GPU, "GLM-5.2" PocketLLM, Implemented
+ * execution path).  Each submitted step copies h [T, D] bf16 from the host,
+ * runs moe_forward / moe_forward_fp8 on the pipeline's compute stream and
+ * copies out [T, D] fp32 back to the host.  The input copy runs on one copy
+ * stream and the output copy on another, so the copies of step n+1 and n-1
+ * overlap the layer of step n; layers run one after another, in submission
+ * order, on the compute stream.
+ *
+ * Memory: the caller owns every buffer.  `dev` (device memory, 256-byte
+ * aligned, at least moe_pipeline_device_bytes(dims) bytes) holds two input
+ * slots, two output slots and the layer's workspace; it, the weights, Wr
+ * and bias must stay valid until moe_pipeline_destroy returns.  The pipeline
+ * itself creates two CUDA streams and six events on the current device (no
+ * device memory) and frees them in moe_pipeline_destroy.  One pipeline is
+ * driven from one host thread at a time. */
+typedef struct moe_pipeline moe_pipeline_t;
+
+/* Device bytes a pipeline needs for these dims (0 if the dims are invalid). */
+size_t moe_pipeline_device_bytes(const moe_dims_t* dims);
+
+/* Creates a pipeline on the current device.  Weights: bf16 (W1..Ws2 as in
+ * moe_forward, w8 = NULL) or FP8 (w8 as in moe_forward_fp8; W1..Ws2 are then
+ * ignored and may be NULL).  `stream` is the compute stream (it may be the
+ * default stream).  *out receives the handle; on failure *out is NULL and
+ * nothing stays allocated. */
+int moe_pipeline_create(const moe_dims_t* dims, const float* Wr, const float* bias,
+                        const void* W1, const void* W3, const void* W2, const void* Ws1,
+                        const void* Ws3, const void* Ws2, const moe_fp8_weights_t* w8,
+                        void* dev, size_t dev_bytes, moe_stream_t stream, moe_pipeline_t** out);
+
+/* Enqueues one step: h_host [T, D] bf16 -> out_host [T, D] fp32, both
+ * page-locked host memory (cudaHostAlloc / cudaHostRegister; pageable memory
+ * is refused with MOE_ERR_INVALID_ARG, since copies from it cannot overlap;
+ * with T = 0 nothing is enqueued and the pointers are not looked at).
+ * Returns without waiting; h_host must not be modified, and out_host not read,
+ * until moe_pipeline_wait returns. */
+int moe_pipeline_submit(moe_pipeline_t* p, const void* h_host, float* out_host);
+
+/* Blocks until every submitted step's output is in host memory; returns
+ * MOE_OK or the first device-side error of those steps (as
+ * moe_get_device_status). */
+int moe_pipeline_wait(moe_pipeline_t* p);
+
+/* Waits for outstanding steps, then frees the pipeline's streams and events.
+ * NULL is allowed. */
+int moe_pipeline_destroy(moe_pipeline_t* p);
+
 /* Routing statistics of the last moe_forward (or moe_permute) that used
  * `ws` with these dims: device pointers into the workspace, valid once the
  * stream has reached the end of that call and until the next call reuses the

@@ -91,6 +91,12 @@ def _load() -> ctypes.CDLL:
         "moe_forward_fp8": (I, [P, P, P, W8, D, P, P, P, P, Z, P]),
         "moe_fp8_dequantize": (I, [P, P, I, I, I, P, P, P]),
         "moe_gather_rows": (I, [P, I, P, I, I, P, P, P]),
+        "moe_pipeline_device_bytes": (Z, [D]),
+        "moe_pipeline_create": (I, [D, P, P, P, P, P, P, P, P, W8, P, Z, P,
+                                    ctypes.POINTER(ctypes.c_void_p)]),
+        "moe_pipeline_submit": (I, [P, P, P]),
+        "moe_pipeline_wait": (I, [P]),
+        "moe_pipeline_destroy": (I, [P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -276,6 +282,84 @@ def moe_forward(h, Wr, bias, W1, W3, W2, Ws1, Ws3, Ws2, d, out, ws, idx_out=None
                             _ptr(Ws3, bf, "Ws3"), _ptr(Ws2, bf, "Ws2"), ctypes.byref(d),
                             _ptr(out, torch.float32, "out"), _ptr(idx_out, torch.int32, "idx_out"),
                             _ptr(w_out, torch.float32, "w_out"), wp, wn, _stream(stream)))
+
+
+class MoePipeline:
+    """Handle of a host-buffer pipeline (moe_pipeline_t).  It holds the
+    tensors the library reads through raw pointers (weights, router, bias,
+    the device buffer) so they outlive the pipeline."""
+
+    def __init__(self, handle: ctypes.c_void_p, d: moe_dims_t, keep):
+        self.handle = handle
+        self.dims = d
+        self._keep = keep
+
+    def __del__(self):
+        if getattr(self, "handle", None) and self.handle.value:
+            try:
+                _lib.moe_pipeline_destroy(self.handle)
+            except Exception:
+                pass
+            self.handle = None
+
+
+def moe_pipeline_device_bytes(d: moe_dims_t) -> int:
+    n = _lib.moe_pipeline_device_bytes(ctypes.byref(d))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, f"invalid dimensions {d}")
+    return n
+
+
+def moe_pipeline_create(d, Wr, bias, W1=None, W3=None, W2=None, Ws1=None, Ws3=None, Ws2=None,
+                        w8: Optional[moe_fp8_weights_t] = None, dev=None, stream=None,
+                        keep=()) -> MoePipeline:
+    """bf16 weights (W1..Ws2) or FP8 weights (w8, whose tensors the caller
+    passes in `keep` or otherwise keeps alive).  `dev` defaults to a fresh
+    device buffer of moe_pipeline_device_bytes(d) bytes."""
+    if dev is None:
+        dev = torch.empty(moe_pipeline_device_bytes(d), dtype=torch.uint8, device=Wr.device)
+    bf = None if w8 is not None else torch.bfloat16
+    handle = ctypes.c_void_p()
+    _check(_lib.moe_pipeline_create(ctypes.byref(d), _ptr(Wr, torch.float32, "Wr"),
+                                    _ptr(bias, torch.float32, "bias"), _ptr(W1, bf, "W1"),
+                                    _ptr(W3, bf, "W3"), _ptr(W2, bf, "W2"), _ptr(Ws1, bf, "Ws1"),
+                                    _ptr(Ws3, bf, "Ws3"), _ptr(Ws2, bf, "Ws2"),
+                                    ctypes.byref(w8) if w8 is not None else None,
+                                    _ptr(dev, torch.uint8, "dev"), dev.numel(), _stream(stream),
+                                    ctypes.byref(handle)))
+    return MoePipeline(handle, d, (Wr, bias, W1, W3, W2, Ws1, Ws3, Ws2, w8, dev, tuple(keep)))
+
+
+def _host_ptr(t: torch.Tensor, dtype, name: str) -> int:
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.is_cuda or not t.is_pinned():
+        raise ValueError(f"{name}: expected a page-locked (pinned) host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def moe_pipeline_submit(p: MoePipeline, h_host: torch.Tensor, out_host: torch.Tensor) -> None:
+    """Enqueues h_host [T, D] bf16 -> out_host [T, D] fp32 (pinned host tensors)."""
+    n = p.dims.T * p.dims.D
+    if h_host.numel() != n or out_host.numel() != n:
+        raise ValueError("h_host and out_host must hold T x D elements")
+    if n == 0:
+        _check(_lib.moe_pipeline_submit(p.handle, None, None))
+        return
+    _check(_lib.moe_pipeline_submit(p.handle, _host_ptr(h_host, torch.bfloat16, "h_host"),
+                                    _host_ptr(out_host, torch.float32, "out_host")))
+
+
+def moe_pipeline_wait(p: MoePipeline) -> None:
+    _check(_lib.moe_pipeline_wait(p.handle))
+
+
+def moe_pipeline_destroy(p: MoePipeline) -> None:
+    handle, p.handle = p.handle, None
+    if handle is not None and handle.value:
+        _check(_lib.moe_pipeline_destroy(handle))
 
 
 def moe_get_device_status(ws, stream=None) -> int:

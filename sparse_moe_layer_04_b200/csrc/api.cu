@@ -2,6 +2,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <new>
 #include <string>
 
 #include "moe_internal.cuh"
@@ -359,6 +360,40 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
   return MOE_OK;
 }
 
+// Device memory of a host-buffer pipeline: two input slots, two output slots
+// and the layer's workspace, each 256-byte aligned.
+struct PipeLayout {
+  size_t h[2], out[2], ws, ws_bytes, total;
+};
+
+bool pipe_layout(const moe_dims_t& d, PipeLayout* L) {
+  WsLayout W;
+  if (!ws_layout(d, &W)) return false;
+  const size_t hb = align256((size_t)d.T * d.D * 2), ob = align256((size_t)d.T * d.D * 4);
+  size_t off = 0;
+  for (int s = 0; s < 2; ++s) { L->h[s] = off; off += hb; }
+  for (int s = 0; s < 2; ++s) { L->out[s] = off; off += ob; }
+  L->ws = off;
+  L->ws_bytes = W.total;
+  L->total = off + align256(W.total);
+  return true;
+}
+
+// Host pointers the pipeline copies from or to must be page-locked: a copy
+// from pageable memory is staged by the driver and cannot overlap the layer.
+int check_pinned(const void* p, const char* name) {
+  if (!p) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MOE_ERR_INVALID_ARG, "%s: %s", name, cudaGetErrorString(e));
+  }
+  if (a.type != cudaMemoryTypeHost)
+    return fail(MOE_ERR_INVALID_ARG, "%s is not page-locked host memory", name);
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -701,6 +736,181 @@ int moe_get_device_status(void* ws, moe_stream_t stream) {
     return fail(MOE_ERR_BOUNDS, "device: expert index, group offset or row index out of range");
   if (word & kStTimeout) return fail(MOE_ERR_TIMEOUT, "device: a bounded wait gave up");
   return MOE_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Host-buffer pipeline
+// ---------------------------------------------------------------------------
+// Step n uses slot n % 2.  Before its input copy overwrites input slot s, the
+// copy stream waits for step n-2's layer (which read that slot); before its
+// layer overwrites output slot s, the compute stream waits for step n-2's
+// output copy.  Events never recorded count as complete, so the first two
+// steps wait on nothing.
+struct moe_pipeline {
+  moe_dims_t dims{};
+  moe::ExpertWeights wt{};
+  const float* Wr = nullptr;
+  const float* bias = nullptr;
+  void* h_dev[2] = {nullptr, nullptr};
+  float* out_dev[2] = {nullptr, nullptr};
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  cudaStream_t compute = nullptr, copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t in_done[2] = {nullptr, nullptr};
+  cudaEvent_t layer_done[2] = {nullptr, nullptr};
+  cudaEvent_t out_done[2] = {nullptr, nullptr};
+  long long steps = 0;
+  int device = 0;
+};
+
+namespace {
+
+// Waits for the pipeline's outstanding work and frees its streams and
+// events; returns the first CUDA error met.
+cudaError_t pipeline_release(moe_pipeline* p) {
+  cudaError_t first = cudaSuccess;
+  auto keep = [&first](cudaError_t e) {
+    if (first == cudaSuccess && e != cudaSuccess) first = e;
+  };
+  if (p->copy_in) keep(cudaStreamSynchronize(p->copy_in));
+  for (int s = 0; s < 2; ++s)
+    if (p->layer_done[s]) keep(cudaEventSynchronize(p->layer_done[s]));
+  if (p->copy_out) keep(cudaStreamSynchronize(p->copy_out));
+  for (int s = 0; s < 2; ++s) {
+    if (p->in_done[s]) keep(cudaEventDestroy(p->in_done[s]));
+    if (p->layer_done[s]) keep(cudaEventDestroy(p->layer_done[s]));
+    if (p->out_done[s]) keep(cudaEventDestroy(p->out_done[s]));
+  }
+  if (p->copy_in) keep(cudaStreamDestroy(p->copy_in));
+  if (p->copy_out) keep(cudaStreamDestroy(p->copy_out));
+  delete p;
+  return first;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_pipeline_device_bytes(const moe_dims_t* dims) {
+  if (check_dims(dims) != MOE_OK) return 0;
+  PipeLayout L;
+  if (!pipe_layout(*dims, &L)) return 0;
+  return L.total;
+}
+
+int moe_pipeline_create(const moe_dims_t* dims, const float* Wr, const float* bias,
+                        const void* W1, const void* W3, const void* W2, const void* Ws1,
+                        const void* Ws3, const void* Ws2, const moe_fp8_weights_t* w8,
+                        void* dev, size_t dev_bytes, moe_stream_t stream, moe_pipeline_t** out) {
+  if (out) *out = nullptr;
+  int rc = begin(dims);
+  if (rc) return rc;
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+  MOE_CHECK_PTR(Wr);
+  MOE_CHECK_PTR(bias);
+  ExpertWeights wt;
+  if (w8) {
+    if ((rc = check_fp8_dims(dims))) return rc;
+    if ((rc = check_fp8_weights(w8, dims, &wt))) return rc;
+  } else if ((rc = check_bf16_weights(W1, W3, W2, Ws1, Ws3, Ws2, dims, &wt))) {
+    return rc;
+  }
+  PipeLayout L;
+  if (!pipe_layout(*dims, &L)) return fail(MOE_ERR_INVALID_ARG, "pipeline layout overflow");
+  if (!dev) return fail(MOE_ERR_WORKSPACE, "dev is NULL");
+  if (reinterpret_cast<uintptr_t>(dev) & 255u)
+    return fail(MOE_ERR_WORKSPACE, "dev is not 256-byte aligned");
+  if (dev_bytes < L.total)
+    return fail(MOE_ERR_WORKSPACE, "dev has %zu bytes, needs %zu", dev_bytes, L.total);
+  if ((rc = check_device())) return rc;
+
+  moe_pipeline* p = new (std::nothrow) moe_pipeline();
+  if (!p) return fail(MOE_ERR_UNSUPPORTED, "out of host memory");
+  p->dims = *dims;
+  p->wt = wt;
+  p->Wr = Wr;
+  p->bias = bias;
+  uint8_t* base = static_cast<uint8_t*>(dev);
+  for (int s = 0; s < 2; ++s) {
+    p->h_dev[s] = base + L.h[s];
+    p->out_dev[s] = reinterpret_cast<float*>(base + L.out[s]);
+  }
+  p->ws = base + L.ws;
+  p->ws_bytes = L.ws_bytes;
+  p->compute = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->copy_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->copy_out, cudaStreamNonBlocking);
+  for (int s = 0; s < 2 && e == cudaSuccess; ++s) {
+    e = cudaEventCreateWithFlags(&p->in_done[s], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->layer_done[s], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->out_done[s], cudaEventDisableTiming);
+  }
+  // the workspace starts zeroed (status word and counters)
+  if (e == cudaSuccess) e = cudaMemsetAsync(p->ws, 0, p->ws_bytes, p->compute);
+  if (e != cudaSuccess) {
+    pipeline_release(p);
+    return cuda_fail(e, "pipeline create");
+  }
+  *out = p;
+  return MOE_OK;
+}
+
+int moe_pipeline_submit(moe_pipeline_t* p, const void* h_host, float* out_host) {
+  g_err.clear();
+  g_launches = 0;
+  if (!p) return fail(MOE_ERR_INVALID_ARG, "pipeline is NULL");
+  if (p->dims.T == 0) return MOE_OK;  // nothing to copy or compute
+  int rc;
+  if ((rc = check_pinned(h_host, "h_host"))) return rc;
+  if ((rc = check_pinned(out_host, "out_host"))) return rc;
+  int cur = 0;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (cur != p->device)
+    return fail(MOE_ERR_INVALID_ARG, "current device %d is not the pipeline's device %d", cur,
+                p->device);
+  const int s = static_cast<int>(p->steps & 1);
+  const size_t hb = (size_t)p->dims.T * p->dims.D * 2, ob = (size_t)p->dims.T * p->dims.D * 4;
+  e = cudaStreamWaitEvent(p->copy_in, p->layer_done[s], 0);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(p->h_dev[s], h_host, hb, cudaMemcpyHostToDevice, p->copy_in);
+  if (e == cudaSuccess) e = cudaEventRecord(p->in_done[s], p->copy_in);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(p->compute, p->in_done[s], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(p->compute, p->out_done[s], 0);
+  if (e != cudaSuccess) return cuda_fail(e, "pipeline input copy");
+  rc = forward_impl(p->h_dev[s], p->Wr, p->bias, p->wt, &p->dims, p->out_dev[s], nullptr, nullptr,
+                    p->ws, p->ws_bytes, reinterpret_cast<moe_stream_t>(p->compute));
+  if (rc) return rc;
+  const int n = g_launches;
+  e = cudaEventRecord(p->layer_done[s], p->compute);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(p->copy_out, p->layer_done[s], 0);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(out_host, p->out_dev[s], ob, cudaMemcpyDeviceToHost, p->copy_out);
+  if (e == cudaSuccess) e = cudaEventRecord(p->out_done[s], p->copy_out);
+  if (e != cudaSuccess) return cuda_fail(e, "pipeline output copy");
+  ++p->steps;
+  g_launches = n;
+  return MOE_OK;
+}
+
+int moe_pipeline_wait(moe_pipeline_t* p) {
+  g_err.clear();
+  if (!p) return fail(MOE_ERR_INVALID_ARG, "pipeline is NULL");
+  cudaError_t e = cudaStreamSynchronize(p->copy_in);
+  for (int s = 0; s < 2 && e == cudaSuccess; ++s) e = cudaEventSynchronize(p->layer_done[s]);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(p->copy_out);
+  if (e != cudaSuccess) return cuda_fail(e, "pipeline wait");
+  return moe_get_device_status(p->ws, reinterpret_cast<moe_stream_t>(p->compute));
+}
+
+int moe_pipeline_destroy(moe_pipeline_t* p) {
+  g_err.clear();
+  if (!p) return MOE_OK;
+  const cudaError_t e = pipeline_release(p);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "pipeline destroy");
 }
 
 }  // extern "C"

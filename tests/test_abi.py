@@ -186,3 +186,66 @@ def test_gather_rows_argument_checks(mod):
     assert lib.moe_gather_rows(FAKE, 10, None, 4, 32, FAKE, None, None) == mod.MOE_ERR_INVALID_ARG
     assert lib.moe_gather_rows(FAKE, 10, FAKE, 4, 32, FAKE, FAKE + 16, None) == mod.MOE_ERR_WORKSPACE
     assert lib.moe_gather_rows(None, 0, None, 0, 32, None, None, None) == mod.MOE_OK
+
+
+def test_pipeline_argument_checks(mod):
+    lib = mod._lib
+    d = mod.dims(T=8, D=128, E=8, F=64, k=2)
+
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    need = mod.moe_pipeline_device_bytes(d)
+    assert need == 2 * a256(8 * 128 * 2) + 2 * a256(8 * 128 * 4) + a256(mod.moe_workspace_size(d))
+    assert lib.moe_pipeline_device_bytes(ctypes.byref(mod.dims(T=4, D=12, E=8, F=64, k=2))) == 0
+    h = ctypes.c_void_p(FAKE)
+    P = ctypes.c_void_p
+
+    def create(dd, Wr=FAKE, W1=FAKE, w8=None, dev=FAKE, n=None, out=True):
+        handle = ctypes.c_void_p(FAKE)
+        rc = lib.moe_pipeline_create(ctypes.byref(dd), Wr, FAKE, W1, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                     w8, dev, need if n is None else n, None,
+                                     ctypes.byref(handle) if out else None)
+        if out:
+            assert handle.value is None   # cleared on failure
+        return rc, mod.moe_last_error()
+
+    rc, msg = create(d, out=False)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "out is NULL" in msg
+    rc, msg = create(d, Wr=None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "Wr" in msg
+    rc, msg = create(d, W1=None)
+    assert rc == mod.MOE_ERR_INVALID_ARG and "W1" in msg
+    rc, msg = create(d, dev=None)
+    assert rc == mod.MOE_ERR_WORKSPACE and "dev is NULL" in msg
+    rc, msg = create(d, dev=FAKE + 16)
+    assert rc == mod.MOE_ERR_WORKSPACE and "256-byte" in msg
+    rc, msg = create(d, n=need - 1)
+    assert rc == mod.MOE_ERR_WORKSPACE and "needs" in msg
+    rc, msg = create(mod.dims(T=8, D=128, E=8, F=64, k=9))
+    assert rc == mod.MOE_ERR_INVALID_ARG
+    # FP8 weights: the bf16 pointers are ignored, the FP8 rules apply
+    w8 = mod.moe_fp8_weights_t()
+    rc, msg = create(d, w8=ctypes.byref(w8))          # bf16 W1 given, w8->W1 NULL
+    assert rc == mod.MOE_ERR_INVALID_ARG and "W1 is NULL" in msg
+    d24 = mod.dims(T=8, D=136, E=8, F=64, k=2)
+    rc, msg = create(d24, W1=None, w8=ctypes.byref(w8))
+    assert rc == mod.MOE_ERR_INVALID_ARG and "multiple of 16" in msg
+
+    assert lib.moe_pipeline_submit(None, h, h) == mod.MOE_ERR_INVALID_ARG
+    assert "pipeline is NULL" in mod.moe_last_error()
+    assert lib.moe_pipeline_wait(None) == mod.MOE_ERR_INVALID_ARG
+    assert lib.moe_pipeline_destroy(None) == mod.MOE_OK
+
+
+def test_pipeline_binding_checks_host_tensors(mod):
+    import torch
+    d = mod.dims(T=2, D=16, E=8, F=16, k=2)
+    p = mod.MoePipeline(ctypes.c_void_p(None), d, ())
+    with pytest.raises(ValueError, match="T x D"):
+        mod.moe_pipeline_submit(p, torch.zeros(3, 16, dtype=torch.bfloat16),
+                                torch.zeros(2, 16, dtype=torch.float32))
+    with pytest.raises((ValueError, RuntimeError)):
+        # pageable (or, without a GPU, unpinnable) host memory is refused
+        mod.moe_pipeline_submit(p, torch.zeros(2, 16, dtype=torch.bfloat16),
+                                torch.zeros(2, 16, dtype=torch.float32))
