@@ -157,6 +157,7 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
     return at;
   };
   L->status = take(256);
+  L->ticket = take(256);
   L->partials = take((size_t)sp.nsplit * T * E * 4);
   L->wr3 = take(sp.tensor ? E * 3 * D * 2 : 0);
   L->idx = take(T * k * 4);
@@ -334,14 +335,26 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
   if (e == cudaSuccess) e = launch_router(hb, Wr, *dims, sp, w, partials, st, &n, &rwhy);
   if (e == cudaSuccess) e = mark(1, st);
   if (e != cudaSuccess) return cuda_fail(e, rwhy);
-  e = launch_route(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw, w.status(), st);
-  if (e == cudaSuccess) e = mark(2, st);
-  if (e != cudaSuccess) return cuda_fail(e, "route launch");
-  n += 1;
-  e = launch_permute(idx, T, E, k, counts, offsets, perm, inv, w.at<int32_t>(w.L.blk_base),
-                     w.status(), w.at<int32_t>(w.L.touched), st, &n);
-  if (e == cudaSuccess) e = mark(3, st);
-  if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  if (T <= kPermBlockTokens) {
+    // small batches: the routing kernel's last block also groups the pairs
+    const RouteGrouping grp{counts, offsets, perm, inv, w.at<int32_t>(w.L.touched),
+                            w.at<int>(w.L.ticket)};
+    e = launch_route_and_group(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw,
+                               w.status(), grp, st);
+    if (e == cudaSuccess) e = mark(2, st);
+    if (e == cudaSuccess) e = mark(3, st);
+    if (e != cudaSuccess) return cuda_fail(e, "route launch");
+    n += 1;
+  } else {
+    e = launch_route(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw, w.status(), st);
+    if (e == cudaSuccess) e = mark(2, st);
+    if (e != cudaSuccess) return cuda_fail(e, "route launch");
+    n += 1;
+    e = launch_permute(idx, T, E, k, counts, offsets, perm, inv, w.at<int32_t>(w.L.blk_base),
+                       w.status(), w.at<int32_t>(w.L.touched), st, &n);
+    if (e == cudaSuccess) e = mark(3, st);
+    if (e != cudaSuccess) return cuda_fail(e, "permute launch");
+  }
   uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
   int32_t* counters = w.at<int32_t>(w.L.counters);
   e = launch_gather_rows(hb, perm, T * k, D, T, xperm, counters, E + dims->S + 1, st);

@@ -46,7 +46,7 @@ cudaError_t noalloc_scratch(int32_t** out);
 
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
 struct WsLayout {
-  size_t status, partials, wr3, idx, w, counts, offsets, perm, inv, blk_base, counters, xperm,
+  size_t status, ticket, partials, wr3, idx, w, counts, offsets, perm, inv, blk_base, counters, xperm,
       act_r, act_s, y, touched, total;
 };
 bool ws_layout(const moe_dims_t& d, WsLayout* out);
@@ -82,6 +82,21 @@ cudaError_t launch_reduce_partials(const float* partials, int nsplit, size_t n, 
                                    cudaStream_t st);
 cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T, int E, int k,
                          float scale, int32_t* idx, float* w, int* status, cudaStream_t st);
+// Outputs of the grouping done by the routing kernel's last block (as
+// launch_permute's); `ticket` is an int that is zero before the launch and
+// is left zero after it.
+struct RouteGrouping {
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv;
+  int32_t* touched;
+  int* ticket;  // nullptr: no grouping
+};
+// Routing and grouping in one launch; T <= kPermBlockTokens.
+cudaError_t launch_route_and_group(const float* src, int nsplit, const float* bias, int T, int E,
+                                   int k, float scale, int32_t* idx, float* w, int* status,
+                                   const RouteGrouping& grp, cudaStream_t st);
 // `touched` (nullable): number of experts with at least one pair.
 cudaError_t launch_route_grouped(const float* logits, const float* bias, int T, int E, int k,
                                  float scale, int n_group, int topk_group, int32_t* idx, float* w,

@@ -14,11 +14,12 @@
 // Batches of at most 256 tokens (one counting block) run all three phases in
 // one launch.  All integer work: exact and deterministic.
 #include "moe_internal.cuh"
+#include "permute_block.cuh"
 #include "sm100_ptx.cuh"
 
 namespace moe {
 
-constexpr int kWordsPerBlock = kPermBlockTokens / 32;
+constexpr int kWordsPerBlock = kPermWords;
 
 __global__ void __launch_bounds__(kPermBlockTokens) permute_count_kernel(
     const int32_t* __restrict__ idx, int T, int E, int k, int32_t* __restrict__ blk_counts,
@@ -143,77 +144,7 @@ __global__ void __launch_bounds__(kPermBlockTokens) permute_single_block_kernel(
   ptx::pdl_launch_dependents();
   ptx::pdl_wait();
   extern __shared__ int sm[];
-  int* cnt = sm;                                          // [E]
-  unsigned* mask = reinterpret_cast<unsigned*>(sm + E);   // [E][kWordsPerBlock]
-  __shared__ int warp_tot[kPermBlockTokens / 32];
-  for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[i] = 0;
-  for (int i = threadIdx.x; i < E * kWordsPerBlock; i += blockDim.x) mask[i] = 0u;
-  __syncthreads();
-  const int t = threadIdx.x;
-  const int word = t >> 5;
-  const unsigned bit = 1u << (t & 31);
-  bool bad = false;
-  if (t < T) {
-    for (int j = 0; j < k; ++j) {
-      const int e = idx[(size_t)t * k + j];
-      if (e < 0 || e >= E) {
-        bad = true;
-        continue;
-      }
-      atomicAdd(&cnt[e], 1);
-      const unsigned old = atomicOr(&mask[e * kWordsPerBlock + word], bit);
-      if (old & bit) bad = true;
-    }
-  }
-  __syncthreads();
-  // exclusive scan of cnt over experts: thread i owns experts [i*per, (i+1)*per)
-  const int per = (E + kPermBlockTokens - 1) / kPermBlockTokens;
-  const int e0 = threadIdx.x * per;
-  int local = 0;
-  for (int e = e0; e < e0 + per && e < E; ++e) local += cnt[e];
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int incl = local;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += v;
-  }
-  if (lane == 31) warp_tot[wid] = incl;
-  __syncthreads();
-  int base = incl - local;
-  for (int q = 0; q < wid; ++q) base += warp_tot[q];
-  __syncthreads();  // everyone has read warp_tot; cnt becomes the offsets
-  int nz = 0;
-  for (int e = e0; e < e0 + per && e < E; ++e) {
-    const int c = cnt[e];
-    counts[e] = c;
-    offsets[e] = base;
-    cnt[e] = base;
-    base += c;
-    nz += c > 0;
-  }
-  if (threadIdx.x == kPermBlockTokens - 1) offsets[E] = base;  // the last thread ends at the total
-  if (touched) {  // block sum of the per-thread counts of experts with pairs
-    __shared__ int nz_total;
-    if (threadIdx.x == 0) nz_total = 0;
-    __syncthreads();
-    if (nz) atomicAdd(&nz_total, nz);
-    __syncthreads();
-    if (threadIdx.x == 0) *touched = nz_total;
-  }
-  __syncthreads();
-  if (t < T && !bad) {
-    for (int j = 0; j < k; ++j) {
-      const int e = idx[(size_t)t * k + j];
-      const unsigned* m = mask + e * kWordsPerBlock;
-      int rank = __popc(m[word] & (bit - 1u));
-      for (int q = 0; q < word; ++q) rank += __popc(m[q]);
-      const int row = cnt[e] + rank;
-      perm[row] = t;
-      inv[(size_t)t * k + j] = row;
-    }
-  }
-  if (bad && status) atomicOr(status, kStBounds);
+  permute_block(idx, T, E, k, counts, offsets, perm, inv, status, touched, sm);
 }
 
 // ---------------------------------------------------------------------------
@@ -249,7 +180,7 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
                            int* status, int32_t* touched, cudaStream_t st, int* nlaunch) {
   const int nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
   if (nblk == 1) {
-    const size_t smem = (size_t)E * sizeof(int) + (size_t)E * kWordsPerBlock * sizeof(unsigned);
+    const size_t smem = permute_block_smem(E);
     *nlaunch += 1;
     return launch_pdl(permute_single_block_kernel, dim3(1), dim3(kPermBlockTokens), smem, st, idx,
                       T, E, k, counts, offsets, perm, inv, status, touched);

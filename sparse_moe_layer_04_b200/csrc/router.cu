@@ -17,6 +17,7 @@
 #include <climits>
 
 #include "moe_internal.cuh"
+#include "permute_block.cuh"
 #include "sm100_ptx.cuh"
 
 namespace moe {
@@ -211,30 +212,30 @@ cudaError_t launch_reduce_partials(const float* partials, int nsplit, size_t n, 
 // ---------------------------------------------------------------------------
 // routing: one block per token, one thread per expert
 // ---------------------------------------------------------------------------
-// (key, expert) pair a precedes b under (key descending, index ascending).
-__device__ __forceinline__ bool precedes(float ka, int ea, float kb, int eb) {
-  return ka > kb || (ka == kb && ea < eb);
+// Selection order: key descending, then expert index ascending.  A key is
+// mapped to an unsigned integer that orders the same way (-0 as +0; NaN, and
+// "no candidate", as 0, below every key), so one warp-wide max reduction
+// finds the best key and one min reduction over the lanes holding it the
+// lowest expert index.
+__device__ __forceinline__ uint32_t key_order(float key) {
+  uint32_t u = __float_as_uint(key);
+  if (key != key) return 0u;
+  if (u == 0x80000000u) u = 0u;  // -0 ranks as +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Arg-max of (key, index) pairs across a warp; every lane gets the winner.
-__device__ __forceinline__ void warp_best(float& bk, int& be, float& bs) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-    const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-    if (precedes(ok, oe, bk, be)) {
-      bk = ok;
-      be = oe;
-      bs = os;
-    }
-  }
+// Best (order, expert) pair of the warp; every lane gets the winner.
+__device__ __forceinline__ void warp_best(uint32_t& bu, int& be) {
+  const uint32_t m = __reduce_max_sync(0xffffffffu, bu);
+  const uint32_t e = __reduce_min_sync(0xffffffffu, bu == m ? (uint32_t)be : 0xffffffffu);
+  bu = m;
+  be = (int)e;
 }
 
 constexpr int kMaxSlots = 32;
 
 // Top-k of one token held one expert per thread (key, score, index; threads
-// past E hold -inf / INT_MAX), in the block's shared candidate arrays: each
+// past E hold index INT_MAX), in the block's shared candidate arrays: each
 // warp extracts its k best (key, index) pairs by warp arg-max rounds; the
 // union of the warps' lists holds the token's top k, which warp 0 extracts
 // the same way, in selection order, and writes with the renormalised weights
@@ -242,21 +243,20 @@ constexpr int kMaxSlots = 32;
 // Must be called by every thread of the block.
 __device__ __forceinline__ void block_topk_write(float key, float sc, int me, int t, int k,
                                                  float scale, int32_t* __restrict__ idx,
-                                                 float* __restrict__ w, float* c_key,
-                                                 float* c_sc, int* c_e) {
+                                                 float* __restrict__ w, uint32_t* c_u, int* c_e,
+                                                 float* s_sc) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  bool taken = false;
+  uint32_t u = me != INT_MAX ? key_order(key) : 0u;
+  if (me != INT_MAX) s_sc[me] = sc;
   for (int j = 0; j < k; ++j) {
-    float bk = taken ? -INFINITY : key;
-    int be = taken ? INT_MAX : me;
-    float bs = sc;
-    warp_best(bk, be, bs);
+    uint32_t bu = u;
+    int be = me;
+    warp_best(bu, be);
     if (lane == 0) {
-      c_key[wid * k + j] = bk;
-      c_e[wid * k + j] = be;
-      c_sc[wid * k + j] = bs;
+      c_u[wid * k + j] = bu;
+      c_e[wid * k + j] = bu ? be : INT_MAX;
     }
-    if (be == me) taken = true;
+    if (be == me) u = 0u;
   }
   __syncthreads();
   if (wid != 0) return;
@@ -265,20 +265,22 @@ __device__ __forceinline__ void block_topk_write(float key, float sc, int me, in
   int my_e = 0;
   float my_s = 0.f, sum = 0.f;
   for (int j = 0; j < k; ++j) {
-    float bk = -INFINITY, bs = 0.f;
+    uint32_t bu = 0u;
     int be = INT_MAX, bq = -1;
     for (int q = 0, c = lane; c < nc; ++q, c += 32) {
       if ((done >> q) & 1u) continue;
-      if (c_e[c] != INT_MAX && precedes(c_key[c], c_e[c], bk, be)) {
-        bk = c_key[c];
-        be = c_e[c];
-        bs = c_sc[c];
+      const uint32_t cu = c_u[c];
+      const int ce = c_e[c];
+      if (ce != INT_MAX && (cu > bu || (cu == bu && ce < be))) {
+        bu = cu;
+        be = ce;
         bq = q;
       }
     }
     const int mine = be;
-    warp_best(bk, be, bs);
+    warp_best(bu, be);
     if (bq >= 0 && mine == be) done |= 1u << bq;
+    const float bs = be != INT_MAX ? s_sc[be] : 0.f;
     if (lane == j) {
       my_e = be;
       my_s = bs;
@@ -313,15 +315,19 @@ __device__ __forceinline__ bool score_and_key(const float* __restrict__ src, int
 }
 
 // Routing with one block per token, one thread per expert.
+//
+// With grp.ticket set (T <= kPermBlockTokens), the kernel also groups the
+// pairs by expert (permute_block) in whichever block finishes last, which
+// saves the grouping kernel's launch on small batches.
 __global__ void __launch_bounds__(1024) route_kernel(
     const float* __restrict__ src, int nsplit, const float* __restrict__ bias, int T, int E,
     int k, float scale, int32_t* __restrict__ idx, float* __restrict__ w,
-    int* __restrict__ status) {
+    int* __restrict__ status, RouteGrouping grp) {
   ptx::pdl_launch_dependents();
   ptx::pdl_wait();
-  __shared__ float c_key[kMaxSlots * kMaxSlots];
-  __shared__ float c_sc[kMaxSlots * kMaxSlots];
+  __shared__ uint32_t c_u[kMaxSlots * kMaxSlots];
   __shared__ int c_e[kMaxSlots * kMaxSlots];
+  __shared__ float s_sc[1024];
   const int t = blockIdx.x;
   const int e = threadIdx.x;
   float key = -INFINITY, sc = 0.f;
@@ -331,7 +337,21 @@ __global__ void __launch_bounds__(1024) route_kernel(
     me = e;
   }
   if (__syncthreads_or(bad) && e == 0 && status) atomicOr(status, kStNonFinite);
-  block_topk_write(key, sc, me, t, k, scale, idx, w, c_key, c_sc, c_e);
+  block_topk_write(key, sc, me, t, k, scale, idx, w, c_u, c_e, s_sc);
+  if (!grp.ticket) return;
+  // The last block to finish groups every token's pairs by expert: each
+  // block's indices are visible GPU-wide before it takes its ticket.
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(grp.ticket, 1) == T - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  extern __shared__ int grp_smem[];
+  permute_block(idx, T, E, k, grp.counts, grp.offsets, grp.perm, grp.inv, status, grp.touched,
+                grp_smem);
+  if (threadIdx.x == 0) *grp.ticket = 0;  // ready for the next call
 }
 
 // Group-limited routing: experts form n_group contiguous groups of E/n_group;
@@ -344,9 +364,9 @@ __global__ void __launch_bounds__(1024) route_grouped_kernel(
     int* __restrict__ status) {
   ptx::pdl_launch_dependents();
   ptx::pdl_wait();
-  __shared__ float c_key[kMaxSlots * kMaxSlots];
-  __shared__ float c_sc[kMaxSlots * kMaxSlots];
+  __shared__ uint32_t c_u[kMaxSlots * kMaxSlots];
   __shared__ int c_e[kMaxSlots * kMaxSlots];
+  __shared__ float s_sc[1024];
   __shared__ float s_key[1024];
   __shared__ float g_score[32];
   __shared__ int g_keep[32];
@@ -380,17 +400,16 @@ __global__ void __launch_bounds__(1024) route_grouped_kernel(
   if (e < 32) {
     bool taken = false;
     for (int j = 0; j < topk_group; ++j) {
-      float bk = (lane < n_group && !taken) ? g_score[lane] : -INFINITY;
+      uint32_t bu = (lane < n_group && !taken) ? key_order(g_score[lane]) : 0u;
       int be = (lane < n_group && !taken) ? lane : INT_MAX;
-      float unused = 0.f;
-      warp_best(bk, be, unused);
-      if (be == lane) taken = true;
+      warp_best(bu, be);
+      if (bu && be == lane) taken = true;
     }
     if (lane < n_group) g_keep[lane] = taken ? 1 : 0;
   }
   __syncthreads();
   if (e < E && !g_keep[e / G]) key = -INFINITY;
-  block_topk_write(key, sc, me, t, k, scale, idx, w, c_key, c_sc, c_e);
+  block_topk_write(key, sc, me, t, k, scale, idx, w, c_u, c_e, s_sc);
 }
 
 // Large batches: one warp per token (four tokens per block), each lane
@@ -434,23 +453,33 @@ __global__ void __launch_bounds__(128) route_warp_kernel(
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0 && status) atomicOr(status, kStNonFinite);
 
-  unsigned taken = 0u;  // bit i: expert lane + 32 i already selected
+  uint32_t ord[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) ord[i] = (lane + 32 * i < E) ? key_order(key[i]) : 0u;
   int my_e = 0;
   float my_s = 0.f, sum = 0.f;
   for (int j = 0; j < k; ++j) {
-    float bk = -INFINITY, bs = 0.f;
+    uint32_t bu = 0u;
     int be = INT_MAX;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !(taken & (1u << i)) && precedes(key[i], e, bk, be)) {
-        bk = key[i];
-        be = e;
-        bs = sc[i];
+      // increasing i visits increasing experts: ties keep the lower index
+      if (ord[i] > bu) {
+        bu = ord[i];
+        be = lane + 32 * i;
       }
     }
-    warp_best(bk, be, bs);
-    if (be != INT_MAX && (be & 31) == lane) taken |= 1u << (be >> 5);
+    warp_best(bu, be);
+    // the owner lane takes the winner out and broadcasts its score
+    float os = 0.f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+      if (be == lane + 32 * i) {
+        os = sc[i];
+        ord[i] = 0u;
+      }
+    const float bs = bu ? __shfl_sync(0xffffffffu, os, be & 31) : 0.f;
+    if (!bu) be = INT_MAX;
     if (lane == j) {
       my_e = be;
       my_s = bs;
@@ -487,7 +516,7 @@ cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T,
   if (T <= kRouteBlockPerTokenMaxT) {
     const int threads = (E + 31) / 32 * 32;
     return launch_pdl(route_kernel, dim3(T), dim3(threads), 0, st, src, nsplit, bias, T, E, k,
-                      scale, idx, w, status);
+                      scale, idx, w, status, RouteGrouping{});
   }
   const int epl = (E + 31) / 32;
   if (epl <= 1) return launch_route_warp<1>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
@@ -496,6 +525,25 @@ cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T,
   if (epl <= 8) return launch_route_warp<8>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
   if (epl <= 16) return launch_route_warp<16>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
   return launch_route_warp<32>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
+}
+
+cudaError_t launch_route_and_group(const float* src, int nsplit, const float* bias, int T, int E,
+                                   int k, float scale, int32_t* idx, float* w, int* status,
+                                   const RouteGrouping& grp, cudaStream_t st) {
+  if (T > kPermBlockTokens || !grp.ticket) return cudaErrorInvalidValue;
+  static int configured_dev = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (configured_dev != dev) {
+    e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)permute_block_smem(1024));
+    if (e != cudaSuccess) return e;
+    configured_dev = dev;
+  }
+  const int threads = (E + 31) / 32 * 32;
+  return launch_pdl(route_kernel, dim3(T), dim3(threads), permute_block_smem(E), st, src, nsplit,
+                    bias, T, E, k, scale, idx, w, status, grp);
 }
 
 }  // namespace moe

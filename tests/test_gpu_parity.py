@@ -301,7 +301,7 @@ def test_forward_tiny_pure_fp32_oracle(moe):
     assert rel_l2(got[same], ref[same]) <= 2e-2
 
 
-@pytest.mark.parametrize("T", [0, 1, 2, 127, 129, 300])
+@pytest.mark.parametrize("T", [0, 1, 2, 127, 129, 256, 257, 300])
 def test_forward_ragged_and_empty(moe, T):
     cfg = mi.custom_config("tiny", T=max(T, 1), name="tiny")
     inp = layer_on_device(cfg)
