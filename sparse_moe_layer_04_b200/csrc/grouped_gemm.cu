@@ -21,8 +21,8 @@
 // CTAs running at the same time share each weight tile through L2), then the
 // shared experts.  CTA c takes tile c first and then claims further tiles in
 // increasing order from a counter in the workspace (zeroed by the row-gather
-// kernel), so CTAs that finish early take more tiles; the producer passes each
-// claimed tile to the MMA and epilogue warps through a small shared-memory
+// kernel), so CTAs that finish early take more tiles; the weight producer passes
+// each claimed tile to the other roles through a small shared-memory
 // queue (the router GEMM, which has no such counter, takes c, c + gridDim.x,
 // ...).  A down tile of an
 // expert waits until every gate/up tile of that expert has been stored: each
@@ -39,10 +39,17 @@
 // finer to keep all 148 SMs busy.  The same kernel also computes the router
 // logits as a dense split-K GEMM (one problem, one shared group per K chunk).
 //
-// CTA structure (224 threads, one CTA per SM):
-//   warp 0      TMA producer: ring of (A 128x64, B Nx64) bf16 tiles (4 stages
-//               for N = 256, 6 for N = 128), 128-byte swizzled, completion
-//               counted on "full" mbarriers.
+// CTA structure (256 threads, one CTA per SM):
+//   warp 7      weight producer and tile claimer: claims the tiles, hands them
+//               to the other roles, and streams the weight tiles (N x 64 bf16,
+//               128-byte swizzled) into a ring of their own by TMA: 8 stages
+//               for N = 128, 4 for N = 256.  It never waits for the gate/up ->
+//               down hand-off, so weight loads run ahead of the activations.
+//   warp 0      token / activation producer: TMA of the A tiles (128 x 64
+//               bf16) into a 4-stage ring (they come from L2); waits for the
+//               hand-off before a down tile.  A token stage is free again when
+//               the MMAs of the K-block four back have completed, which the
+//               producer reads off that K-block's weight-stage barrier.
 //   warp 1      TMEM allocator (512 columns) and MMA issuer:
 //               tcgen05.mma.cta_group::1.kind::f16, M = 128, N, K = 16,
 //               fp32 accumulators in TMEM, two accumulator buffers so the
@@ -62,16 +69,20 @@ namespace {
 
 using namespace ffn;
 
-constexpr int THREADS = 224;             // warps 0-5 and the second MMA issuer (warp 6)
-constexpr int MMA_WARP1 = 6;
-constexpr int RING_BYTES = 192 * 1024;    // operand ring budget
-constexpr int MAX_STAGES = 6;
+constexpr int THREADS = 256;             // warps 0-7
+constexpr int MMA_WARP1 = 6;             // second MMA issuer (N = 128)
+constexpr int BPROD_WARP = 7;            // weight producer and tile claimer
+constexpr int RING_BYTES = 192 * 1024;   // budget of the two operand rings
+constexpr int A_STAGES = 4;              // token / activation ring (its tiles come from L2)
+constexpr int MAX_B_STAGES = 8;
 
 template <int MMA_N>
 struct Shape {
   static constexpr int B_BYTES = MMA_N * BK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = RING_BYTES / STAGE_BYTES;    // 4 (N=256) or 6 (N=128)
+  // The weight ring takes what the token ring leaves: 8 stages for N = 128,
+  // 4 for N = 256.  The weights stream from HBM, so the bytes a CTA keeps in
+  // flight on them set the rate at which a decode batch reads its experts.
+  static constexpr int B_STAGES = (RING_BYTES - A_STAGES * A_BYTES) / B_BYTES;
   static constexpr int ACC_COLS = MMA_N;                     // fp32 TMEM columns per accumulator
   // One thread issues a tcgen05.mma every ~100 cycles at best, longer than an
   // N = 128 MMA executes: N = 128 tiles split their K-blocks between two
@@ -81,18 +92,26 @@ struct Shape {
   static constexpr uint32_t TMEM_COLS = 2 * BUF_COLS;        // double buffered
   static_assert(TMEM_COLS <= 512, "TMEM columns");
   static_assert(MMA_WARPS <= 2, "one drain barrier per MMA issuer (SharedState::drain)");
+  static_assert(B_STAGES <= MAX_B_STAGES, "weight ring barriers");
+  // The token producer reuses a token stage once the MMAs of the K-block
+  // A_STAGES earlier have completed, which it learns from that K-block's
+  // weight-stage "empty" barrier; with B_STAGES >= A_STAGES that barrier cannot
+  // have moved on by a further phase before the producer looks.
+  static_assert(B_STAGES >= A_STAGES, "token stages are released through the weight ring");
   // Each stage must always be consumed by the same issuer (stage s by issuer
   // s % MMA_WARPS): mbarrier waits tell phases apart only modulo 2, so a warp
-  // may never skip a use of a stage it waits on.  With the ring a multiple of
+  // may never skip a use of a stage it waits on.  With both rings multiples of
   // the issuer count and every tile's K-blocks padded to whole rounds, stage
   // and issuer stay paired.
-  static_assert(STAGES % MMA_WARPS == 0, "stages pair with issuers");
+  static_assert(A_STAGES % MMA_WARPS == 0 && B_STAGES % MMA_WARPS == 0,
+                "stages pair with issuers");
   static constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, MMA_N);
 };
 
 struct SharedState {
-  uint64_t full[MAX_STAGES];
-  uint64_t empty[MAX_STAGES];
+  uint64_t a_full[A_STAGES];       // token tile landed (TMA transaction bytes)
+  uint64_t b_full[MAX_B_STAGES];   // weight tile landed
+  uint64_t b_empty[MAX_B_STAGES];  // the K-block's MMAs completed (tcgen05.commit)
   uint64_t tq_full[TILE_Q], tq_empty[TILE_Q];
   int tq_tile[TILE_Q];
   uint64_t tmem_full[2];
@@ -106,8 +125,8 @@ struct SharedState {
 template <int MMA_N>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   using Sh = Shape<MMA_N>;
-  constexpr int STAGES = Sh::STAGES;
-  constexpr int STAGE_BYTES = Sh::STAGE_BYTES;
+  constexpr int B_STAGES = Sh::B_STAGES;
+  constexpr int B_BYTES = Sh::B_BYTES;
   constexpr int ACC_COLS = Sh::ACC_COLS;
   constexpr uint32_t TMEM_COLS = Sh::TMEM_COLS;
   constexpr uint32_t IDESC = Sh::IDESC;
@@ -115,10 +134,12 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   constexpr int BUF_COLS = Sh::BUF_COLS;
   constexpr int HALF = MMA_N / 2;  // gate/up: W1 rows [0, HALF), W3 rows [HALF, MMA_N)
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned operand ring (128-byte swizzle atoms span 1024 bytes)
+  // 1024-byte aligned operand rings (128-byte swizzle atoms span 1024 bytes):
+  // the token ring, then the weight ring
   const uint32_t raw_addr = ptx::smem_addr(smem_raw);
-  uint8_t* ring = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  SharedState& ss = *reinterpret_cast<SharedState*>(ring + STAGES * STAGE_BYTES);
+  uint8_t* ring_a = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* ring_b = ring_a + A_STAGES * A_BYTES;
+  SharedState& ss = *reinterpret_cast<SharedState*>(ring_b + B_STAGES * B_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -129,9 +150,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     ptx::tmem_relinquish();
   }
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      ptx::mbar_init(&ss.full[i], 1);
-      ptx::mbar_init(&ss.empty[i], 1);
+    for (int i = 0; i < A_STAGES; ++i) ptx::mbar_init(&ss.a_full[i], 1);
+    for (int i = 0; i < B_STAGES; ++i) {
+      ptx::mbar_init(&ss.b_full[i], 1);
+      ptx::mbar_init(&ss.b_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&ss.tmem_full[i], MW);
@@ -141,13 +163,15 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     ptx::mbar_init(&ss.drain[1], 1);
     for (int i = 0; i < TILE_Q; ++i) {
       ptx::mbar_init(&ss.tq_full[i], 1);
-      ptx::mbar_init(&ss.tq_empty[i], MW + EPI_WARPS);
+      // the token producer, the MMA issuers and the epilogue warps take each tile
+      ptx::mbar_init(&ss.tq_empty[i], 1 + MW + EPI_WARPS);
     }
     ss.abort = 0;
     ptx::fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     ptx::tma_prefetch_desc(&p.pr[0].a_r);
+  } else if (warp == BPROD_WARP && lane == 0) {
     ptx::tma_prefetch_desc(&p.pr[0].b0_r);
     ptx::tma_prefetch_desc(&p.pr[0].b1_r);
   }
@@ -165,8 +189,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   const int total = tiles0 + (p.nprob > 1 ? problem_tiles(p.pr[1], ss.tm, p) : 0);
   volatile int* abort = &ss.abort;
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
+  if (warp == BPROD_WARP) {
+    // ---------------- weight producer and tile claimer ----------------
     if (lane == 0) {
       const uint64_t w_policy = ptx::l2_policy_evict_first();
       int stage = 0;
@@ -177,12 +201,72 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       int tile = blockIdx.x;
       int next = tile < total ? claim_tile(p, tile) : total;
       for (;;) {
-        // hand the tile (or the end mark) to the MMA and epilogue warps
+        // hand the tile (or the end mark) to the other roles
         if (!ptx::mbar_wait(&ss.tq_empty[qslot], qphase ^ 1u, abort)) break;
         ss.tq_tile[qslot] = tile < total ? tile : -1;
         ptx::mbar_arrive(&ss.tq_full[qslot]);
         if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
         if (tile >= total) break;
+        const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
+        const Problem& P = p.pr[ti.prob];
+        const CUtensorMap* b0 = ti.shared ? &P.b0_s : &P.b0_r;
+        const CUtensorMap* b1 = ti.shared ? &P.b1_s : &P.b1_r;
+        const int b_row = ti.grp * (ti.shared ? P.b_s_group_rows : P.b_r_group_rows) + ti.n0;
+        int kbeg, K;
+        tile_k_range(ti, P, &kbeg, &K);
+        const int nk = (K + BK - 1) / BK;
+        bool ok = true;
+        for (int kb = 0; kb < round_up(nk, MW); ++kb) {
+          if (!ptx::mbar_wait(&ss.b_empty[stage], phase ^ 1u, abort)) { ok = false; break; }
+          if (kb >= nk) {
+            ptx::mbar_arrive(&ss.b_full[stage]);   // padding stage: no data
+          } else {
+            uint8_t* sb = ring_b + stage * B_BYTES;
+            const int xb = kbeg + kb * BK;
+            ptx::mbar_arrive_expect_tx(&ss.b_full[stage], B_BYTES);
+            if (p.weights_once) {
+              // weight tiles read once: evict them first, keeping the activations
+              // and expert outputs in L2 for the down tiles and the merge
+              ptx::tma_load_2d_hint(sb, b0, &ss.b_full[stage], xb, b_row, w_policy);
+              if (P.gateup)
+                ptx::tma_load_2d_hint(sb + HALF * BK * 2, b1, &ss.b_full[stage], xb, b_row,
+                                      w_policy);
+            } else {
+              ptx::tma_load_2d(sb, b0, &ss.b_full[stage], xb, b_row);
+              if (P.gateup)
+                ptx::tma_load_2d(sb + HALF * BK * 2, b1, &ss.b_full[stage], xb, b_row);
+            }
+          }
+          issued_mask |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == B_STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tile = next;
+        next = tile < total ? claim_tile(p, tile) : total;
+      }
+      // every issued load has landed before the CTA may retire
+      for (int s = 0; s < B_STAGES; ++s)
+        if (issued_mask & (1u << s)) wait_drain(&ss.b_full[s], (last_parity >> s) & 1u, abort);
+    }
+  } else if (warp == 0) {
+    // ---------------- token / activation producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, last_parity = 0;
+      // position, in the weight ring, of the K-block A_STAGES behind this one
+      int rstage = 0;
+      uint32_t rphase = 0;
+      int lag = A_STAGES;  // K-blocks still to go before that position exists
+      int qslot = 0;
+      uint32_t qphase = 0;
+      for (;;) {
+        if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
+        const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
+        ptx::mbar_arrive(&ss.tq_empty[qslot]);
+        if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+        if (tile < 0) break;
         const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
         const Problem& P = p.pr[ti.prob];
         if (ti.prob == 1) {
@@ -192,48 +276,36 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           ptx::fence_proxy_async_global();
         }
         const CUtensorMap* amap = ti.shared ? &P.a_s : &P.a_r;
-        const CUtensorMap* b0 = ti.shared ? &P.b0_s : &P.b0_r;
-        const CUtensorMap* b1 = ti.shared ? &P.b1_s : &P.b1_r;
         const int a_row = ti.shared ? ti.grp * P.a_s_group_stride + ti.m0 : ti.row0 + ti.m0;
-        const int b_row = ti.grp * (ti.shared ? P.b_s_group_rows : P.b_r_group_rows) + ti.n0;
         int kbeg, K;
         tile_k_range(ti, P, &kbeg, &K);
         const int nk = (K + BK - 1) / BK;
         bool ok = true;
         for (int kb = 0; kb < round_up(nk, MW); ++kb) {
-          if (!ptx::mbar_wait(&ss.empty[stage], phase ^ 1u, abort)) { ok = false; break; }
-          if (kb >= nk) {
-            ptx::mbar_arrive(&ss.full[stage]);   // padding stage: no data
+          // the stage's previous K-block (A_STAGES back) has finished its MMAs
+          if (lag > 0) {
+            --lag;
           } else {
-            uint8_t* sa = ring + stage * STAGE_BYTES;
-            uint8_t* sb = sa + A_BYTES;
+            if (!ptx::mbar_wait(&ss.b_empty[rstage], rphase, abort)) { ok = false; break; }
+            if (++rstage == B_STAGES) { rstage = 0; rphase ^= 1u; }
+          }
+          if (kb >= nk) {
+            ptx::mbar_arrive(&ss.a_full[stage]);   // padding stage: no data
+          } else {
+            uint8_t* sa = ring_a + stage * A_BYTES;
             const int xb = kbeg + kb * BK;
             const int xa = P.a_k_mod > 0 ? xb % P.a_k_mod : xb;
-            ptx::mbar_arrive_expect_tx(&ss.full[stage], STAGE_BYTES);
-            ptx::tma_load_2d(sa, amap, &ss.full[stage], xa, a_row);
-            if (p.weights_once) {
-              // weight tiles read once: evict them first, keeping the activations
-              // and expert outputs in L2 for the down tiles and the merge
-              ptx::tma_load_2d_hint(sb, b0, &ss.full[stage], xb, b_row, w_policy);
-              if (P.gateup)
-                ptx::tma_load_2d_hint(sb + HALF * BK * 2, b1, &ss.full[stage], xb, b_row,
-                                      w_policy);
-            } else {
-              ptx::tma_load_2d(sb, b0, &ss.full[stage], xb, b_row);
-              if (P.gateup) ptx::tma_load_2d(sb + HALF * BK * 2, b1, &ss.full[stage], xb, b_row);
-            }
+            ptx::mbar_arrive_expect_tx(&ss.a_full[stage], A_BYTES);
+            ptx::tma_load_2d(sa, amap, &ss.a_full[stage], xa, a_row);
           }
           issued_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == A_STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tile = next;
-        next = tile < total ? claim_tile(p, tile) : total;
       }
-      // every issued load has landed before the CTA may retire
-      for (int s = 0; s < STAGES; ++s)
-        if (issued_mask & (1u << s)) wait_drain(&ss.full[s], (last_parity >> s) & 1u, abort);
+      for (int s = 0; s < A_STAGES; ++s)
+        if (issued_mask & (1u << s)) wait_drain(&ss.a_full[s], (last_parity >> s) & 1u, abort);
     }
   } else if (warp == 1 || (MW > 1 && warp == MMA_WARP1)) {
     // ---------------- MMA issuers ----------------
@@ -241,8 +313,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     // accumulator m of the tile's buffer; all issuers walk the same stages.
     const int m = warp == 1 ? 0 : 1;
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      int astage = 0, bstage = 0;
+      uint32_t aphase = 0, bphase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       int qslot = 0;
@@ -263,24 +335,30 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         bool ok = true;
         uint32_t accumulate = 0;
         for (int kb = 0; kb < round_up(nk, MW); ++kb) {
-          const int cur = stage;
-          const uint32_t cur_phase = phase;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          const int ca = astage, cb = bstage;
+          const uint32_t pa = aphase, pb = bphase;
+          if (++astage == A_STAGES) { astage = 0; aphase ^= 1u; }
+          if (++bstage == B_STAGES) { bstage = 0; bphase ^= 1u; }
           if (kb % MW != m) continue;
-          if (!ptx::mbar_wait(&ss.full[cur], cur_phase, abort)) { ok = false; break; }
+          if (!ptx::mbar_wait(&ss.a_full[ca], pa, abort) ||
+              !ptx::mbar_wait(&ss.b_full[cb], pb, abort)) {
+            ok = false;
+            break;
+          }
           if (kb < nk) {
             ptx::tc_fence_after();
-            const uint32_t sa = ptx::smem_addr(ring + cur * STAGE_BYTES);
             // descriptor start-address fields count 16-byte units: +2 per K step
-            const uint64_t a_desc = ptx::smem_desc_sw128(sa);
-            const uint64_t b_desc = ptx::smem_desc_sw128(sa + A_BYTES);
+            const uint64_t a_desc = ptx::smem_desc_sw128(ptx::smem_addr(ring_a + ca * A_BYTES));
+            const uint64_t b_desc = ptx::smem_desc_sw128(ptx::smem_addr(ring_b + cb * B_BYTES));
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
               ptx::mma_f16_ss(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, IDESC, accumulate);
               accumulate = 1;
             }
           }
-          ptx::mma_commit(&ss.empty[cur]);     // frees the smem stage when these MMAs finish
+          // frees the weight stage, and the token stage to the producer's next
+          // lap, when these MMAs finish
+          ptx::mma_commit(&ss.b_empty[cb]);
         }
         if (!ok) break;
         ptx::mma_commit(&ss.tmem_full[acc]);   // accumulator ready for the epilogue
@@ -338,7 +416,8 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 template <int MMA_N>
 constexpr size_t smem_bytes() {
-  return 1024 + Shape<MMA_N>::STAGES * Shape<MMA_N>::STAGE_BYTES + sizeof(SharedState);
+  return 1024 + A_STAGES * A_BYTES + Shape<MMA_N>::B_STAGES * Shape<MMA_N>::B_BYTES +
+         sizeof(SharedState);
 }
 static_assert(smem_bytes<256>() <= 227 * 1024 && smem_bytes<128>() <= 227 * 1024,
               "shared memory budget");
