@@ -187,8 +187,10 @@ int moe_combine(const float* y, const float* w, const int32_t* inv, const moe_di
                 float* out, void* ws, moe_stream_t stream);
 
 /* The whole layer: moe_router_logits, moe_route, moe_permute, the row
- * gather, moe_expert_ffn and moe_combine in one call on one stream, with no
- * host synchronisation (capturable in a CUDA graph).
+ * gather, moe_expert_ffn and moe_combine in one call on `stream`, with no
+ * host synchronisation (capturable in a CUDA graph).  For small batches the
+ * shared experts' FFN runs on an internal stream forked from and joined back
+ * into `stream` (moe_forward_shared_overlap says when).
  * h [T, D] bf16; Wr [E, D] fp32; bias [E] fp32; weights as in
  * moe_expert_ffn; out [T, D] fp32.  idx_out [T, k] int32 and w_out [T, k]
  * fp32 are optional (NULL: kept in the workspace).  ws_bytes must be at
@@ -197,6 +199,22 @@ int moe_forward(const void* h, const float* Wr, const float* bias, const void* W
                 const void* W3, const void* W2, const void* Ws1, const void* Ws3,
                 const void* Ws2, const moe_dims_t* dims, float* out, int32_t* idx_out,
                 float* w_out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* 1 if moe_forward (bf16 weights, fp8_weights = 0) or moe_forward_fp8
+ * (fp8_weights = 1) runs the shared experts' FFN for these dims on an
+ * internal stream, next to the routing: the shared experts need no routing,
+ * so their weights stream on 32 SMs while the routing kernels run, and the
+ * routed experts' FFN launch that follows on `stream` no longer carries them.
+ * That is done for bf16 weights when S > 0, T <= 512 and the shared experts'
+ * weights are at least 16 MiB (smaller ones cost less than the fork and join
+ * save; the FP8 kernel is bound by per-SM MMA issue and decoding, so 32 SMs
+ * would finish its shared experts after the routing).  The internal stream
+ * and its two events are created on the first such call of each host thread
+ * and device and kept for the life of the process; the call still returns
+ * without host synchronisation and stays capturable in a CUDA graph (the
+ * internal stream forks from and joins back into `stream`).  0 otherwise, or
+ * for invalid dims. */
+int moe_forward_shared_overlap(const moe_dims_t* dims, int fp8_weights);
 
 /* ---- FP8 expert weights ------------------------------------------------
  * The "Inside GLM" course outline names BF16 and FP8 GLM-5.2 artifacts (its

@@ -91,6 +91,7 @@ def _load() -> ctypes.CDLL:
         "moe_forward_fp8": (I, [P, P, P, W8, D, P, P, P, P, Z, P]),
         "moe_fp8_dequantize": (I, [P, P, I, I, I, P, P, P]),
         "moe_gather_rows": (I, [P, I, P, I, I, P, P, P]),
+        "moe_forward_shared_overlap": (I, [D, I]),
         "moe_pipeline_device_bytes": (Z, [D]),
         "moe_pipeline_create": (I, [D, P, P, P, P, P, P, P, P, W8, P, Z, P,
                                     ctypes.POINTER(ctypes.c_void_p)]),
@@ -360,6 +361,13 @@ def moe_pipeline_destroy(p: MoePipeline) -> None:
     handle, p.handle = p.handle, None
     if handle is not None and handle.value:
         _check(_lib.moe_pipeline_destroy(handle))
+
+
+def moe_forward_shared_overlap(d: moe_dims_t, fp8_weights: bool = False) -> bool:
+    """True if moe_forward (or, with fp8_weights, moe_forward_fp8) runs the
+    shared experts' FFN beside the routing on an internal stream for these
+    dims (then the routed FFN launch excludes them)."""
+    return bool(_lib.moe_forward_shared_overlap(ctypes.byref(d), 1 if fp8_weights else 0))
 
 
 def moe_get_device_status(ws, stream=None) -> int:

@@ -168,6 +168,7 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
   L->inv = take(T * k * 4);
   L->blk_base = take(nblk * E * 4);
   L->counters = take((E + S + 1) * 4);   // per-group counters + the tile claim counter
+  L->counters_s = take((S + 1) * 4);     // the same for a shared-experts-only launch
   L->xperm = take(T * k * D * 2);
   L->act_r = take(T * k * F * 2);
   L->act_s = take(S * T * Fs * 2);
@@ -306,6 +307,47 @@ int expert_ffn_impl(const void* h, const int32_t* perm, const int32_t* offsets,
   return MOE_OK;
 }
 
+// An internal stream (per host thread and device) that runs the shared
+// experts' FFN next to the routing, with the events that fork it from and join
+// it to the caller's stream.  Created on first use, kept for the process.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+cudaError_t side_stream(SideStream** out) {
+  thread_local SideStream per_dev[kMaxDev];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  SideStream& r = per_dev[dev];
+  if (!r.s) {
+    e = cudaStreamCreateWithFlags(&r.s, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      if (r.fork) cudaEventDestroy(r.fork);
+      if (r.s) cudaStreamDestroy(r.s);
+      r = SideStream{};
+      return e;
+    }
+  }
+  *out = &r;
+  return cudaSuccess;
+}
+
+// Makes `st` wait for the side stream's join event when a forward returns
+// early after forking, so that later work on `st` is ordered after the shared
+// experts' kernels that read and write the workspace.
+struct JoinGuard {
+  cudaStream_t st = nullptr;
+  cudaEvent_t join = nullptr;
+  ~JoinGuard() {
+    if (join) cudaStreamWaitEvent(st, join, 0);
+  }
+};
+
 int forward_impl(const void* h, const float* Wr, const float* bias, const ExpertWeights& wt,
                  const moe_dims_t* dims, float* out, int32_t* idx_out, float* w_out, void* ws,
                  size_t ws_bytes, moe_stream_t stream) {
@@ -330,8 +372,40 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
 
   const RouterSplit sp = router_split(T, D, E);
   float* partials = w.at<float>(w.L.partials);
-  const char* rwhy = "router launch";
+  uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
+  int32_t* counters = w.at<int32_t>(w.L.counters);
   cudaError_t e = mark(0, st);
+  if (e != cudaSuccess) return cuda_fail(e, "profile event");
+
+  // Small batches: the shared experts need no routing, so their FFN runs on a
+  // side stream on a few SMs while the routing kernels run here; the merge
+  // waits for it.  Their weights then no longer lengthen the routed FFN.
+  const bool overlap_shared = moe_forward_shared_overlap(dims, wt.fp8 ? 1 : 0) != 0;
+  SideStream* side = nullptr;
+  JoinGuard guard;
+  if (overlap_shared) {
+    e = side_stream(&side);
+    if (e == cudaSuccess) e = cudaEventRecord(side->fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
+    int32_t* counters_s = w.at<int32_t>(w.L.counters_s);
+    if (e == cudaSuccess)
+      e = cudaMemsetAsync(counters_s, 0, (size_t)(dims->S + 1) * sizeof(int32_t), side->s);
+    if (e != cudaSuccess) return cuda_fail(e, "shared-expert stream");
+    FfnArgs as = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
+    as.part = kFfnShared;
+    as.counters_s = counters_s;
+    as.max_ctas = kSharedCtas;
+    const char* swhy = "launch failed";
+    e = launch_ffn(as, wt, side->s, &n, &swhy, nullptr);
+    if (e != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "shared expert ffn: %s (%s)", swhy, cudaGetErrorString(e));
+    e = cudaEventRecord(side->join, side->s);
+    if (e != cudaSuccess) return cuda_fail(e, "shared-expert stream");
+    guard.st = st;
+    guard.join = side->join;
+  }
+
+  const char* rwhy = "router launch";
   if (e == cudaSuccess) e = launch_router(hb, Wr, *dims, sp, w, partials, st, &n, &rwhy);
   if (e == cudaSuccess) e = mark(1, st);
   if (e != cudaSuccess) return cuda_fail(e, rwhy);
@@ -355,16 +429,20 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
     if (e == cudaSuccess) e = mark(3, st);
     if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   }
-  uint16_t* xperm = w.at<uint16_t>(w.L.xperm);
-  int32_t* counters = w.at<int32_t>(w.L.counters);
   e = launch_gather_rows(hb, perm, T * k, D, T, xperm, counters, E + dims->S + 1, st);
   if (e == cudaSuccess) e = mark(4, st);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   n += 1;
-  const FfnArgs a = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
+  FfnArgs a = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
+  if (overlap_shared) a.part = kFfnRouted;
   const char* why = "launch failed";
   e = launch_ffn(a, wt, st, &n, &why, g_prof_events ? g_prof_events + 5 : nullptr);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
+  if (overlap_shared) {
+    guard.join = nullptr;
+    e = cudaStreamWaitEvent(st, side->join, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "shared-expert stream");
+  }
   e = launch_combine(y, rw, inv, T, D, k, dims->S, out, w.status(), st);
   if (e == cudaSuccess) e = mark(6, st);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
@@ -424,6 +502,15 @@ size_t moe_workspace_size(const moe_dims_t* dims) {
 const char* moe_last_error(void) { return g_err.c_str(); }
 
 int moe_last_launch_count(void) { return g_launches; }
+
+int moe_forward_shared_overlap(const moe_dims_t* dims, int fp8_weights) {
+  if (check_dims(dims) != MOE_OK || fp8_weights) return 0;
+  const double shared_bytes = 3.0 * dims->S * (double)dims->Fs * dims->D * 2;
+  return dims->S > 0 && dims->T > 0 && dims->T <= kOverlapSharedMaxT &&
+                 shared_bytes >= kOverlapSharedMinBytes
+             ? 1
+             : 0;
+}
 
 int moe_set_profile_events(void* const* events, int n) {
   g_err.clear();

@@ -561,7 +561,7 @@ static_assert(smem_bytes8<256>() <= 227 * 1024 && smem_bytes8<128>() <= 227 * 10
 static_assert(smem_bytes8<128>() > 114 * 1024, "one CTA per SM");
 
 template <int NT>
-cudaError_t launch_one8(const GemmParams& p, int tiles_upper, cudaStream_t st) {
+cudaError_t launch_one8(const GemmParams& p, int tiles_upper, cudaStream_t st, int max_ctas) {
   static int configured_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -573,6 +573,7 @@ cudaError_t launch_one8(const GemmParams& p, int tiles_upper, cudaStream_t st) {
     configured_dev = dev;
   }
   int grid = num_sms();
+  if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
   if (tiles_upper < grid) grid = tiles_upper;
   if (grid < 1) grid = 1;
   return launch_pdl(ffn_fp8_kernel<NT>, dim3(grid), dim3(THREADS), smem_bytes8<NT>(), st, p);
@@ -647,10 +648,20 @@ cudaError_t launch_expert_ffn_fp8(const FfnArgs& a, const Fp8Weights& w, cudaStr
   p.rows_r = rows_r;
   p.weights_once = small ? 1 : 0;   // one 128-token block per group: codes read once
   p.sched = a.counters + a.E + a.S; // tile claims, zeroed with the group counters
-  const int tiles_g = mt_upper * cdiv(a.F, GU_FEATS) + a.S * mt_s * cdiv(a.Fs, GU_FEATS);
-  const int tiles_d = (mt_upper + a.S * mt_s) * cdiv(a.D, W_ROWS);
-  cudaError_t err = small ? launch_one8<128>(p, tiles_g + tiles_d, st)
-                          : launch_one8<256>(p, tiles_g + tiles_d, st);
+  // one part of the groups, as in the bf16 launcher
+  int mt_r = mt_upper, S = a.S;
+  if (a.part == kFfnRouted) {
+    p.S = S = 0;
+  } else if (a.part == kFfnShared) {
+    p.E = 0;
+    mt_r = 0;
+    p.counters = a.counters_s;
+    p.sched = a.counters_s + a.S;
+  }
+  const int tiles_g = mt_r * cdiv(a.F, GU_FEATS) + S * mt_s * cdiv(a.Fs, GU_FEATS);
+  const int tiles_d = (mt_r + S * mt_s) * cdiv(a.D, W_ROWS);
+  cudaError_t err = small ? launch_one8<128>(p, tiles_g + tiles_d, st, a.max_ctas)
+                          : launch_one8<256>(p, tiles_g + tiles_d, st, a.max_ctas);
   if (err == cudaSuccess && marks) err = cudaEventRecord(static_cast<cudaEvent_t>(marks[0]), st);
   *nlaunch += 1;
   return err;

@@ -423,7 +423,7 @@ static_assert(smem_bytes<256>() <= 227 * 1024 && smem_bytes<128>() <= 227 * 1024
               "shared memory budget");
 
 template <int MMA_N>
-cudaError_t launch_one(const GemmParams& p, int tiles_upper, cudaStream_t st) {
+cudaError_t launch_one(const GemmParams& p, int tiles_upper, cudaStream_t st, int max_ctas = 0) {
   static int configured_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -435,6 +435,7 @@ cudaError_t launch_one(const GemmParams& p, int tiles_upper, cudaStream_t st) {
     configured_dev = dev;
   }
   int grid = num_sms();
+  if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
   if (tiles_upper < grid) grid = tiles_upper;
   if (grid < 1) grid = 1;
   return launch_pdl(grouped_gemm_kernel<MMA_N>, dim3(grid), dim3(THREADS), smem_bytes<MMA_N>(),
@@ -591,11 +592,22 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, c
   p.nprob = 2;
   p.E = a.E; p.S = a.S; p.T = a.T;
   p.rows_r = rows_r;
-  const int tiles_g = mt_upper * ((a.F + half - 1) / half) + a.S * mt_s * ((a.Fs + half - 1) / half);
+  // one part of the groups: the routed experts (no shared tiles), or the
+  // shared experts (no routed groups; their counters live in counters_s)
+  int mt_r = mt_upper, S = a.S;
+  if (a.part == kFfnRouted) {
+    p.S = S = 0;
+  } else if (a.part == kFfnShared) {
+    p.E = 0;
+    mt_r = 0;
+    p.counters = a.counters_s;
+    p.sched = a.counters_s + a.S;
+  }
+  const int tiles_g = mt_r * ((a.F + half - 1) / half) + S * mt_s * ((a.Fs + half - 1) / half);
   const int nt_d = (a.D + nmma - 1) / nmma;
-  const int tiles_d = mt_upper * nt_d + a.S * mt_s * nt_d;
-  cudaError_t err = narrow ? launch_one<128>(p, tiles_g + tiles_d, st)
-                           : launch_one<256>(p, tiles_g + tiles_d, st);
+  const int tiles_d = mt_r * nt_d + S * mt_s * nt_d;
+  cudaError_t err = narrow ? launch_one<128>(p, tiles_g + tiles_d, st, a.max_ctas)
+                           : launch_one<256>(p, tiles_g + tiles_d, st, a.max_ctas);
   if (err == cudaSuccess && marks) err = cudaEventRecord(static_cast<cudaEvent_t>(marks[0]), st);
   *nlaunch += 1;
   return err;

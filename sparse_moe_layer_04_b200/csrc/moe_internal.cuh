@@ -46,7 +46,8 @@ cudaError_t noalloc_scratch(int32_t** out);
 
 // Workspace layout (byte offsets from the workspace base, 256-aligned).
 struct WsLayout {
-  size_t status, ticket, partials, wr3, idx, w, counts, offsets, perm, inv, blk_base, counters, xperm,
+  size_t status, ticket, partials, wr3, idx, w, counts, offsets, perm, inv, blk_base, counters,
+      counters_s, xperm,
       act_r, act_s, y, touched, total;
 };
 bool ws_layout(const moe_dims_t& d, WsLayout* out);
@@ -123,7 +124,20 @@ struct FfnArgs {
   int* status;
   int* counters;            // [E + S + 1], zero at launch (group counters, tile claims)
   int T, D, E, F, k, S, Fs;
+  // Which groups one launch runs: all, the routed experts only, or the shared
+  // experts only (then `counters_s` [S + 1], zero at launch, holds their group
+  // counters and tile claims, and the grid is at most `max_ctas` CTAs).
+  int part = 0;
+  int* counters_s = nullptr;
+  int max_ctas = 0;
 };
+constexpr int kFfnAll = 0, kFfnRouted = 1, kFfnShared = 2;
+// Batches of at most this many tokens run the shared experts (bf16 weights of
+// at least kOverlapSharedMinBytes) on an internal stream, next to the routing,
+// on at most kSharedCtas SMs.
+constexpr int kOverlapSharedMaxT = 512;
+constexpr double kOverlapSharedMinBytes = 16.0 * 1024 * 1024;
+constexpr int kSharedCtas = 32;
 // `marks` (nullable): one event recorded after the expert FFN kernel.
 cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch,
                               const char** why, void* const* marks);

@@ -249,3 +249,15 @@ def test_pipeline_binding_checks_host_tensors(mod):
         # pageable (or, without a GPU, unpinnable) host memory is refused
         mod.moe_pipeline_submit(p, torch.zeros(2, 16, dtype=torch.bfloat16),
                                 torch.zeros(2, 16, dtype=torch.float32))
+
+
+def test_shared_overlap_rule(mod):
+    f = mod.moe_forward_shared_overlap
+    assert f(mod.dims(T=128, D=6144, E=256, F=2048, k=8, S=1))
+    assert f(mod.dims(T=512, D=4096, E=8, F=64, k=2, S=1, Fs=1408))     # 33 MiB shared
+    assert not f(mod.dims(T=128, D=6144, E=256, F=2048, k=8, S=1), fp8_weights=True)
+    assert not f(mod.dims(T=513, D=6144, E=8, F=64, k=2, S=1, Fs=2048))
+    assert not f(mod.dims(T=128, D=6144, E=8, F=64, k=2, S=0))
+    assert not f(mod.dims(T=0, D=6144, E=8, F=64, k=2, S=1, Fs=2048))
+    assert not f(mod.dims(T=64, D=128, E=8, F=64, k=2, S=1))           # 48 KiB shared
+    assert not f(mod.dims(T=128, D=12, E=8, F=64, k=2, S=1))           # invalid dims

@@ -29,6 +29,9 @@ def test_decode_ffn_bytes_and_flops():
     assert bench.ffn_bytes(cfg, 10) == weights + rows * D * 2 + rows * D * 4 == 872939520
     assert bench.ffn_bytes(cfg, 10, "fp8") == 457728768
     assert bench.ffn_flops(cfg) == 6 * D * F * (T * k + T)
+    # the routed experts alone (shared expert on its own stream)
+    assert bench.ffn_bytes(cfg, 10, shared=False) == 10 * 3 * F * D * 2 + T * k * D * 6
+    assert bench.ffn_flops(cfg, shared=False) == 6 * D * F * T * k
     B, FL = bench.layer_bytes_flops(cfg, 10)
     assert B == weights + cfg.E * D * 4 + cfg.E * 4 + T * D * 2 + T * D * 4 + T * k * 8
     assert FL == 2 * T * D * cfg.E + bench.ffn_flops(cfg)
