@@ -108,6 +108,13 @@ def ffn_flops(cfg, shared: bool = True):
     return 6 * cfg.D * (cfg.F * cfg.T * cfg.k + cfg.Fs * cfg.T * S)
 
 
+def workload_name(cfg) -> str:
+    """The workload a bench line measures, named the same way by both arms."""
+    family = "GLM-4.5-Air" if cfg.weight_family == "glm45air" else "GLM-5.2"
+    return (f"{cfg.name}: {family}-shaped MoE layer T={cfg.T} D={cfg.D} E={cfg.E} k={cfg.k} "
+            f"F={cfg.F} S={cfg.S} Fs={cfg.Fs} scale={cfg.scale}")
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -470,12 +477,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded counter-based generator; random-init weights of the layer's shapes)",
-        "config": {"workload": f"{cfg.name}: GLM-5.2-shaped MoE layer T={cfg.T} D={cfg.D} "
-                               f"E={cfg.E} k={cfg.k} F={cfg.F} S={cfg.S} Fs={cfg.Fs} "
-                               f"scale={cfg.scale}" if cfg.weight_family != "glm45air" else
-                               f"{cfg.name}: GLM-4.5-Air-shaped MoE layer T={cfg.T} D={cfg.D} "
-                               f"E={cfg.E} k={cfg.k} F={cfg.F} S={cfg.S} Fs={cfg.Fs} "
-                               f"scale={cfg.scale}",
+        "config": {"workload": workload_name(cfg),
                    "T": cfg.T, "touched_experts": U, "global_batch": world * cfg.T,
                    "weights": ("fp8 e4m3 codes + power-of-two 128x128 block exponents, decoded "
                                "exactly to bf16 in the kernel" if fp8 is not None else "bf16"),
@@ -562,8 +564,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded counter-based generator)",
-        "config": {"workload": f"{cfg.name}: T={cfg.T} D={cfg.D} E={cfg.E} k={cfg.k} F={cfg.F} "
-                               f"S={cfg.S} Fs={cfg.Fs} scale={cfg.scale}", "T": cfg.T,
+        "config": {"workload": workload_name(cfg), "T": cfg.T,
                    "sample_tokens": n, "weights": args.weights},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},

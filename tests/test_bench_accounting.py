@@ -65,3 +65,10 @@ def test_traffic_record_follows_the_kernel_sources(tmp_path, monkeypatch):
     rec["sources_sha256_16"] = bench.source_digest(rec["sources"])
     (fake / "traffic.json").write_text(json.dumps({"expert_ffn/decode": rec}))
     assert bench.stored_traffic("expert_ffn/decode") == rec["dram_bytes_per_launch"]
+
+
+def test_both_arms_name_the_workload_alike():
+    for name in ("decode", "air", "tiny"):
+        w = bench.workload_name(mi.CONFIGS[name])
+        assert w.startswith(name + ": ") and f"T={mi.CONFIGS[name].T} " in w
+    assert "GLM-4.5-Air" in bench.workload_name(mi.CONFIGS["air"])
