@@ -110,8 +110,9 @@ def ffn_flops(cfg, shared: bool = True):
 
 def workload_name(cfg) -> str:
     """The workload a bench line measures, named the same way by both arms."""
-    family = "GLM-4.5-Air" if cfg.weight_family == "glm45air" else "GLM-5.2"
-    return (f"{cfg.name}: {family}-shaped MoE layer T={cfg.T} D={cfg.D} E={cfg.E} k={cfg.k} "
+    family = {"glm45air": "GLM-4.5-Air-shaped ", "glm52": "GLM-5.2-shaped "}.get(cfg.weight_family,
+                                                                               "small ")
+    return (f"{cfg.name}: {family}MoE layer T={cfg.T} D={cfg.D} E={cfg.E} k={cfg.k} "
             f"F={cfg.F} S={cfg.S} Fs={cfg.Fs} scale={cfg.scale}")
 
 
