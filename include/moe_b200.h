@@ -286,9 +286,11 @@ int moe_gather_rows(const void* src, int src_rows, const int32_t* idx, int n, in
 
 /* ---- Host-buffer pipeline ----------------------------------------------
  * The layer forward from page-locked host memory to page-locked host memory,
- * for callers whose hidden states live on the host (the pages' own runtime
- * stages activations between host and GPU, "GLM-5.2" PocketLLM, Implemented
- * execution path).  Each submitted step copies h [T, D] bf16 from the host,
+ * for callers whose hidden states live on the host.  The pages' decode
+ * profile names host-to-GPU staging (of the active experts) as one of the two
+ * hard floors of their runtime ("GLM-5.2" PocketLLM, Validated performance);
+ * here the weights stay resident and only the activations cross, overlapped
+ * with the layer.  Each submitted step copies h [T, D] bf16 from the host,
  * runs moe_forward / moe_forward_fp8 on the pipeline's compute stream and
  * copies out [T, D] fp32 back to the host.  The input copy runs on one copy
  * stream and the output copy on another, so the copies of step n+1 and n-1
