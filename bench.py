@@ -9,9 +9,17 @@ before every timed step, outside the step's events.  Prints one JSON line.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode]
   python bench.py --impl reference ...   # the CPU oracle on the host cores
 
-Multi-GPU (torchrun, one process per GPU): every rank runs an independent
-replica on its own batch (the layer shards over tokens with no exchange), so
-scaling is weak; the step time is the max over ranks.
+The headline is the --config workload (decode by default).  The same run then
+times the other workloads in `--per-config` (prefill, skew, GLM-4.5-Air and
+the N(0, 1)-hidden decode batch by default) with the same steps, warm-up and
+L2 flush, each with its own roofline and clock record, under
+"per_config" in the JSON line.
+
+Multi-GPU: one process per GPU.  Under torchrun (RANK/WORLD_SIZE set) every
+rank runs an independent replica on its own batch (the layer shards over
+tokens with no exchange), so scaling is weak and the step time is the max
+over ranks.  Without torchrun, `--gpus N` (N > 1) starts the N ranks itself
+through torch.distributed.run.
 """
 from __future__ import annotations
 
@@ -92,11 +100,21 @@ def layer_bytes_flops(cfg, U: int, weights: str = "bf16"):
 
 
 def ffn_bytes(cfg, U: int, weights: str = "bf16", shared: bool = True):
-    """Algorithmic bytes of one expert-FFN launch (gate/up and down GEMMs in one
-    kernel): W1, W3 and W2 of the touched routed experts and (with `shared`) of
-    the shared experts, the gathered bf16 input rows, and the fp32 expert
-    outputs written.  The gated activations stay inside the kernel's working
-    set and are not counted."""
+    """Algorithmic bytes of one expert-FFN launch: W1, W3 and W2 of the touched
+    routed experts and (with `shared`) of the shared experts, plus each token's
+    bf16 hidden row read once.  The gathered rows, the gated activations and
+    the fp32 expert outputs are the kernel's own intermediates and are not
+    counted."""
+    T, D, F, Fs = cfg.T, cfg.D, cfg.F, cfg.Fs
+    S = cfg.S if shared else 0
+    wb = 3 * (U * expert_weight_bytes(F, D, weights) + S * expert_weight_bytes(Fs, D, weights))
+    return wb + T * D * 2
+
+
+def ffn_kernel_bytes(cfg, U: int, weights: str = "bf16", shared: bool = True):
+    """The FFN launch's bytes with its row traffic: the weights, the gathered
+    bf16 input rows read and the fp32 expert outputs written (a secondary
+    figure; the roofline uses ffn_bytes)."""
     T, D, F, k, Fs = cfg.T, cfg.D, cfg.F, cfg.k, cfg.Fs
     S = cfg.S if shared else 0
     wb = 3 * (U * expert_weight_bytes(F, D, weights) + S * expert_weight_bytes(Fs, D, weights))
@@ -156,53 +174,78 @@ def stored_traffic(kernel_key: str):
 # ---------------------------------------------------------------------------
 # clocks
 # ---------------------------------------------------------------------------
-class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+_REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int):
-        self.proc = None
-        self.lines = []
+
+def summarize_clocks(samples):
+    """Clock record of a run from (sm_mhz, sm_max_mhz, reason_bits) samples:
+    median SM clock, the maximum, the throttle reasons seen, and the share of
+    samples with the power cap active."""
+    if not samples:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                "power_cap_fraction": 0.0}
+    reasons = sorted({n for _, _, bits in samples for n, b in _REASON_BITS.items() if bits & b})
+    capped = sum(1 for _, _, bits in samples if bits & _REASON_BITS["sw_power_cap"])
+    return {"sm_mhz": statistics.median(m for m, _, _ in samples),
+            "sm_max_mhz": max(x for _, x, _ in samples), "reasons": reasons,
+            "samples": len(samples), "power_cap_fraction": capped / len(samples)}
+
+
+class ClockSampler:
+    """Samples the SM clock and the clock-event (throttle) reasons of one GPU
+    every `period_s` in a background thread (NVML) between start() and stop(),
+    i.e. during the timed loops."""
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.period_s = period_s
+        self.samples = []
+        self.handle = None
+        self.thread = None
+        self.running = False
         try:
+            import pynvml
+            self.nvml = pynvml
+            pynvml.nvmlInit()
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
             gid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", gid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(gid.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
         except Exception:
-            self.proc = None
+            self.handle = None
+
+    def _run(self):
+        nv = self.nvml
+        while self.running:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                bits = self.reasons_fn(self.handle)
+                self.samples.append((float(mhz), float(self.max_mhz), int(bits)))
+            except Exception:
+                pass
+            time.sleep(self.period_s)
+
+    def start(self):
+        import threading
+        self.samples = []
+        if self.handle is None:
+            return self
+        self.running = True
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+        return self
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        mhz, maxs, reasons = [], [], set()
-        capped = 0
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                mhz.append(float(parts[1].split()[0]))
-                maxs.append(float(parts[2].split()[0]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-            capped += parts[8].lower() == "active"
-        if not mhz:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxs),
-                "reasons": sorted(reasons), "samples": len(mhz),
-                "power_cap_fraction": capped / len(mhz)}
+        if self.thread is not None:
+            self.running = False
+            self.thread.join()
+            self.thread = None
+        rec = summarize_clocks(self.samples)
+        rec["source"] = "NVML, sampled every %.0f ms during the timed loops" % (self.period_s * 1e3) \
+            if self.handle is not None else "unavailable"
+        return rec
 
 
 # ---------------------------------------------------------------------------
@@ -273,6 +316,185 @@ def cpu_baseline_from_device(cfg, inp, n_tokens: int, fp8=None):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+FP8_NAMES = ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2")
+
+
+def pick_tensor_peak(clocks, bf16_burst: float, bf16_sust: float):
+    """The tensor denominator: the burst figure for a step the power cap left
+    alone, the sustained one when the clock record shows the power cap active
+    in at least a quarter of the samples (long tensor-heavy steps run at the
+    capped clock).  Both fractions are reported either way."""
+    capped = bool(clocks) and clocks.get("power_cap_fraction", 0.0) >= 0.25
+    if capped:
+        return bf16_sust, "sustained (sw_power_cap active in >= 25% of the clock samples)"
+    return bf16_burst, "burst (power cap active in < 25% of the clock samples)"
+
+
+def roofline_report(cfg, U: int, weights: str, overlap: bool, ms: float, ffn_ms: float, clocks,
+                    peaks, peak_src: str, fp8: bool):
+    """The dominant kernel's roofline (the expert FFN launch) and the whole
+    layer's, for one measured configuration."""
+    hbm = float(peaks["hbm_gbs"])
+    bf16_burst = float(peaks["bf16_tflops"])
+    bf16_sust = float(peaks.get("bf16_tflops_sustained", bf16_burst))
+    bf16, tc_peak_choice = pick_tensor_peak(clocks, bf16_burst, bf16_sust)
+    B, FL = layer_bytes_flops(cfg, U, weights)
+    t_s = ms / 1e3
+    t_roof_hbm = B / (hbm * 1e9)
+    t_roof_tc = FL / (bf16 * 1e12)
+    # With the shared experts beside the routing on their own stream, the FFN
+    # launch timed here carries the routed experts only.
+    f_bytes = ffn_bytes(cfg, U, weights, shared=not overlap)
+    f_kbytes = ffn_kernel_bytes(cfg, U, weights, shared=not overlap)
+    f_flops = ffn_flops(cfg, shared=not overlap)
+    f_gbs = f_bytes / (ffn_ms / 1e3) / 1e9
+    f_tfs = f_flops / (ffn_ms / 1e3) / 1e12
+    f_bound = "hbm" if f_bytes / (hbm * 1e9) >= f_flops / (bf16 * 1e12) else "tensor"
+    if f_bound == "hbm":
+        roof = {"bound": "hbm", "achieved": f_gbs, "peak": hbm, "unit": "GB/s",
+                "frac": f_gbs / hbm}
+    else:
+        roof = {"bound": "tensor", "achieved": f_tfs, "peak": bf16, "unit": "TFLOP/s",
+                "frac": f_tfs / bf16}
+    traffic_key = (("expert_ffn_fp8" if fp8 else "expert_ffn")
+                   + ("_routed/" if overlap else "/") + cfg.name)
+    kernel = ("ffn_fp8_kernel (fused gate/up + down expert FFN, FP8 weights decoded into TMEM)"
+              if fp8 else "grouped_gemm_kernel (fused gate/up + down expert FFN)")
+    if overlap:
+        kernel += ("; routed experts (the shared expert's FFN runs beside the routing on an "
+                   "internal stream)")
+    roof.update({
+        "traffic": stored_traffic(traffic_key), "kernel": kernel, "ms": ffn_ms,
+        "algorithmic_bytes": f_bytes,
+        "algorithmic_bytes_def": "touched expert weights + each token's hidden row read once",
+        "algorithmic_flops": f_flops,
+        "hbm_frac": f_gbs / hbm,
+        "hbm_frac_with_row_traffic": f_kbytes / (ffn_ms / 1e3) / 1e9 / hbm,
+        "tensor_peak": tc_peak_choice,
+        "tensor_frac_burst": f_tfs / bf16_burst, "tensor_frac_sustained": f_tfs / bf16_sust,
+        "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured"
+        else "fallback (profiling recipe)"})
+    layer = {
+        "bytes": B, "flops": FL, "t_roof_ms": max(t_roof_hbm, t_roof_tc) * 1e3,
+        "binding": "hbm" if t_roof_hbm >= t_roof_tc else "tensor",
+        "frac": max(t_roof_hbm, t_roof_tc) / t_s,
+        "hbm_frac": t_roof_hbm / t_s, "tensor_frac": t_roof_tc / t_s,
+        "tensor_frac_burst": FL / (bf16_burst * 1e12) / t_s,
+        "tensor_frac_sustained": FL / (bf16_sust * 1e12) / t_s,
+        "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "bf16_tflops_burst": bf16_burst,
+                  "bf16_tflops_sustained": bf16_sust, "tensor_peak": tc_peak_choice,
+                  "source": peak_src}}
+    return roof, layer
+
+
+class Layer:
+    """One workload's inputs on the device and the layer call on them."""
+
+    def __init__(self, moe, cfg, inp, w8, dev):
+        self.moe, self.cfg, self.inp, self.w8 = moe, cfg, inp, w8
+        self.d = moe.dims_of(cfg)
+        self.ws = moe.alloc_workspace(self.d, dev)
+        self.out = torch.empty((cfg.T, cfg.D), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
+        self.wgt = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+
+    def forward(self, h, o, i=None, w=None):
+        moe, inp = self.moe, self.inp
+        if self.w8 is not None:
+            moe.moe_forward_fp8(h, inp["Wr"], inp["bias"], self.w8, self.d, o, self.ws, i, w)
+        else:
+            moe.moe_forward(h, inp["Wr"], inp["bias"], inp["W1"], inp["W3"], inp["W2"],
+                            inp["Ws1"], inp["Ws3"], inp["Ws2"], self.d, o, self.ws, i, w)
+
+    def step(self):
+        self.forward(self.inp["h"], self.out, self.idx, self.wgt)
+
+    def status_check(self, where: str):
+        if self.moe.moe_get_device_status(self.ws) != 0:
+            raise RuntimeError(f"device status error {where} ({self.cfg.name}): "
+                               + self.moe.moe_last_error())
+
+    def touched(self) -> int:
+        counts = torch.bincount(self.idx.flatten().long(), minlength=self.cfg.E)
+        return int((counts > 0).sum().item())
+
+
+def time_layer(L: Layer, K: int, warmup: int, flush, world: int, dev, sampler: ClockSampler):
+    """W untimed steps, then K timed steps (one event pair per step, nothing
+    recorded between the step's kernels), then K profiled steps (events at the
+    stage boundaries: stage times and the FFN launch's duration).  L2 flushed
+    before every step.  Returns the per-rank timings and the clock record of
+    the timed loops."""
+    moe = L.moe
+    for _ in range(warmup):
+        flush.zero_()
+        L.step()
+    torch.cuda.synchronize()
+    L.status_check("during warm-up")
+    launches = moe.moe_last_launch_count()
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for e in ev0 + ev1:  # create the CUDA events before the timed region
+        e.record()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_PROFILE_EVENTS)]
+          for _ in range(K)]
+    for evs in ev:
+        for e in evs:
+            e.record()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(K):
+        flush.zero_()
+        ev0[i].record()
+        L.step()
+        ev1[i].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    step_ms = [ev0[i].elapsed_time(ev1[i]) for i in range(K)]
+    for i in range(K):
+        flush.zero_()
+        moe.moe_set_profile_events(ev[i])
+        L.step()
+    moe.moe_set_profile_events(None)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    L.status_check("in the timed region")
+    stage_ms = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K))
+                for j, name in enumerate(STAGES)}
+    profiled_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][len(STAGES)]) for i in range(K))
+    ms, ffn_ms = max_over_ranks([statistics.mean(step_ms), stage_ms["expert_ffn"]], world, dev)
+    return {"ms": ms, "ffn_ms": ffn_ms, "step_ms": step_ms, "stage_ms": stage_ms,
+            "profiled_ms": profiled_ms, "launches": launches, "clocks": clocks}
+
+
+def config_inputs(moe, cfg, rank: int, dev, cache: dict, fp8_mode: bool):
+    """Device inputs of a workload: the weights of its family (generated once
+    per family and shared, with their FP8 codes in FP8 mode), its bias and its
+    hidden states (seeded by rank)."""
+    fam = cfg.weight_family
+    if fam not in cache:
+        w = mi.layer_weights(cfg, 0, device=dev)
+        w8 = None
+        if fp8_mode:
+            # the FP8 layer stores only codes and block exponents
+            q = mi.fp8_layer_weights(w)
+            for n in FP8_NAMES:
+                del w[n]
+            torch.cuda.empty_cache()
+            w8 = moe.fp8_weights(*(q[n + "q"] for n in FP8_NAMES), *(q[n + "e"] for n in FP8_NAMES))
+            w["_fp8"] = q
+        cache[fam] = (w, w8)
+    w, w8 = cache[fam]
+    inp = dict(w)
+    inp["bias"] = mi.correction_bias(cfg, 0, device=dev)
+    inp["h"] = mi.hidden(cfg, seed=replica_seed(rank), device=dev)
+    return inp, w8
+
+
 def run_ours(args, rank, world, local_rank):
     import sparse_moe_layer_04_b200 as moe
 
@@ -281,89 +503,18 @@ def run_ours(args, rank, world, local_rank):
     cfg = mi.CONFIGS[args.config]
     if args.experts or args.tokens:
         cfg = mi.custom_config(args.config, E=args.experts or cfg.E, T=args.tokens or cfg.T)
-    inp = mi.layer_weights(cfg, 0, device=dev)
-    inp["h"] = mi.hidden(cfg, seed=replica_seed(rank), device=dev)
-    fp8 = None
-    if args.weights == "fp8":
-        # the FP8 layer stores only codes and block exponents
-        fp8 = mi.fp8_layer_weights(inp)
-        for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2"):
-            del inp[n]
-        torch.cuda.empty_cache()
-        w8 = moe.fp8_weights(*(fp8[n + "q"] for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2")),
-                             *(fp8[n + "e"] for n in ("W1", "W3", "W2", "Ws1", "Ws3", "Ws2")))
-    d = moe.dims_of(cfg)
-    ws = moe.alloc_workspace(d, dev)
-    out = torch.empty((cfg.T, cfg.D), dtype=torch.float32, device=dev)
-    idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
-    wgt = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+    fp8_mode = args.weights == "fp8"
+    cache = {}
+    inp, w8 = config_inputs(moe, cfg, rank, dev, cache, fp8_mode)
+    L = Layer(moe, cfg, inp, w8, dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    def forward(h, o, i=None, w=None):
-        if fp8 is not None:
-            moe.moe_forward_fp8(h, inp["Wr"], inp["bias"], w8, d, o, ws, i, w)
-        else:
-            moe.moe_forward(h, inp["Wr"], inp["bias"], inp["W1"], inp["W3"], inp["W2"],
-                            inp["Ws1"], inp["Ws3"], inp["Ws2"], d, o, ws, i, w)
-
-    def step():
-        forward(inp["h"], out, idx, wgt)
-
     sampler = ClockSampler(local_rank)
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    if moe.moe_get_device_status(ws) != 0:
-        raise RuntimeError("device status error during warm-up: " + moe.moe_last_error())
-    launches_per_step = moe.moe_last_launch_count()
+    peaks, peak_src = load_peaks()
 
     K = args.steps
-    # headline loop: one event pair around each step (nothing recorded between
-    # the step's kernels, so their programmatic launch overlap is intact)
-    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    for e in ev0 + ev1:  # create the CUDA events before the timed region
-        e.record()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    for i in range(K):
-        flush.zero_()
-        ev0[i].record()
-        step()
-        ev1[i].record()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    step_ms = [ev0[i].elapsed_time(ev1[i]) for i in range(K)]
-
-    # profiled loop: events at every stage boundary (stage times and the
-    # dominant kernel's duration, measured on the launching stream)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.MOE_PROFILE_EVENTS)]
-          for _ in range(K)]
-    for evs in ev:
-        for e in evs:
-            e.record()
-    torch.cuda.synchronize()
-    for i in range(K):
-        flush.zero_()
-        moe.moe_set_profile_events(ev[i])
-        step()
-    moe.moe_set_profile_events(None)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    if moe.moe_get_device_status(ws) != 0:
-        raise RuntimeError("device status error in the timed region: " + moe.moe_last_error())
-
-    stage_ms = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K))
-                for j, name in enumerate(STAGES)}
-    profiled_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][len(STAGES)]) for i in range(K))
-    ms, ffn_ms = max_over_ranks([statistics.mean(step_ms), stage_ms["expert_ffn"]], world, dev)
-
-    counts = torch.bincount(idx.flatten().long(), minlength=cfg.E)
-    U = int((counts > 0).sum().item())
+    t = time_layer(L, K, args.warmup, flush, world, dev, sampler)
+    ms, ffn_ms = t["ms"], t["ffn_ms"]
+    U = L.touched()
 
     # end to end, serial: pinned host input -> device -> layer -> pinned host
     # output, each step waited for (context for the pipelined figure below)
@@ -372,13 +523,14 @@ def run_ours(args, rank, world, local_rank):
     h_dev = torch.empty_like(inp["h"])
     e2e_steps = min(K, 200)
     e2e_ms = []
+    sampler_e2e = ClockSampler(local_rank).start()
     for i in range(e2e_steps + 3):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         h_dev.copy_(h_pin, non_blocking=True)
-        forward(h_dev, out)
-        out_pin.copy_(out, non_blocking=True)
+        L.forward(h_dev, L.out)
+        out_pin.copy_(L.out, non_blocking=True)
         b.record()
         b.synchronize()
         if i >= 3:
@@ -391,11 +543,11 @@ def run_ours(args, rank, world, local_rank):
     # the copies of steps n+1 and n-1 run on their own streams while step n's
     # layer runs.  Timed over all steps, from an idle device to the last
     # output in host memory.
-    if fp8 is not None:
-        pipe = moe.moe_pipeline_create(d, inp["Wr"], inp["bias"], w8=w8, keep=(fp8,))
+    if w8 is not None:
+        pipe = moe.moe_pipeline_create(L.d, inp["Wr"], inp["bias"], w8=w8, keep=(inp["_fp8"],))
     else:
-        pipe = moe.moe_pipeline_create(d, inp["Wr"], inp["bias"], inp["W1"], inp["W3"], inp["W2"],
-                                       inp["Ws1"], inp["Ws3"], inp["Ws2"])
+        pipe = moe.moe_pipeline_create(L.d, inp["Wr"], inp["bias"], inp["W1"], inp["W3"],
+                                       inp["W2"], inp["Ws1"], inp["Ws3"], inp["Ws2"])
     outs_pin = [out_pin, torch.empty_like(out_pin).pin_memory()]
     for i in range(3):
         moe.moe_pipeline_submit(pipe, h_pin, outs_pin[i % 2])
@@ -415,55 +567,41 @@ def run_ours(args, rank, world, local_rank):
     moe.moe_pipeline_wait(pipe)   # every output is in host memory
     b.record()
     b.synchronize()
+    clocks_e2e = sampler_e2e.stop()
     moe.moe_pipeline_destroy(pipe)
     e2e = max_over_ranks([a.elapsed_time(b) / e2e_steps], world, dev)[0]
 
+    overlap = bool(moe.moe_forward_shared_overlap(L.d, w8 is not None))
+    roof, layer = roofline_report(cfg, U, args.weights, overlap, ms, ffn_ms, t["clocks"], peaks,
+                                  peak_src, w8 is not None)
+
+    # the other workloads, same steps, warm-up and L2 flush
+    per_config = {}
+    names = [n for n in (args.per_config.split(",") if args.per_config else []) if n]
+    for name in names:
+        if name == cfg.name:
+            continue
+        c = mi.CONFIGS[name]
+        cinp, cw8 = config_inputs(moe, c, rank, dev, cache, fp8_mode)
+        CL = Layer(moe, c, cinp, cw8, dev)
+        ct = time_layer(CL, K, args.warmup, flush, world, dev, sampler)
+        cU = CL.touched()
+        c_overlap = bool(moe.moe_forward_shared_overlap(CL.d, cw8 is not None))
+        croof, clayer = roofline_report(c, cU, args.weights, c_overlap, ct["ms"], ct["ffn_ms"],
+                                        ct["clocks"], peaks, peak_src, cw8 is not None)
+        per_config[name] = {
+            "workload": workload_name(c), "T": c.T, "touched_experts": cU,
+            "value": aggregate_tokens_per_s(c.T, world, ct["ms"]), "unit": "tokens/s",
+            "ms_per_step": ct["ms"],
+            "ms_p10_p90": [float(np.percentile(ct["step_ms"], 10)),
+                           float(np.percentile(ct["step_ms"], 90))],
+            "stage_ms": ct["stage_ms"], "roofline": croof, "layer_roofline": clayer,
+            "clocks": ct["clocks"], "gpu_launches": ct["launches"] * K}
+        del CL, cinp
+        torch.cuda.empty_cache()
+
     if rank != 0:
         return None
-
-    peaks, peak_src = load_peaks()
-    hbm = float(peaks["hbm_gbs"])
-    bf16_burst = float(peaks["bf16_tflops"])
-    bf16_sust = float(peaks.get("bf16_tflops_sustained", bf16_burst))
-    # The tensor denominator: the burst figure for a step the power cap left
-    # alone, the sustained one when the clock record of the run shows the power
-    # cap active in at least a quarter of the samples (long tensor-heavy steps
-    # run at the capped clock).  Both fractions are reported.
-    capped = bool(clocks) and clocks.get("power_cap_fraction", 0.0) >= 0.25
-    bf16 = bf16_sust if capped else bf16_burst
-    tc_peak_choice = ("sustained (sw_power_cap active in >= 25% of the clock samples)" if capped
-                      else "burst (power cap active in < 25% of the clock samples)")
-    B, FL = layer_bytes_flops(cfg, U, args.weights)
-    t_s = ms / 1e3
-    t_roof_hbm = B / (hbm * 1e9)
-    t_roof_tc = FL / (bf16 * 1e12)
-    # With the shared experts beside the routing on their own stream, the FFN
-    # launch timed here carries the routed experts only.
-    overlap = moe.moe_forward_shared_overlap(d, fp8 is not None)
-    f_bytes = ffn_bytes(cfg, U, args.weights, shared=not overlap)
-    f_flops = ffn_flops(cfg, shared=not overlap)
-    f_gbs = f_bytes / (ffn_ms / 1e3) / 1e9
-    f_tfs = f_flops / (ffn_ms / 1e3) / 1e12
-    f_bound = "hbm" if f_bytes / (hbm * 1e9) >= f_flops / (bf16 * 1e12) else "tensor"
-    if f_bound == "hbm":
-        roof = {"bound": "hbm", "achieved": f_gbs, "peak": hbm, "unit": "GB/s",
-                "frac": f_gbs / hbm}
-    else:
-        roof = {"bound": "tensor", "achieved": f_tfs, "peak": bf16, "unit": "TFLOP/s",
-                "frac": f_tfs / bf16}
-    traffic_key = (("expert_ffn_fp8" if fp8 is not None else "expert_ffn")
-                   + ("_routed/" if overlap else "/") + cfg.name)
-    kernel = ("ffn_fp8_kernel (fused gate/up + down expert FFN, FP8 weights decoded into TMEM)"
-              if fp8 is not None else "grouped_gemm_kernel (fused gate/up + down expert FFN)")
-    if overlap:
-        kernel += ("; routed experts (the shared expert's FFN runs beside the routing on an "
-                   "internal stream)")
-    roof.update({"traffic": stored_traffic(traffic_key), "kernel": kernel, "ms": ffn_ms,
-                 "algorithmic_bytes": f_bytes, "algorithmic_flops": f_flops,
-                 "tensor_peak": tc_peak_choice,
-                 "tensor_frac_burst": f_tfs / bf16_burst, "tensor_frac_sustained": f_tfs / bf16_sust,
-                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured"
-                 else "fallback (profiling recipe)"})
 
     res = {
         "metric": METRIC,
@@ -481,22 +619,14 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": workload_name(cfg),
                    "T": cfg.T, "touched_experts": U, "global_batch": world * cfg.T,
                    "weights": ("fp8 e4m3 codes + power-of-two 128x128 block exponents, decoded "
-                               "exactly to bf16 in the kernel" if fp8 is not None else "bf16"),
+                               "exactly to bf16 in the kernel" if w8 is not None else "bf16"),
                    "parallelism": f"replicas x{world} (token-parallel, no exchange)",
                    "l2": "flushed: 256 MiB memset before every timed step, outside its events",
-                   "ms_p10_p90": [float(np.percentile(step_ms, 10)), float(np.percentile(step_ms, 90))],
-                   "stage_ms": stage_ms, "profiled_step_ms": profiled_ms},
+                   "ms_p10_p90": [float(np.percentile(t["step_ms"], 10)),
+                                  float(np.percentile(t["step_ms"], 90))],
+                   "stage_ms": t["stage_ms"], "profiled_step_ms": t["profiled_ms"]},
         "roofline": roof,
-        "layer_roofline": {
-            "bytes": B, "flops": FL, "t_roof_ms": max(t_roof_hbm, t_roof_tc) * 1e3,
-            "binding": "hbm" if t_roof_hbm >= t_roof_tc else "tensor",
-            "frac": max(t_roof_hbm, t_roof_tc) / t_s,
-            "hbm_frac": t_roof_hbm / t_s, "tensor_frac": t_roof_tc / t_s,
-            "tensor_frac_burst": FL / (bf16_burst * 1e12) / t_s,
-            "tensor_frac_sustained": FL / (bf16_sust * 1e12) / t_s,
-            "peaks": {"hbm_gbs": hbm, "bf16_tflops": bf16, "bf16_tflops_burst": bf16_burst,
-                      "bf16_tflops_sustained": bf16_sust, "tensor_peak": tc_peak_choice,
-                      "source": peak_src}},
+        "layer_roofline": layer,
         "e2e": {"value": aggregate_tokens_per_s(cfg.T, world, e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": cfg.T * cfg.D * 2, "d2h_bytes_per_step": cfg.T * cfg.D * 4,
                 "ms_per_step": e2e, "steps": e2e_steps,
@@ -506,22 +636,33 @@ def run_ours(args, rank, world, local_rank):
                             "L2 flushed between steps inside the timed region" if flush_e2e else
                             "L2 not flushed (each step streams the touched experts' weights, "
                             "more than twice the 126 MB L2)"),
+                "clocks": clocks_e2e,
                 "serial": {"value": aggregate_tokens_per_s(cfg.T, world, e2e_serial),
                            "ms_per_step": e2e_serial,
                            "mode": "copy in, layer, copy out, then wait, per step; L2 flushed "
                                    "before every step outside its events"}},
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": t["launches"] * K,
         "gpu_launches_note": "kernels of the headline timed loop (the profiled loop runs as many again)",
-        "clocks": clocks,
+        "clocks": t["clocks"],
+        "per_config": per_config,
     }
     if world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline_from_device(cfg, inp, min(cfg.T, args.cpu_tokens), fp8)
+        res["cpu_baseline"] = cpu_baseline_from_device(
+            cfg, inp, min(cfg.T, args.cpu_tokens), inp.get("_fp8"))
     return res
 
 
 # ---------------------------------------------------------------------------
 # reference arm: the CPU oracle, as it stands, on the host cores
 # ---------------------------------------------------------------------------
+def host_memory_available() -> int:
+    try:
+        import psutil
+        return int(psutil.virtual_memory().available)
+    except Exception:
+        return 0
+
+
 def run_reference(args):
     from oracle import moe_oracle as orc
 
@@ -530,7 +671,15 @@ def run_reference(args):
     h = mi.hidden(cfg, 0).float().numpy()[:n]
     Wr = mi.router_weight(cfg, 0).numpy()
     bias = mi.correction_bias(cfg, 0).numpy()
+    # The oracle takes each selected expert's weights as fp64 arrays.  They are
+    # made once, before timing, and kept when they fit in half the free host
+    # memory; otherwise each pass makes them again from bf16 host copies (and
+    # that conversion is then inside the timed passes).
+    touched = np.unique(orc.route(orc.router_logits(h, Wr), bias, cfg.k, cfg.scale)[0])
+    per_expert = 3 * cfg.D * cfg.F * 8
+    keep_fp64 = len(touched) * per_expert <= host_memory_available() // 2
     cache = {}
+    bf16_copies = {}
 
     def matrices(ws):
         if args.weights == "fp8":   # the weights the FP8 codes stand for
@@ -539,9 +688,13 @@ def run_reference(args):
         return tuple(x.double().numpy() for x in ws)
 
     def expert(e):
-        if e not in cache:
-            cache[e] = matrices(mi.expert_weights(cfg, e, 0))
-        return cache[e]
+        if keep_fp64:
+            if e not in cache:
+                cache[e] = matrices(mi.expert_weights(cfg, e, 0))
+            return cache[e]
+        if e not in bf16_copies:
+            bf16_copies[e] = mi.expert_weights(cfg, e, 0)
+        return matrices(bf16_copies[e])
     shared = [matrices(mi.expert_weights(cfg, s, 0, shared=True)) for s in range(cfg.S)]
 
     def step():
@@ -558,9 +711,11 @@ def run_reference(args):
     ms = statistics.mean(times) * 1e3
     value = n / (ms / 1e3)
     cores = _blas_threads()
-    sample = (f"first {n} tokens of the {cfg.name} batch per step, whole layer in numpy "
-              f"(fp32 routing, fp64 experts); touched experts generated before timing")
-    return {
+    sample = (f"first {n} of {cfg.T} tokens of the {cfg.name} batch per step, whole layer in "
+              f"numpy (fp32 routing, fp64 experts); {len(touched)} touched experts' weights "
+              + ("made before timing" if keep_fp64 else
+                 "converted from bf16 host copies inside every pass (fp64 copies would not fit)"))
+    res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -572,6 +727,48 @@ def run_reference(args):
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
+    if n < cfg.T:
+        # linear extrapolation of the sample's rate to the whole batch (marked)
+        res["config"]["full_batch_s_extrapolated"] = cfg.T / value
+    return res
+
+
+# ---------------------------------------------------------------------------
+# launcher
+# ---------------------------------------------------------------------------
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def spawn_ranks(n: int, argv) -> int:
+    """Runs this script as n ranks (one process per GPU) under
+    torch.distributed.run on this node; returns its exit code."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={free_port()}",
+           os.path.abspath(__file__), *argv]
+    env = dict(os.environ)
+    env.setdefault("NCCL_DEBUG", "INFO")   # the NCCL log shows the rank count
+    env.setdefault("OMP_NUM_THREADS", "1")
+    return subprocess.call(cmd, env=env)
+
+
+def launcher_check(args, rank: int, world: int) -> int:
+    """Checks the rank layout without any CUDA work: every rank joins the
+    process group (gloo) and rank 0 prints the ranks it saw."""
+    torch.distributed.init_process_group("gloo", timeout=timedelta(seconds=60))
+    try:
+        seen = [None] * world
+        torch.distributed.all_gather_object(seen, {"rank": rank, "pid": os.getpid()})
+        if rank == 0:
+            print(json.dumps({"launcher_check": True, "n_gpus": world, "gpus_requested": args.gpus,
+                              "ranks": sorted(r["rank"] for r in seen),
+                              "pids": len({r["pid"] for r in seen})}), flush=True)
+    finally:
+        torch.distributed.destroy_process_group()
+    return 0
 
 
 def main():
@@ -580,6 +777,8 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", default="decode", choices=sorted(mi.CONFIGS))
+    ap.add_argument("--per-config", default="prefill,skew,air,decode_b",
+                    help="comma-separated workloads timed after the headline (empty: none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-tokens", type=int, default=128,
                     help="tokens of the batch the CPU oracle processes per pass")
@@ -591,11 +790,23 @@ def main():
                     help="override E (small cases for profiler captures; not a bench line)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (small cases for profiler captures; not a bench line)")
+    ap.add_argument("--launcher-check", action="store_true",
+                    help="start the ranks and report them over gloo, without any CUDA work")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    for name in (args.per_config.split(",") if args.per_config else []):
+        if name and name not in mi.CONFIGS:
+            ap.error(f"--per-config: unknown workload {name}")
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return spawn_ranks(args.gpus, sys.argv[1:])
     rank, world, local_rank = rank_env()
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but {world} ranks were started")
+
+    if args.launcher_check:
+        return launcher_check(args, rank, world)
 
     if args.impl == "reference":
         if rank != 0:

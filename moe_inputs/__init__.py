@@ -23,14 +23,16 @@ weights can be regenerated alone without materialising the others.
 
 Workloads (the layer shapes the GLM-5.2 and GLM-4.5-Air pages give)
 --------------------------------------------------------------------
-``CONFIGS`` lists the five workloads: a tiny layer for exhaustive checks, the
+``CONFIGS`` lists the workloads: a tiny layer for exhaustive checks, the
 GLM-5.2 layer at decode (T=128), prefill (T=4096) and skewed-load (T=16384)
-batch sizes, and the GLM-4.5-Air layer (T=8192).  Expert weights are
-N(0, 1/sqrt(fan_in)) (std = 1/sqrt(in-features)), the router is fp32
-N(0, 0.02), the correction bias fp32 N(0, 0.1).  The decode, prefill and skew
-workloads share one set of GLM-5.2 weights.  The skew workload replaces the
-bias by a stored calibrated vector (``skew_bias_T16384_seed0.txt``) that makes
-expert popularity follow Zipf(1.1) with 16 experts that receive no tokens.
+batch sizes, the GLM-4.5-Air layer (T=8192), and a second decode batch
+("decode_b") whose hidden states are N(0, 1) instead of N(0, 1/sqrt(D)).
+Expert weights are N(0, 1/sqrt(fan_in)) (std = 1/sqrt(in-features)), the
+router is fp32 N(0, 0.02), the correction bias fp32 N(0, 0.1).  The decode,
+decode_b, prefill and skew workloads share one set of GLM-5.2 weights.  The
+skew workload replaces the bias by a stored calibrated vector
+(``skew_bias_T16384_seed0.txt``) that makes expert popularity follow Zipf(1.1)
+with 16 experts that receive no tokens.
 """
 from __future__ import annotations
 
@@ -74,6 +76,10 @@ CONFIGS: Dict[str, LayerConfig] = {
     "decode": LayerConfig("decode", T=128, D=6144, E=256, k=8, F=2048, S=1, Fs=2048,
                           scale=2.5, hidden_std=1.0 / math.sqrt(6144),
                           weight_family="glm52"),
+    # decode batch with N(0, 1) hidden states: the router logits then spread the
+    # selection over about 108 experts instead of about 10 (reported, not a target)
+    "decode_b": LayerConfig("decode_b", T=128, D=6144, E=256, k=8, F=2048, S=1, Fs=2048,
+                            scale=2.5, hidden_std=1.0, weight_family="glm52"),
     "prefill": LayerConfig("prefill", T=4096, D=6144, E=256, k=8, F=2048, S=1, Fs=2048,
                            scale=2.5, hidden_std=1.0, weight_family="glm52"),
     "skew": LayerConfig("skew", T=16384, D=6144, E=256, k=8, F=2048, S=1, Fs=2048,

@@ -26,15 +26,49 @@ def test_decode_ffn_bytes_and_flops():
     T, D, F, k = cfg.T, cfg.D, cfg.F, cfg.k
     rows = T * k + T                                   # routed rows + shared rows
     weights = 11 * 3 * F * D * 2                       # 10 touched + 1 shared expert
-    assert bench.ffn_bytes(cfg, 10) == weights + rows * D * 2 + rows * D * 4 == 872939520
-    assert bench.ffn_bytes(cfg, 10, "fp8") == 457728768
+    # algorithmic: the touched weights and each token's hidden row read once
+    assert bench.ffn_bytes(cfg, 10) == weights + T * D * 2 == 832045056
+    # with the kernel's own row traffic (gathered rows in, fp32 rows out)
+    assert bench.ffn_kernel_bytes(cfg, 10) == weights + rows * D * 2 + rows * D * 4 == 872939520
+    assert bench.ffn_kernel_bytes(cfg, 10, "fp8") == 457728768
+    assert bench.ffn_bytes(cfg, 10, "fp8") == 3 * 11 * (F * D + 16 * 48) + T * D * 2
     assert bench.ffn_flops(cfg) == 6 * D * F * (T * k + T)
     # the routed experts alone (shared expert on its own stream)
-    assert bench.ffn_bytes(cfg, 10, shared=False) == 10 * 3 * F * D * 2 + T * k * D * 6
+    assert bench.ffn_bytes(cfg, 10, shared=False) == 10 * 3 * F * D * 2 + T * D * 2
+    assert bench.ffn_kernel_bytes(cfg, 10, shared=False) == 10 * 3 * F * D * 2 + T * k * D * 6
     assert bench.ffn_flops(cfg, shared=False) == 6 * D * F * T * k
     B, FL = bench.layer_bytes_flops(cfg, 10)
     assert B == weights + cfg.E * D * 4 + cfg.E * 4 + T * D * 2 + T * D * 4 + T * k * 8
     assert FL == 2 * T * D * cfg.E + bench.ffn_flops(cfg)
+
+
+def test_roofline_frac_is_algorithmic_bytes_over_time_over_peak():
+    cfg = mi.CONFIGS["decode"]
+    peaks = {"hbm_gbs": 6541.1, "bf16_tflops": 1650.0, "bf16_tflops_sustained": 1382.0}
+    clocks = bench.summarize_clocks([(1965.0, 1965.0, 0)] * 4)
+    roof, layer = bench.roofline_report(cfg, 10, "bf16", True, 0.18677, 0.13878, clocks, peaks,
+                                        "measured", False)
+    assert roof["bound"] == "hbm"
+    expect = bench.ffn_bytes(cfg, 10, shared=False) / 0.13878e-3 / 1e9 / 6541.1
+    assert roof["frac"] == pytest.approx(expect) and roof["frac"] == pytest.approx(0.8334, abs=1e-3)
+    assert roof["hbm_frac_with_row_traffic"] > roof["frac"]
+    B, _ = bench.layer_bytes_flops(cfg, 10)
+    assert layer["frac"] == pytest.approx(B / 6541.1e9 / 0.18677e-3)
+
+
+def test_clock_record_and_tensor_peak_choice():
+    assert bench.summarize_clocks([])["samples"] == 0
+    s = [(1965.0, 1965.0, 0), (1300.0, 1965.0, 0x4), (1290.0, 1965.0, 0x4 | 0x1),
+         (1310.0, 1965.0, 0x4)]
+    rec = bench.summarize_clocks(s)
+    assert rec["samples"] == 4 and rec["sm_mhz"] == pytest.approx(1305.0)
+    assert rec["sm_max_mhz"] == 1965.0
+    assert rec["reasons"] == ["sw_power_cap"] and rec["power_cap_fraction"] == 0.75
+    assert bench.pick_tensor_peak(rec, 1650.0, 1382.0)[0] == 1382.0
+    quiet = bench.summarize_clocks([(1965.0, 1965.0, 0)] * 4 + [(1965.0, 1965.0, 0x4)])
+    assert bench.pick_tensor_peak(quiet, 1650.0, 1382.0)[0] == 1650.0
+    hot = bench.summarize_clocks([(1700.0, 1965.0, 0x40 | 0x8)])
+    assert hot["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
 
 
 def test_throughput_counts_every_rank():

@@ -94,3 +94,32 @@ def test_failed_rank_ends_the_other_ranks_collective_with_an_error():
     assert procs[1].exitcode == 3
     msg = q.get(timeout=30)
     assert msg.startswith("error:")
+
+
+def test_bench_starts_the_ranks_it_is_asked_for():
+    """`bench.py --gpus 2` without torchrun starts two ranks itself (through
+    torch.distributed.run); the launcher check joins them over gloo without any
+    CUDA work and reports both."""
+    import json
+    import subprocess
+    env = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                          "--launcher-check"], capture_output=True, text=True, timeout=300,
+                         env=env, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [json.loads(x) for x in res.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    rec = lines[0]
+    assert rec["launcher_check"] and rec["n_gpus"] == 2 and rec["gpus_requested"] == 2
+    assert rec["ranks"] == [0, 1] and rec["pids"] == 2
+
+
+def test_bench_refuses_a_world_size_other_than_gpus():
+    import subprocess
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                          "--launcher-check"], capture_output=True, text=True, timeout=300,
+                         env=env, cwd=ROOT)
+    assert res.returncode != 0 and "--gpus 2 but 1 ranks" in res.stderr
