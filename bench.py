@@ -668,9 +668,13 @@ def run_reference(args):
 
     cfg = mi.CONFIGS[args.config]
     n = min(cfg.T, args.cpu_tokens)
-    h = mi.hidden(cfg, 0).float().numpy()[:n]
-    Wr = mi.router_weight(cfg, 0).numpy()
-    bias = mi.correction_bias(cfg, 0).numpy()
+    # the seeded inputs are made on the GPU when there is one (the same values
+    # as on the CPU, much faster) and copied to the host; the timed oracle
+    # passes run on the host cores only
+    gen = "cuda" if torch.cuda.is_available() else "cpu"
+    h = mi.hidden(cfg, 0, device=gen).float().cpu().numpy()[:n]
+    Wr = mi.router_weight(cfg, 0, device=gen).cpu().numpy()
+    bias = mi.correction_bias(cfg, 0, device=gen).cpu().numpy()
     # The oracle takes each selected expert's weights as fp64 arrays.  They are
     # made once, before timing, and kept when they fit in half the free host
     # memory; otherwise each pass makes them again from bf16 host copies (and
@@ -687,15 +691,18 @@ def run_reference(args):
                          for x in ws)
         return tuple(x.double().numpy() for x in ws)
 
+    def host_weights(e, shared=False):
+        return tuple(x.cpu() for x in mi.expert_weights(cfg, e, 0, device=gen, shared=shared))
+
     def expert(e):
         if keep_fp64:
             if e not in cache:
-                cache[e] = matrices(mi.expert_weights(cfg, e, 0))
+                cache[e] = matrices(host_weights(e))
             return cache[e]
         if e not in bf16_copies:
-            bf16_copies[e] = mi.expert_weights(cfg, e, 0)
+            bf16_copies[e] = host_weights(e)
         return matrices(bf16_copies[e])
-    shared = [matrices(mi.expert_weights(cfg, s, 0, shared=True)) for s in range(cfg.S)]
+    shared = [matrices(host_weights(s, shared=True)) for s in range(cfg.S)]
 
     def step():
         return orc.moe_layer_tokens(h, Wr, bias, cfg.k, cfg.scale, expert, shared)

@@ -156,7 +156,11 @@ int moe_permute(const int32_t* idx, const moe_dims_t* dims, int32_t* counts, int
  *    clearing.  Calls whose work overlaps on the GPU (different streams, or
  *    different host threads) race on the array and give wrong groupings.
  *  - Device-detected errors (an expert index out of range or repeated) are
- *    not recorded: there is no workspace to hold a status word. */
+ *    not recorded: there is no workspace to hold a status word.  With such
+ *    an idx, perm and inv are undefined (rows of the offending tokens keep
+ *    whatever the buffers held), so validate idx first when it may be bad.
+ *  - The looked-up address is cached per device and is not refreshed after
+ *    cudaDeviceReset; do not use the library across a device reset. */
 int moe_permute_noalloc(const int32_t* idx, const moe_dims_t* dims, int32_t* counts,
                         int32_t* offsets, int32_t* perm, int32_t* inv, moe_stream_t stream);
 
@@ -357,6 +361,17 @@ const int32_t* moe_ws_touched_experts(const void* ws, const moe_dims_t* dims);
  * moe_get_device_status) and returns; the CUDA context stays usable.  Takes
  * about two seconds of GPU time.  `ws` needs at least 256 bytes. */
 int moe_selftest_bounded_wait(void* ws, moe_stream_t stream);
+
+/* Self-test of forward progress under shared SMs: launches `nctas` CTAs on
+ * `stream`, each holding one SM (120 KB of shared memory, so no expert-FFN CTA
+ * fits beside it) for `cycles` SM clock cycles and then returning; they wait
+ * on nothing but their own clock.  A layer call issued meanwhile on another
+ * stream runs on the SMs that are left, and must finish there: the expert
+ * FFN's tiles are claimed only by CTAs that are already running, so none of
+ * its waits depends on a CTA that is not resident.
+ * nctas in [1, number of SMs], cycles in [0, 2^33] (about 4.4 s at the
+ * B200's maximum clock); MOE_ERR_INVALID_ARG otherwise.  No workspace. */
+int moe_selftest_occupy(int nctas, long long cycles, moe_stream_t stream);
 
 /* Synchronises `stream`, returns the first error recorded in the status word
  * of `ws` (MOE_OK if none) and clears the word. */

@@ -82,6 +82,7 @@ def _load() -> ctypes.CDLL:
         "moe_forward": (I, [P, P, P, P, P, P, P, P, P, D, P, P, P, P, Z, P]),
         "moe_get_device_status": (I, [P, P]),
         "moe_selftest_bounded_wait": (I, [P, P]),
+        "moe_selftest_occupy": (I, [I, ctypes.c_longlong, P]),
         "moe_ws_expert_counts": (P, [P, D]),
         "moe_ws_touched_experts": (P, [P, D]),
         "moe_last_error": (ctypes.c_char_p, []),
@@ -397,6 +398,11 @@ def _view_int32(ws: torch.Tensor, addr: int, n: int) -> torch.Tensor:
 def moe_selftest_bounded_wait(ws, stream=None) -> None:
     """Runs the bounded-wait self-test; moe_get_device_status then reports MOE_ERR_TIMEOUT."""
     _check(_lib.moe_selftest_bounded_wait(_ptr(ws, torch.uint8, "ws"), _stream(stream)))
+
+
+def moe_selftest_occupy(nctas: int, cycles: int, stream=None) -> None:
+    """Holds `nctas` SMs for `cycles` SM clock cycles on `stream` (waits on nothing else)."""
+    _check(_lib.moe_selftest_occupy(int(nctas), int(cycles), _stream(stream)))
 
 
 def moe_last_error() -> str:

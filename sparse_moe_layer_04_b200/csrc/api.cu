@@ -35,6 +35,8 @@ int cuda_fail(cudaError_t e, const char* what) {
 }
 
 constexpr int kMaxDev = 64;
+// Longest hold of moe_selftest_occupy: 2^33 cycles, about 4.4 s at 1.965 GHz.
+constexpr long long kOccupyMaxCycles = 1ll << 33;
 
 int check_device() {
   static int checked[kMaxDev] = {0};  // 0 unknown, 1 ok, -1 unsupported
@@ -275,8 +277,10 @@ FfnArgs ffn_args(const uint16_t* h, const uint16_t* xperm, const int32_t* offset
 
 cudaError_t launch_ffn(const FfnArgs& a, const ExpertWeights& wt, cudaStream_t st, int* n,
                        const char** why, void* const* marks) {
-  return wt.fp8 ? launch_expert_ffn_fp8(a, wt.f8, st, n, why, marks)
-                : launch_expert_ffn(a, st, n, why, marks);
+  if (wt.fp8) return launch_expert_ffn_fp8(a, wt.f8, st, n, why, marks);
+  // large batches: 256-row MMAs over SM pairs, tokens as the MMA's N
+  if (use_pair_ffn(a.T) && a.part == kFfnAll) return launch_expert_ffn_pair(a, st, n, why, marks);
+  return launch_expert_ffn(a, st, n, why, marks);
 }
 
 int expert_ffn_impl(const void* h, const int32_t* perm, const int32_t* offsets,
@@ -409,10 +413,16 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
   if (e == cudaSuccess) e = launch_router(hb, Wr, *dims, sp, w, partials, st, &n, &rwhy);
   if (e == cudaSuccess) e = mark(1, st);
   if (e != cudaSuccess) return cuda_fail(e, rwhy);
+  // Batches of at most 128 tokens with bf16 weights: the routed gate/up tiles
+  // read the token matrix itself (one row tile holds the whole batch), so no
+  // gathered copy is made; the routing kernel's grouping zeroes the FFN's
+  // counters instead of the gather kernel.
+  const bool dense = !wt.fp8 && T <= kDenseMaxT;
   if (T <= kPermBlockTokens) {
     // small batches: the routing kernel's last block also groups the pairs
     const RouteGrouping grp{counts, offsets, perm, inv, w.at<int32_t>(w.L.touched),
-                            w.at<int>(w.L.ticket)};
+                            w.at<int>(w.L.ticket), dense ? counters : nullptr,
+                            E + dims->S + 1};
     e = launch_route_and_group(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw,
                                w.status(), grp, st);
     if (e == cudaSuccess) e = mark(2, st);
@@ -429,12 +439,19 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
     if (e == cudaSuccess) e = mark(3, st);
     if (e != cudaSuccess) return cuda_fail(e, "permute launch");
   }
-  e = launch_gather_rows(hb, perm, T * k, D, T, xperm, counters, E + dims->S + 1, st);
+  if (!dense) {
+    e = launch_gather_rows(hb, perm, T * k, D, T, xperm, counters, E + dims->S + 1, st);
+    n += 1;
+  }
   if (e == cudaSuccess) e = mark(4, st);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
-  n += 1;
   FfnArgs a = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
   if (overlap_shared) a.part = kFfnRouted;
+  if (dense) {
+    a.dense_a = 1;
+    a.idx = idx;
+    a.inv = inv;
+  }
   const char* why = "launch failed";
   e = launch_ffn(a, wt, st, &n, &why, g_prof_events ? g_prof_events + 5 : nullptr);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
@@ -817,6 +834,21 @@ int moe_selftest_bounded_wait(void* ws, moe_stream_t stream) {
   cudaError_t e = launch_bounded_wait_selftest(static_cast<int*>(ws),
                                                reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  g_launches = 1;
+  return MOE_OK;
+}
+
+int moe_selftest_occupy(int nctas, long long cycles, moe_stream_t stream) {
+  g_err.clear();
+  g_launches = 0;
+  int rc = check_device();
+  if (rc) return rc;
+  if (nctas < 1 || nctas > num_sms())
+    return fail(MOE_ERR_INVALID_ARG, "nctas = %d outside [1, %d]", nctas, num_sms());
+  if (cycles < 0 || cycles > kOccupyMaxCycles)
+    return fail(MOE_ERR_INVALID_ARG, "cycles = %lld outside [0, %lld]", cycles, kOccupyMaxCycles);
+  cudaError_t e = launch_occupy_selftest(nctas, cycles, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "occupy self-test launch");
   g_launches = 1;
   return MOE_OK;
 }

@@ -59,6 +59,15 @@ struct GemmParams {
   int nprob;                 // 1 or 2
   int E, S, T;
   int rows_r;                // T * k
+  // Batches of at most 128 tokens (one row tile): the A operand of every
+  // routed gate/up tile is the whole token matrix (a_r maps h [T, D]), so no
+  // gathered copy is made, and the epilogue writes the row of each token
+  // routed to the tile's expert at that pair's grouped row (from idx / inv);
+  // the other tokens' rows are dropped.
+  int dense_a;
+  int k;
+  const int32_t* idx;        // [T, k] (dense_a)
+  const int32_t* inv;        // [T, k] (dense_a)
 };
 
 // Row blocks of the routed groups, built on the device from the group
@@ -182,13 +191,18 @@ __device__ __forceinline__ void tile_k_range(const TileInfo& ti, const Problem& 
   }
 }
 
-// Tile scheduling.  CTA c starts with tile c; later tiles are claimed in
-// increasing order from a global counter (the first claim returns gridDim.x),
-// so CTAs that finish early take more tiles; without a counter, CTA c takes
-// c, c + gridDim.x, ...  Either way every tile below a claimed one has been
-// taken by a running CTA, which the gate/up -> down hand-off relies on.
+// Tile scheduling.  With a claim counter (the expert FFN) a CTA claims every
+// tile it runs, its first one included, from the counter, so tiles are handed
+// out in increasing order and only to CTAs that are already running: a tile
+// that another tile waits for (a gate/up tile of a down tile's group) is
+// always held by a resident CTA, however many SMs other kernels occupy.  CTAs
+// that finish early take more tiles.  Without a counter (the router GEMM,
+// whose tiles wait on nothing) CTA c takes c, c + gridDim.x, ...
+__device__ __forceinline__ int first_tile(const GemmParams& p) {
+  return p.sched ? atomicAdd(p.sched, 1) : (int)blockIdx.x;
+}
 __device__ __forceinline__ int claim_tile(const GemmParams& p, int tile) {
-  return p.sched ? (int)gridDim.x + atomicAdd(p.sched, 1) : tile + (int)gridDim.x;
+  return p.sched ? atomicAdd(p.sched, 1) : tile + (int)gridDim.x;
 }
 
 // Queue of claimed tiles from the producer to the other roles of the CTA.
@@ -238,14 +252,14 @@ __device__ __forceinline__ void load_acc16(uint32_t taddr, uint32_t d1_off, bool
 // up in [HALF, 2 HALF)) and store bf16; down tiles store fp32.  `taddr` is the
 // warp's TMEM lane quarter at the accumulator's first column; with `two` the
 // tile is the sum of that accumulator and the one d1_off columns further.
+// `row_ok` / `out_row`: whether this lane's accumulator row is stored, and
+// the output row it goes to.
 template <int MMA_N>
 __device__ __forceinline__ void store_tile(const TileInfo& ti, const Problem& P, uint32_t taddr,
-                                           uint32_t d1_off, bool two, int q, int lane) {
+                                           uint32_t d1_off, bool two, bool row_ok,
+                                           size_t out_row) {
   constexpr int HALF = MMA_N / 2;
-  const int r = ti.m0 + q * 32 + lane;       // row within the group
-  const bool row_ok = r < ti.rows;
   const int N = ti.shared ? P.N_s : P.N_r;
-  const size_t out_row = (size_t)ti.row0 + r;
   if (P.gateup) {
     uint16_t* out = static_cast<uint16_t*>(ti.shared ? P.out_s : P.out_r);
 #pragma unroll 1

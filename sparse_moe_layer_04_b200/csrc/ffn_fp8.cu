@@ -24,8 +24,10 @@
 //            (lanes 0-15) and up rows (lanes 16-31) of the same 16 features,
 //            and the epilogue warp pairs them with one lane shuffle;
 //   down     one group x 128 output columns x a token block.
-// Ordering, dynamic tile claiming and the gate/up -> down hand-off (per-group
-// counters, bounded acquire waits) are those of the bf16 kernel.
+// Ordering, dynamic tile claiming (every tile, the first one included, from
+// the workspace counter, so waits never depend on CTAs that are not resident)
+// and the gate/up -> down hand-off (per-group counters, bounded acquire waits)
+// are those of the bf16 kernel.
 //
 // CTA (512 threads, one per SM):
 //   warp 0      token producer: TMA of token tiles (bf16, 128-byte swizzle,
@@ -257,6 +259,10 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
   // everything below reads what earlier kernels in the stream wrote
   ptx::pdl_wait();
 
+  // The weight producer claims the CTA's first tile now: the claim's latency
+  // hides under the construction of the tile map.
+  int first = 0;
+  if (warp == WPROD_WARP && lane == 0) first = first_tile(p);
   if (warp == 2) build_tile_map<NT>(ss.tm, p, lane);
   ptx::tc_fence_before();
   __syncthreads();
@@ -330,7 +336,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       uint32_t issued = 0, par = 0;
       int qslot = 0;
       uint32_t qphase = 0;
-      int tile = blockIdx.x;
+      int tile = first;
       int next = tile < total ? claim_tile(p, tile) : total;
       for (;;) {
         // hand the tile (or the end mark) to the other roles

@@ -19,20 +19,20 @@
 // Tiles are numbered problem 0 first, then problem 1; within a problem routed
 // experts first (expert, column tile, row tile with the row tile fastest, so
 // CTAs running at the same time share each weight tile through L2), then the
-// shared experts.  CTA c takes tile c first and then claims further tiles in
-// increasing order from a counter in the workspace (zeroed by the row-gather
-// kernel), so CTAs that finish early take more tiles; the weight producer passes
-// each claimed tile to the other roles through a small shared-memory
-// queue (the router GEMM, which has no such counter, takes c, c + gridDim.x,
-// ...).  A down tile of an
-// expert waits until every gate/up tile of that expert has been stored: each
-// gate/up epilogue warp releases a per-expert counter after a proxy fence, and
-// the producer acquires it before its TMA loads read the activations.  Down tiles
-// therefore fill the SMs that the tail of the gate/up tiles leaves idle.
-// Because tiles are taken in increasing order and all CTAs are resident (one
-// per SM), every counter a CTA waits on is advanced by tiles that precede it
-// and are held by running CTAs, so the waits always end; they are bounded all
-// the same.
+// shared experts.  Every CTA claims each of its tiles, the first one
+// included, in increasing order from a counter in the workspace (zeroed by the
+// row-gather kernel), so CTAs that finish early take more tiles; the weight
+// producer passes each claimed tile to the other roles through a small
+// shared-memory queue (the router GEMM, which has no such counter, takes c,
+// c + gridDim.x, ...).  A down tile of an expert waits until every gate/up
+// tile of that expert has been stored: each gate/up epilogue warp releases a
+// per-expert counter after a proxy fence, and the producer acquires it before
+// its TMA loads read the activations.  Down tiles therefore fill the SMs that
+// the tail of the gate/up tiles leaves idle.  A tile is only ever claimed by a
+// CTA that is already running, and all gate/up tiles precede all down tiles,
+// so every counter a CTA waits on is advanced by tiles held by running CTAs:
+// the waits end even when other kernels hold some of the SMs and only part of
+// the grid is resident.  They are bounded all the same.
 //
 // N (the MMA width) is 256 for large batches and 128 for small ones, where
 // each expert has only a row tile or two and the weight stream must be cut
@@ -178,6 +178,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   // everything below reads what earlier kernels in the stream wrote
   ptx::pdl_wait();
 
+  // The weight producer claims the CTA's first tile now: the claim's latency
+  // hides under the construction of the tile map.
+  int first = 0;
+  if (warp == BPROD_WARP && lane == 0) first = first_tile(p);
   // Routed row-tile map from the group offsets.
   if (warp == 2) build_tile_map(ss.tm, p, lane);
   ptx::tc_fence_before();
@@ -198,7 +202,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       uint32_t issued_mask = 0, last_parity = 0;
       int qslot = 0;
       uint32_t qphase = 0;
-      int tile = blockIdx.x;
+      int tile = first;
       int next = tile < total ? claim_tile(p, tile) : total;
       for (;;) {
         // hand the tile (or the end mark) to the other roles
@@ -276,7 +280,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           ptx::fence_proxy_async_global();
         }
         const CUtensorMap* amap = ti.shared ? &P.a_s : &P.a_r;
-        const int a_row = ti.shared ? ti.grp * P.a_s_group_stride + ti.m0 : ti.row0 + ti.m0;
+        const int a_row = ti.shared                    ? ti.grp * P.a_s_group_stride + ti.m0
+                          : (p.dense_a && ti.prob == 0) ? ti.m0
+                                                        : ti.row0 + ti.m0;
         int kbeg, K;
         tile_k_range(ti, P, &kbeg, &K);
         const int nk = (K + BK - 1) / BK;
@@ -389,7 +395,22 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       if (!ptx::mbar_wait(&ss.tmem_full[acc], acc_phase, abort)) break;
       ptx::tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BUF_COLS;
-      store_tile<MMA_N>(ti, P, taddr, ACC_COLS, two, q, lane);
+      const int r = ti.m0 + q * 32 + lane;   // accumulator row of this lane
+      bool row_ok = r < ti.rows;
+      size_t out_row = (size_t)ti.row0 + r;
+      if (p.dense_a && ti.prob == 0 && !ti.shared) {
+        // row r is token r: kept if the token chose this tile's expert
+        row_ok = false;
+        if (r < p.T) {
+          for (int j = 0; j < p.k; ++j) {
+            if (__ldcg(p.idx + (size_t)r * p.k + j) == ti.grp) {
+              row_ok = true;
+              out_row = (size_t)__ldcg(p.inv + (size_t)r * p.k + j);
+            }
+          }
+        }
+      }
+      store_tile<MMA_N>(ti, P, taddr, ACC_COLS, two, row_ok, out_row);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ss.tmem_empty[acc]);
@@ -538,7 +559,9 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, c
   GemmParams p{};
   // ---- problem 0: gate/up ----
   Problem& G = p.pr[0];
-  bool ok = make_map(&G.a_r, a.xperm, rows_r, a.D, BM) &&
+  const bool dense = a.dense_a != 0;
+  bool ok = (dense ? make_map(&G.a_r, a.h, a.T, a.D, BM)
+                   : make_map(&G.a_r, a.xperm, rows_r, a.D, BM)) &&
             make_map(&G.b0_r, a.W1, (uint64_t)a.E * a.F, a.D, half) &&
             make_map(&G.b1_r, a.W3, (uint64_t)a.E * a.F, a.D, half);
   if (ok && a.S > 0)
@@ -592,6 +615,10 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, c
   p.nprob = 2;
   p.E = a.E; p.S = a.S; p.T = a.T;
   p.rows_r = rows_r;
+  p.dense_a = dense ? 1 : 0;
+  p.k = a.k;
+  p.idx = a.idx;
+  p.inv = a.inv;
   // one part of the groups: the routed experts (no shared tiles), or the
   // shared experts (no routed groups; their counters live in counters_s)
   int mt_r = mt_upper, S = a.S;

@@ -93,6 +93,8 @@ struct RouteGrouping {
   int32_t* inv;
   int32_t* touched;
   int* ticket;  // nullptr: no grouping
+  int* zero;    // nullable: `nzero` ints the last block also sets to zero (the
+  int nzero;    // expert FFN's counters, when no row-gather kernel runs)
 };
 // Routing and grouping in one launch; T <= kPermBlockTokens.
 cudaError_t launch_route_and_group(const float* src, int nsplit, const float* bias, int T, int E,
@@ -130,7 +132,13 @@ struct FfnArgs {
   int part = 0;
   int* counters_s = nullptr;
   int max_ctas = 0;
+  // T <= kDenseMaxT with bf16 weights: the routed gate/up A operand is h
+  // itself (xperm is not used) and rows are placed by idx / inv [T, k].
+  int dense_a = 0;
+  const int32_t* idx = nullptr;
+  const int32_t* inv = nullptr;
 };
+constexpr int kDenseMaxT = 128;
 constexpr int kFfnAll = 0, kFfnRouted = 1, kFfnShared = 2;
 // Batches of at most this many tokens run the shared experts (bf16 weights of
 // at least kOverlapSharedMinBytes) on an internal stream, next to the routing,
@@ -141,6 +149,14 @@ constexpr int kSharedCtas = 32;
 // `marks` (nullable): one event recorded after the expert FFN kernel.
 cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch,
                               const char** why, void* const* marks);
+
+// The same expert MLPs for large batches (use_pair_ffn(T)): 256-row
+// tcgen05.mma.cta_group::2 tiles over SM pairs with the weights as the M
+// operand and the tokens of one group as N.  All groups in one launch
+// (a.part must be kFfnAll).
+bool use_pair_ffn(int T);
+cudaError_t launch_expert_ffn_pair(const FfnArgs& a, cudaStream_t st, int* nlaunch,
+                                   const char** why, void* const* marks);
 
 // FP8 expert weights: E4M3 codes and int8 block exponents (one per 128 x 128
 // block of each expert's [rows, K] matrix).
@@ -163,5 +179,6 @@ cudaError_t launch_gather_bytes(const void* src, int src_rows, const int32_t* id
 int num_sms();
 
 cudaError_t launch_bounded_wait_selftest(int* status, cudaStream_t st);
+cudaError_t launch_occupy_selftest(int nctas, long long cycles, cudaStream_t st);
 
 }  // namespace moe

@@ -13,6 +13,8 @@
 //             follow increasing token order, i.e. (token, slot) order.
 // Batches of at most 256 tokens (one counting block) run all three phases in
 // one launch.  All integer work: exact and deterministic.
+#include <atomic>
+
 #include "moe_internal.cuh"
 #include "permute_block.cuh"
 #include "sm100_ptx.cuh"
@@ -157,21 +159,25 @@ static __device__ __align__(256) int32_t g_perm_scratch[kNoAllocMaxBlocks * kNoA
 
 // Device address of the scratch array on the current device.  Host code only
 // sees a stand-in symbol for a __device__ array, so the address is looked up
-// with cudaGetSymbolAddress, once per device, with that device current.
+// with cudaGetSymbolAddress, once per device, with that device current.  The
+// cache is one atomic pointer per device: host threads whose first calls race
+// may each look the address up, and they store the same value.
 cudaError_t noalloc_scratch(int32_t** out) {
   constexpr int kMaxDevices = 64;
-  static int32_t* addr[kMaxDevices] = {};
+  static std::atomic<int32_t*> addr[kMaxDevices];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  if (!addr[dev]) {
+  int32_t* a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_perm_scratch);
     if (e != cudaSuccess) return e;
-    addr[dev] = static_cast<int32_t*>(p);
+    a = static_cast<int32_t*>(p);
+    addr[dev].store(a, std::memory_order_release);
   }
-  *out = addr[dev];
+  *out = a;
   return cudaSuccess;
 }
 
@@ -199,32 +205,51 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
 
 // xperm[r] = h[perm[r]] for every grouped row r (16-byte vector copies).  A
 // token id outside [0, T) (left by an invalid routing) yields a zero row.
-__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ h,
-                                                          const int32_t* __restrict__ perm,
-                                                          int D, int T,
-                                                          uint16_t* __restrict__ xperm,
-                                                          int* __restrict__ counters,
-                                                          int ncounters) {
+// One warp per row, the grid's warps striding over the rows; each lane keeps
+// eight 16-byte loads in flight before it stores them.
+constexpr int kGatherThreads = 256;
+constexpr int kGatherUnroll = 8;
+
+__global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(
+    const uint16_t* __restrict__ h, const int32_t* __restrict__ perm, int rows, int D, int T,
+    uint16_t* __restrict__ xperm, int* __restrict__ counters, int ncounters) {
   ptx::pdl_launch_dependents();
   ptx::pdl_wait();
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < ncounters; i += blockDim.x) counters[i] = 0;
-  const int r = blockIdx.x;
-  const int t = perm[r];
-  uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)r * D);
-  if (t < 0 || t >= T) {
-    for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
-    return;
+  const int lane = threadIdx.x & 31;
+  const int wpb = kGatherThreads / 32;
+  const int nwarps = gridDim.x * wpb;
+  const int n16 = D / 8;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < rows; r += nwarps) {
+    const int t = perm[r];
+    uint4* dst = reinterpret_cast<uint4*>(xperm + (size_t)r * D);
+    if (t < 0 || t >= T) {
+      for (int i = lane; i < n16; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(h + (size_t)t * D);
+    for (int i0 = lane; i0 < n16; i0 += 32 * kGatherUnroll) {
+      uint4 v[kGatherUnroll];
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u)
+        if (i0 + 32 * u < n16) v[u] = src[i0 + 32 * u];
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u)
+        if (i0 + 32 * u < n16) dst[i0 + 32 * u] = v[u];
+    }
   }
-  const uint4* src = reinterpret_cast<const uint4*>(h + (size_t)t * D);
-  for (int i = threadIdx.x; i < D / 8; i += blockDim.x) dst[i] = src[i];
 }
 
 cudaError_t launch_gather_rows(const uint16_t* h, const int32_t* perm, int rows, int D, int T,
                                uint16_t* xperm, int* counters, int ncounters, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-  return launch_pdl(gather_rows_kernel, dim3(rows), dim3(256), 0, st, h, perm, D, T, xperm,
-                    counters, ncounters);
+  const int wpb = kGatherThreads / 32;
+  int blocks = (rows + wpb - 1) / wpb;
+  const int cap = num_sms() * 4;
+  if (blocks > cap) blocks = cap;
+  return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(kGatherThreads), 0, st, h, perm, rows,
+                    D, T, xperm, counters, ncounters);
 }
 
 }  // namespace moe

@@ -185,9 +185,29 @@ FFN_CASES = [
 
 @pytest.mark.parametrize("T,D,E,F,k,S,Fs", FFN_CASES)
 def test_expert_ffn(moe, T, D, E, F, k, S, Fs):
+    _check_expert_ffn(moe, T, D, E, F, k, S, Fs, mi.synthetic_topk(T, E, k, 0, f"ffn{T}"))
+
+
+# Batches above 512 tokens run on SM pairs with up to 256 tokens of one expert
+# per tile: expert sizes around the 256-token block (0, 1, 15, 16, 17, 255,
+# 256, 257, 513 rows), a K tail (D = 136), features not a multiple of the
+# 128-feature pair tile (F = 192, 64) and output columns not a multiple of
+# the 256-column pair tile.
+PAIR_EDGE_COUNTS = [256, 257, 1, 0, 15, 16, 17, 138, 255, 513]
+
+
+@pytest.mark.parametrize("D,F,S,Fs", [(256, 256, 1, 128), (136, 192, 2, 64), (384, 64, 0, 0)])
+def test_expert_ffn_pair_block_edges(moe, D, F, S, Fs):
+    E = len(PAIR_EDGE_COUNTS)
+    idx = np.repeat(np.arange(E, dtype=np.int32), PAIR_EDGE_COUNTS)
+    order = mi.uniform_int(len(idx), 1 << 30, 0, "pair_edges").numpy().argsort(kind="stable")
+    idx = torch.from_numpy(idx[order].reshape(-1, 1).copy())   # k = 1, tokens shuffled
+    _check_expert_ffn(moe, len(idx), D, E, F, 1, S, Fs, idx)
+
+
+def _check_expert_ffn(moe, T, D, E, F, k, S, Fs, idx):
     cfg = mi.LayerConfig("ffn", T, D, E, k, F, S, max(Fs, 8), 2.5, 1.0, f"ffn{T}x{D}x{E}")
     inp = layer_on_device(cfg)
-    idx = mi.synthetic_topk(T, E, k, 0, f"ffn{T}")
     _, offsets, perm, _ = orc.group_by_expert(idx.numpy(), E)
     d = moe.dims(T=T, D=D, E=E, F=F, k=k, S=S, Fs=max(Fs, 8))
     ws = _ws(moe, d)
@@ -385,6 +405,46 @@ def test_forward_glm52_full_size(moe, glm52, name, n):
     assert int(moe.moe_ws_touched_experts(ws, d).item()) == int((counts > 0).sum())
     if name == "skew":
         assert (counts == 0).sum() >= 16 and counts.max() > 10 * counts.mean()
+
+
+def test_expert_ffn_full_size_heavy_experts(moe, glm52):
+    """Every row of the three heaviest experts of the skewed workload (thousands
+    of rows over many token blocks: the dynamic tile claims and the per-expert
+    gate/up -> down hand-off at their busiest) and of one expert whose last
+    token block is partial, at the GLM-5.2 sizes, against the oracle's expert
+    MLP on the same grouped rows."""
+    cfg = mi.CONFIGS["skew"]
+    T, E, k, D = cfg.T, cfg.E, cfg.k, cfg.D
+    inp = dict(glm52)
+    inp["h"] = mi.hidden(cfg, 0, device="cuda")
+    d = moe.dims_of(cfg)
+    ws = _ws(moe, d)
+    logits = torch.empty((T, E), device="cuda")
+    moe.moe_router_logits(inp["h"], inp["Wr"], d, logits, ws)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), device="cuda")
+    moe.moe_route(logits, inp["bias"], d, idx, w, ws)
+    counts, offsets, perm, _ = orc.group_by_expert(idx.cpu().numpy(), E)
+    y = torch.full((T * k + cfg.S * T, D), float("nan"), device="cuda")
+    moe.moe_expert_ffn(inp["h"], torch.from_numpy(perm).cuda(), torch.from_numpy(offsets).cuda(),
+                       inp["W1"], inp["W3"], inp["W2"], inp["Ws1"], inp["Ws3"], inp["Ws2"], d, y,
+                       ws)
+    assert moe.moe_get_device_status(ws) == 0
+    by_load = np.argsort(-counts, kind="stable")
+    heavy = [int(e) for e in by_load[:3]]
+    partial = next(int(e) for e in by_load[3:] if counts[e] > 256 and counts[e] % 128)
+    assert counts[heavy[-1]] > 1000
+    h = host_f32(inp["h"])
+    ex = HostExperts(inp["W1"], inp["W3"], inp["W2"])
+    for e in heavy + [partial]:
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        ref = orc.swiglu_expert(h[perm[a:b]], *ex(e))
+        got = y[a:b].cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(got))
+        assert rel_l2(got, ref) < 4e-3, e
+        row_err = np.linalg.norm(got - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1),
+                                                                 1e-30)
+        assert row_err.max() < 2e-2, e
 
 
 def test_forward_air_full_size(moe):

@@ -5,8 +5,10 @@ component, or a loop that may not take an allocation's device-wide
 synchronisation), so they cannot hand the library a workspace.  This checks,
 through the C ABI, that the variant whose scratch lives in the library's own
 static device array gives exactly the grouping of moe_permute with a caller
-workspace, on two calls in a row, for both the single-block (T <= 256) and the
-multi-block path, and that sizes beyond the array are refused.
+workspace and of the oracle's counting sort, on two calls in a row, for both
+the single-block (T <= 256) and the multi-block path, including the largest
+case the array holds (T = 16384, E = 1024: all 64 x 1024 entries), and that
+sizes beyond the array are refused.
 
 This file is collected last so that a failure here does not stop a run that
 stops at the first failure before every other test has run.
@@ -16,6 +18,7 @@ import pytest
 import torch
 
 import moe_inputs as mi
+from oracle import moe_oracle as orc
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +37,8 @@ def _outs(T, E, k):
             torch.empty((T, k), dtype=torch.int32, device="cuda"))
 
 
-@pytest.mark.parametrize("T,E,k", [(200, 256, 8), (3000, 256, 8), (16384, 64, 4), (777, 1024, 32)])
+@pytest.mark.parametrize("T,E,k", [(200, 256, 8), (3000, 256, 8), (16384, 64, 4), (777, 1024, 32),
+                                   (16384, 1024, 8)])
 def test_noalloc_matches_workspace_grouping_twice(moe, T, E, k):
     d = moe.dims(T=T, D=64, E=E, F=64, k=k)
     ws = moe.alloc_workspace(d)
@@ -49,6 +53,10 @@ def test_noalloc_matches_workspace_grouping_twice(moe, T, E, k):
         torch.cuda.synchronize()
         for a, b in zip(got, ref):
             assert torch.equal(a, b)
+        # and the oracle's counting sort of the same pairs, bit for bit
+        counts, offsets, perm, inv = orc.group_by_expert(idx.cpu().numpy(), E)
+        for a, b in zip(got, (counts, offsets, perm, inv)):
+            assert np.array_equal(a.cpu().numpy(), b)
 
 
 def test_noalloc_rejects_sizes_beyond_the_scratch(moe):
