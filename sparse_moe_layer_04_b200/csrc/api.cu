@@ -277,10 +277,8 @@ FfnArgs ffn_args(const uint16_t* h, const uint16_t* xperm, const int32_t* offset
 
 cudaError_t launch_ffn(const FfnArgs& a, const ExpertWeights& wt, cudaStream_t st, int* n,
                        const char** why, void* const* marks) {
-  if (wt.fp8) return launch_expert_ffn_fp8(a, wt.f8, st, n, why, marks);
-  // large batches: 256-row MMAs over SM pairs, tokens as the MMA's N
-  if (use_pair_ffn(a.T) && a.part == kFfnAll) return launch_expert_ffn_pair(a, st, n, why, marks);
-  return launch_expert_ffn(a, st, n, why, marks);
+  return wt.fp8 ? launch_expert_ffn_fp8(a, wt.f8, st, n, why, marks)
+                : launch_expert_ffn(a, st, n, why, marks);
 }
 
 int expert_ffn_impl(const void* h, const int32_t* perm, const int32_t* offsets,

@@ -39,10 +39,10 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
   const int v = blockIdx.y * kCombineThreads + threadIdx.x;
   if (v >= D / 4) return;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < S; ++s) {
-    const float4 a = reinterpret_cast<const float4*>(y + (rows_r + (size_t)s * T + t) * D)[v];
-    acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
-  }
+  // the first shared row is loaded with the first batch of routed rows, so a
+  // layer with one shared expert and k <= 8 reads all its rows in one round
+  float4 sh0 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (S > 0) sh0 = reinterpret_cast<const float4*>(y + (rows_r + t) * D)[v];
   for (int j0 = 0; j0 < k; j0 += 8) {
     float4 a[8];
 #pragma unroll
@@ -50,6 +50,14 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
       const int r = (j0 + q < k) ? s_row[j0 + q] : -1;
       a[q] = r >= 0 ? reinterpret_cast<const float4*>(y + (size_t)r * D)[v]
                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (j0 == 0) {
+      // shared experts first, in order
+      acc.x += sh0.x; acc.y += sh0.y; acc.z += sh0.z; acc.w += sh0.w;
+      for (int s = 1; s < S; ++s) {
+        const float4 b = reinterpret_cast<const float4*>(y + (rows_r + (size_t)s * T + t) * D)[v];
+        acc.x += b.x; acc.y += b.y; acc.z += b.z; acc.w += b.w;
+      }
     }
 #pragma unroll
     for (int q = 0; q < 8; ++q) {

@@ -402,11 +402,19 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         // row r is token r: kept if the token chose this tile's expert
         row_ok = false;
         if (r < p.T) {
-          for (int j = 0; j < p.k; ++j) {
-            if (__ldcg(p.idx + (size_t)r * p.k + j) == ti.grp) {
-              row_ok = true;
-              out_row = (size_t)__ldcg(p.inv + (size_t)r * p.k + j);
-            }
+          int hit = -1;
+          for (int j0 = 0; j0 < p.k; j0 += 8) {
+            int ev[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              ev[u] = (j0 + u < p.k) ? __ldcg(p.idx + (size_t)r * p.k + j0 + u) : -1;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              if (ev[u] == ti.grp) hit = j0 + u;
+          }
+          if (hit >= 0) {
+            row_ok = true;
+            out_row = (size_t)__ldcg(p.inv + (size_t)r * p.k + hit);
           }
         }
       }

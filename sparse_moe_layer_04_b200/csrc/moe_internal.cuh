@@ -150,14 +150,6 @@ constexpr int kSharedCtas = 32;
 cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch,
                               const char** why, void* const* marks);
 
-// The same expert MLPs for large batches (use_pair_ffn(T)): 256-row
-// tcgen05.mma.cta_group::2 tiles over SM pairs with the weights as the M
-// operand and the tokens of one group as N.  All groups in one launch
-// (a.part must be kFfnAll).
-bool use_pair_ffn(int T);
-cudaError_t launch_expert_ffn_pair(const FfnArgs& a, cudaStream_t st, int* nlaunch,
-                                   const char** why, void* const* marks);
-
 // FP8 expert weights: E4M3 codes and int8 block exponents (one per 128 x 128
 // block of each expert's [rows, K] matrix).
 struct Fp8Weights {

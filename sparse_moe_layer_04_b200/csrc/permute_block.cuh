@@ -19,6 +19,14 @@ inline size_t permute_block_smem(int E) {
   return (size_t)E * sizeof(int) + (size_t)E * kPermWords * sizeof(unsigned);
 }
 
+// Expert choices of one token read per batch, all loads in flight together.
+constexpr int kIdxBatch = 8;
+__device__ __forceinline__ void load_idx_batch(const int32_t* row, int j0, int k,
+                                               int (&ev)[kIdxBatch]) {
+#pragma unroll
+  for (int u = 0; u < kIdxBatch; ++u) ev[u] = (j0 + u < k) ? __ldcg(row + j0 + u) : 0;
+}
+
 // idx [T, k] is read with L2-coherent loads: it may have been written by
 // other blocks of the same grid just before.  Must be called by every thread
 // of the block; `sm` is permute_block_smem(E) bytes of shared memory.
@@ -42,15 +50,21 @@ __device__ __forceinline__ void permute_block(const int32_t* idx, int T, int E, 
     const int word = t >> 5;
     const unsigned bit = 1u << (t & 31);
     bool bad = false;
-    for (int j = 0; j < k; ++j) {
-      const int e = __ldcg(idx + (size_t)t * k + j);
-      if (e < 0 || e >= E) {
-        bad = true;
-        continue;
+    for (int j0 = 0; j0 < k; j0 += kIdxBatch) {
+      int ev[kIdxBatch];
+      load_idx_batch(idx + (size_t)t * k, j0, k, ev);   // all loads in flight together
+#pragma unroll
+      for (int u = 0; u < kIdxBatch; ++u) {
+        if (j0 + u >= k) break;
+        const int e = ev[u];
+        if (e < 0 || e >= E) {
+          bad = true;
+          continue;
+        }
+        atomicAdd(&cnt[e], 1);
+        const unsigned old = atomicOr(&mask[e * kPermWords + word], bit);
+        if (old & bit) bad = true;  // the same expert twice in one token
       }
-      atomicAdd(&cnt[e], 1);
-      const unsigned old = atomicOr(&mask[e * kPermWords + word], bit);
-      if (old & bit) bad = true;  // the same expert twice in one token
     }
     if (bad) {
       atomicOr(&bad_tok[word], bit);
@@ -92,14 +106,20 @@ __device__ __forceinline__ void permute_block(const int32_t* idx, int T, int E, 
     const int word = t >> 5;
     const unsigned bit = 1u << (t & 31);
     if (bad_tok[word] & bit) continue;
-    for (int j = 0; j < k; ++j) {
-      const int e = __ldcg(idx + (size_t)t * k + j);
-      const unsigned* m = mask + e * kPermWords;
-      int rank = __popc(m[word] & (bit - 1u));
-      for (int q = 0; q < word; ++q) rank += __popc(m[q]);
-      const int row = cnt[e] + rank;
-      perm[row] = t;
-      inv[(size_t)t * k + j] = row;
+    for (int j0 = 0; j0 < k; j0 += kIdxBatch) {
+      int ev[kIdxBatch];
+      load_idx_batch(idx + (size_t)t * k, j0, k, ev);
+#pragma unroll
+      for (int u = 0; u < kIdxBatch; ++u) {
+        if (j0 + u >= k) break;
+        const int e = ev[u];
+        const unsigned* m = mask + e * kPermWords;
+        int rank = __popc(m[word] & (bit - 1u));
+        for (int q = 0; q < word; ++q) rank += __popc(m[q]);
+        const int row = cnt[e] + rank;
+        perm[row] = t;
+        inv[(size_t)t * k + j0 + u] = row;
+      }
     }
   }
   if (any_bad && status) atomicOr(status, kStBounds);

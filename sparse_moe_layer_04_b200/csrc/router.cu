@@ -300,12 +300,14 @@ __device__ __forceinline__ bool score_and_key(const float* __restrict__ src, int
                                               float* key) {
   const float* p = src + at;
   float l = p[0];
-  for (int s0 = 1; s0 < nsplit; s0 += 16) {
-    float v[16];
+  // up to 32 plane loads in flight at once (the tensor-core router writes up
+  // to 64 planes); the sum still runs in plane order
+  for (int s0 = 1; s0 < nsplit; s0 += 32) {
+    float v[32];
 #pragma unroll
-    for (int q = 0; q < 16; ++q) v[q] = (s0 + q < nsplit) ? p[(s0 + q) * plane] : 0.f;
+    for (int q = 0; q < 32; ++q) v[q] = (s0 + q < nsplit) ? p[(s0 + q) * plane] : 0.f;
 #pragma unroll
-    for (int q = 0; q < 16; ++q)
+    for (int q = 0; q < 32; ++q)
       if (s0 + q < nsplit) l = __fadd_rn(l, v[q]);
   }
   const double sd = 1.0 / (1.0 + exp(-(double)l));

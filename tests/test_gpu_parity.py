@@ -188,18 +188,17 @@ def test_expert_ffn(moe, T, D, E, F, k, S, Fs):
     _check_expert_ffn(moe, T, D, E, F, k, S, Fs, mi.synthetic_topk(T, E, k, 0, f"ffn{T}"))
 
 
-# Batches above 512 tokens run on SM pairs with up to 256 tokens of one expert
-# per tile: expert sizes around the 256-token block (0, 1, 15, 16, 17, 255,
-# 256, 257, 513 rows), a K tail (D = 136), features not a multiple of the
-# 128-feature pair tile (F = 192, 64) and output columns not a multiple of
-# the 256-column pair tile.
-PAIR_EDGE_COUNTS = [256, 257, 1, 0, 15, 16, 17, 138, 255, 513]
+# Batches above 512 tokens (256-wide tiles): expert sizes around the 128-row
+# tile (0, 1, 15-17, 127-129, 255-257, 513 rows), a K tail (D = 136), F and Fs
+# not multiples of the 128-feature gate/up tile and D not a multiple of the
+# 256-column down tile.
+BLOCK_EDGE_COUNTS = [256, 257, 1, 0, 15, 16, 17, 138, 255, 513, 127, 128, 129]
 
 
 @pytest.mark.parametrize("D,F,S,Fs", [(256, 256, 1, 128), (136, 192, 2, 64), (384, 64, 0, 0)])
-def test_expert_ffn_pair_block_edges(moe, D, F, S, Fs):
-    E = len(PAIR_EDGE_COUNTS)
-    idx = np.repeat(np.arange(E, dtype=np.int32), PAIR_EDGE_COUNTS)
+def test_expert_ffn_block_edges(moe, D, F, S, Fs):
+    E = len(BLOCK_EDGE_COUNTS)
+    idx = np.repeat(np.arange(E, dtype=np.int32), BLOCK_EDGE_COUNTS)
     order = mi.uniform_int(len(idx), 1 << 30, 0, "pair_edges").numpy().argsort(kind="stable")
     idx = torch.from_numpy(idx[order].reshape(-1, 1).copy())   # k = 1, tokens shuffled
     _check_expert_ffn(moe, len(idx), D, E, F, 1, S, Fs, idx)

@@ -28,7 +28,7 @@ FREE_SMS = 40
 HOLD_CYCLES = 3_000_000_000
 
 CASES = {
-    # 256-wide tiles (T > 512): ~40 row tiles x 8 column tiles per GEMM
+    # 256-wide tiles (T > 512): ~40 row tiles x 8 or 4 column tiles per GEMM
     "wide": mi.custom_config("prefill", T=1024, D=2048, E=32, k=4, F=1024, S=1, Fs=1024,
                              name="progress_wide"),
     # 128-wide tiles with the shared expert's FFN beside the routing (25 MB of shared weights)
