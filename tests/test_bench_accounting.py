@@ -88,17 +88,17 @@ def test_traffic_record_follows_the_kernel_sources(tmp_path, monkeypatch):
     # a record taken on other sources is not reported
     fake = tmp_path / "profiles"
     fake.mkdir()
-    rec = dict(recs["expert_ffn/decode"], sources_sha256_16="0" * 16)
-    (fake / "traffic.json").write_text(json.dumps({"expert_ffn/decode": rec}))
+    rec = dict(recs["expert_ffn_routed/decode"], sources_sha256_16="0" * 16)
+    (fake / "traffic.json").write_text(json.dumps({"expert_ffn_routed/decode": rec}))
     for src in rec["sources"]:
         dst = tmp_path / src
         dst.parent.mkdir(parents=True, exist_ok=True)
         dst.write_bytes(open(os.path.join(ROOT, src), "rb").read())
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.stored_traffic("expert_ffn/decode") is None
+    assert bench.stored_traffic("expert_ffn_routed/decode") is None
     rec["sources_sha256_16"] = bench.source_digest(rec["sources"])
-    (fake / "traffic.json").write_text(json.dumps({"expert_ffn/decode": rec}))
-    assert bench.stored_traffic("expert_ffn/decode") == rec["dram_bytes_per_launch"]
+    (fake / "traffic.json").write_text(json.dumps({"expert_ffn_routed/decode": rec}))
+    assert bench.stored_traffic("expert_ffn_routed/decode") == rec["dram_bytes_per_launch"]
 
 
 def test_both_arms_name_the_workload_alike():
