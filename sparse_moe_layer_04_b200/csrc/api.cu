@@ -170,7 +170,7 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
   L->inv = take(T * k * 4);
   L->blk_base = take(nblk * E * 4);
   L->counters = take((E + S + 1) * 4);   // per-group counters + the tile claim counter
-  L->counters_s = take((S + 1) * 4);     // the same for a shared-experts-only launch
+  L->counters_s = take((S + 2) * 4);     // the same for a shared-experts-only launch, + its exit ticket
   L->xperm = take(T * k * D * 2);
   L->act_r = take(T * k * F * 2);
   L->act_s = take(S * T * Fs * 2);
@@ -389,9 +389,9 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
     e = side_stream(&side);
     if (e == cudaSuccess) e = cudaEventRecord(side->fork, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
+    // the shared launch's counters are zero: the workspace starts zeroed and
+    // the launch's last CTA to finish zeroes them again
     int32_t* counters_s = w.at<int32_t>(w.L.counters_s);
-    if (e == cudaSuccess)
-      e = cudaMemsetAsync(counters_s, 0, (size_t)(dims->S + 1) * sizeof(int32_t), side->s);
     if (e != cudaSuccess) return cuda_fail(e, "shared-expert stream");
     FfnArgs as = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
     as.part = kFfnShared;

@@ -54,6 +54,8 @@ struct GemmParams {
   int* status;
   int* counters;             // [E+S] gate/up tiles stored per group (two problems)
   int* sched;                // tile claim counter, zero at launch; nullptr: static round-robin
+  int* exit_ticket;          // nullable: the CTA that takes the last ticket at exit zeroes
+  int nreset;                // `counters[0, nreset)`, the claim counter and the ticket
   int weights_once;          // 1: weight tiles are read by about one row tile each, so
                              // they are loaded with an L2 evict-first policy
   int nprob;                 // 1 or 2
@@ -203,6 +205,22 @@ __device__ __forceinline__ int first_tile(const GemmParams& p) {
 }
 __device__ __forceinline__ int claim_tile(const GemmParams& p, int tile) {
   return p.sched ? atomicAdd(p.sched, 1) : tile + (int)gridDim.x;
+}
+
+// Leaves a launch's counters zero for the next launch that uses them: every
+// CTA takes an exit ticket once all its work is done; the last one (the
+// whole grid has finished its tiles) zeroes the group counters, the claim
+// counter and the ticket.  Called by one thread per CTA after the final
+// block-wide barrier.
+__device__ __forceinline__ void reset_counters_at_exit(const GemmParams& p) {
+  if (!p.exit_ticket) return;
+  __threadfence();
+  if (atomicAdd(p.exit_ticket, 1) == (int)gridDim.x - 1) {
+    for (int i = 0; i < p.nreset; ++i) p.counters[i] = 0;
+    *p.sched = 0;
+    *p.exit_ticket = 0;
+    __threadfence();
+  }
 }
 
 // Queue of claimed tiles from the producer to the other roles of the CTA.

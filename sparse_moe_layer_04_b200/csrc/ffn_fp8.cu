@@ -553,6 +553,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     ptx::tmem_dealloc(tmem_base, TMEM_COLS);
   }
   if (threadIdx.x == 0 && ss.abort && p.status) atomicOr(p.status, kStTimeout);
+  if (threadIdx.x == 0) reset_counters_at_exit(p);
 }
 
 template <int NT>
@@ -663,6 +664,8 @@ cudaError_t launch_expert_ffn_fp8(const FfnArgs& a, const Fp8Weights& w, cudaStr
     mt_r = 0;
     p.counters = a.counters_s;
     p.sched = a.counters_s + a.S;
+    p.exit_ticket = a.counters_s + a.S + 1;
+    p.nreset = a.S;
   }
   const int tiles_g = mt_r * cdiv(a.F, GU_FEATS) + S * mt_s * cdiv(a.Fs, GU_FEATS);
   const int tiles_d = (mt_r + S * mt_s) * cdiv(a.D, W_ROWS);

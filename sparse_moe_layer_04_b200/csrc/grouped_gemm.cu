@@ -434,6 +434,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     ptx::tmem_dealloc(tmem_base, TMEM_COLS);
   }
   if (threadIdx.x == 0 && ss.abort && p.status) atomicOr(p.status, kStTimeout);
+  if (threadIdx.x == 0) reset_counters_at_exit(p);
 }
 
 // ---------------------------------------------------------------------------
@@ -637,6 +638,8 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, c
     mt_r = 0;
     p.counters = a.counters_s;
     p.sched = a.counters_s + a.S;
+    p.exit_ticket = a.counters_s + a.S + 1;
+    p.nreset = a.S;
   }
   const int tiles_g = mt_r * ((a.F + half - 1) / half) + S * mt_s * ((a.Fs + half - 1) / half);
   const int nt_d = (a.D + nmma - 1) / nmma;

@@ -127,8 +127,9 @@ struct FfnArgs {
   int* counters;            // [E + S + 1], zero at launch (group counters, tile claims)
   int T, D, E, F, k, S, Fs;
   // Which groups one launch runs: all, the routed experts only, or the shared
-  // experts only (then `counters_s` [S + 1], zero at launch, holds their group
-  // counters and tile claims, and the grid is at most `max_ctas` CTAs).
+  // experts only (then `counters_s` [S + 2] holds their group counters, tile
+  // claims and an exit ticket; zero at launch, and the launch's last CTA to
+  // finish zeroes them again; the grid is at most `max_ctas` CTAs).
   int part = 0;
   int* counters_s = nullptr;
   int max_ctas = 0;
