@@ -34,8 +34,10 @@
  *    offsets, a bounded wait that ran out) raise bits of a status word kept at
  *    the start of the workspace; moe_get_device_status() reads and clears it.
  *    The caller zeroes the workspace once after allocating it (the library
- *    only ever ORs bits into the word).  Kernels never trap; after such an
- *    error the outputs are unspecified.
+ *    only ever ORs bits into the word, and the counters it keeps there are
+ *    left zero by every call that completes).  Kernels never trap; after such
+ *    an error the outputs are unspecified, and the workspace is zeroed again
+ *    before its next use.
  *  - Limits: 1 <= E <= 1024, 1 <= k <= min(E, 32), 0 <= S <= 16,
  *    T >= 0 (T = 0 enqueues nothing), D, F and Fs positive multiples of 8,
  *    scale finite, T * k < 2^31, and every buffer smaller than 2^31 rows.
