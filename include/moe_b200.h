@@ -36,8 +36,9 @@
  *    The caller zeroes the workspace once after allocating it (the library
  *    only ever ORs bits into the word, and the counters it keeps there are
  *    left zero by every call that completes).  Kernels never trap; after such
- *    an error the outputs are unspecified, and the workspace is zeroed again
- *    before its next use.
+ *    an error, or a negative return from a composite call whose earlier steps
+ *    were enqueued, the outputs are unspecified and the workspace is zeroed
+ *    again before its next use.
  *  - Limits: 1 <= E <= 1024, 1 <= k <= min(E, 32), 0 <= S <= 16,
  *    T >= 0 (T = 0 enqueues nothing), D, F and Fs positive multiples of 8,
  *    scale finite, T * k < 2^31, and every buffer smaller than 2^31 rows.
@@ -89,10 +90,13 @@ size_t moe_workspace_size(const moe_dims_t* dims);
  * h [T, D] bf16, Wr [E, D] fp32, logits [T, E] fp32 (output).  fp32-accurate:
  * when D % 64 == 0 and E % 8 == 0 the products run on the tensor cores
  * against an exact three-piece bf16 split of Wr (hi + mid + lo, within 2^-24
- * relative of Wr) with fp32 accumulation; otherwise with fp32 FMAs.  Either
+ * relative of Wr) with fp32 accumulation; otherwise with fp32 FMAs.  For
+ * T <= 256 with E % 64 == 0 one kernel reads Wr itself and splits each tile
+ * in shared memory; otherwise the split is written to `ws` first.  Either
  * way the summation order is fixed, so repeated calls give identical bits.
- * `ws` (>= moe_workspace_size bytes) holds the split weight and the partial
- * sums; it may be NULL only when neither is needed (small FMA cases). */
+ * `ws` (>= moe_workspace_size bytes) holds the split weight (when written),
+ * the partial sums and the status word; it may be NULL only in the small FMA
+ * cases that need none of them (then no status is kept). */
 int moe_router_logits(const void* h, const float* Wr, const moe_dims_t* dims, float* logits,
                       void* ws, size_t ws_bytes, moe_stream_t stream);
 

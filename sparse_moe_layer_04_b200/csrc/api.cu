@@ -117,6 +117,12 @@ int begin(const moe_dims_t* d) {
 cudaError_t launch_router(const uint16_t* h, const float* Wr, const moe_dims_t& d,
                           const RouterSplit& sp, const Ws& w, float* dst, cudaStream_t st, int* n,
                           const char** why) {
+  if (sp.fused) {
+    *n += 1;
+    *why = "router launch";
+    return launch_router_tc_fused(h, Wr, d.T, d.D, d.E, sp.nsplit, sp.chunk / 64, dst,
+                                  w.status(), st, why);
+  }
   if (sp.tensor) {
     uint16_t* wr3 = w.at<uint16_t>(w.L.wr3);
     cudaError_t e = launch_split_router(Wr, d.E, d.D, wr3, st);
@@ -161,7 +167,7 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
   L->status = take(256);
   L->ticket = take(256);
   L->partials = take((size_t)sp.nsplit * T * E * 4);
-  L->wr3 = take(sp.tensor ? E * 3 * D * 2 : 0);
+  L->wr3 = take(sp.tensor && !sp.fused ? E * 3 * D * 2 : 0);
   L->idx = take(T * k * 4);
   L->w = take(T * k * 4);
   L->counts = take(E * 4);
@@ -170,12 +176,14 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
   L->inv = take(T * k * 4);
   L->blk_base = take(nblk * E * 4);
   L->counters = take((E + S + 1) * 4);   // per-group counters + the tile claim counter
-  L->counters_s = take((S + 2) * 4);     // the same for a shared-experts-only launch, + its exit ticket
+  L->counters_s = take((S + 3) * 4);     // the same for a shared-experts-only launch, + its exit
+                                         // ticket and its "rows stored" flag
   L->xperm = take(T * k * D * 2);
   L->act_r = take(T * k * F * 2);
   L->act_s = take(S * T * Fs * 2);
   L->y = take((T * k + S * T) * D * 4);
   L->touched = take(4);
+  L->gmask = take(T <= kPermBlockTokens ? E * (kPermBlockTokens / 32) * 4 : 0);
   L->total = off;
   return true;
 }
@@ -396,6 +404,7 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
     FfnArgs as = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
     as.part = kFfnShared;
     as.counters_s = counters_s;
+    if (!wt.fp8) as.shared_done = counters_s + dims->S + 2;
     as.max_ctas = kSharedCtas;
     const char* swhy = "launch failed";
     e = launch_ffn(as, wt, side->s, &n, &swhy, nullptr);
@@ -420,7 +429,7 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
     // small batches: the routing kernel's last block also groups the pairs
     const RouteGrouping grp{counts, offsets, perm, inv, w.at<int32_t>(w.L.touched),
                             w.at<int>(w.L.ticket), dense ? counters : nullptr,
-                            E + dims->S + 1};
+                            E + dims->S + 1, w.at<uint32_t>(w.L.gmask)};
     e = launch_route_and_group(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw,
                                w.status(), grp, st);
     if (e == cudaSuccess) e = mark(2, st);
@@ -444,7 +453,10 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
   if (e == cudaSuccess) e = mark(4, st);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   FfnArgs a = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
-  if (overlap_shared) a.part = kFfnRouted;
+  if (overlap_shared) {
+    a.part = kFfnRouted;
+    if (!wt.fp8) a.shared_done = w.at<int32_t>(w.L.counters_s) + dims->S + 2;
+  }
   if (dense) {
     a.dense_a = 1;
     a.idx = idx;
@@ -453,7 +465,12 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
   const char* why = "launch failed";
   e = launch_ffn(a, wt, st, &n, &why, g_prof_events ? g_prof_events + 5 : nullptr);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
-  if (overlap_shared) {
+  // With the flag hand-off the routed launch completes only after the shared
+  // rows are stored, so the merge follows it directly (its launch overlaps the
+  // FFN's tail) and the streams are joined after it; otherwise the join comes
+  // first.
+  const bool flag_join = overlap_shared && a.shared_done;
+  if (overlap_shared && !flag_join) {
     guard.join = nullptr;
     e = cudaStreamWaitEvent(st, side->join, 0);
     if (e != cudaSuccess) return cuda_fail(e, "shared-expert stream");
@@ -462,6 +479,11 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
   if (e == cudaSuccess) e = mark(6, st);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   n += 1;
+  if (flag_join) {
+    guard.join = nullptr;
+    e = cudaStreamWaitEvent(st, side->join, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "shared-expert stream");
+  }
   g_launches = n;
   return MOE_OK;
 }

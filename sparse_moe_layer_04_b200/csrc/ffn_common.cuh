@@ -70,6 +70,13 @@ struct GemmParams {
   int k;
   const int32_t* idx;        // [T, k] (dense_a)
   const int32_t* inv;        // [T, k] (dense_a)
+  // Shared experts on an internal stream beside a routed-only launch: the
+  // shared launch's last CTA sets *done_flag once all its rows are stored;
+  // CTA 0 of the routed launch waits for *wait_flag (the same word) before it
+  // exits and clears it, so whatever follows the routed launch on its stream
+  // also sees the shared rows.  nullptr: no such hand-off.
+  int* done_flag;
+  int* wait_flag;
 };
 
 // Row blocks of the routed groups, built on the device from the group
@@ -220,7 +227,20 @@ __device__ __forceinline__ void reset_counters_at_exit(const GemmParams& p) {
     *p.sched = 0;
     *p.exit_ticket = 0;
     __threadfence();
+    if (p.done_flag) ptx::st_release_gpu(p.done_flag, 1);
   }
+}
+
+// CTA 0 of a routed-only launch: waits (bounded) until the shared launch on
+// the internal stream has stored all its rows, then clears the flag for the
+// next call.  Only this one CTA waits, once its own tiles are done; the other
+// CTAs exit and leave their SMs to the shared launch if it is still running.
+// Returns false if the wait gave up.
+__device__ __forceinline__ bool wait_shared_at_exit(const GemmParams& p, volatile int* abort) {
+  if (!p.wait_flag || blockIdx.x != 0) return true;
+  if (!ptx::counter_wait(p.wait_flag, 1, abort)) return false;
+  *p.wait_flag = 0;
+  return true;
 }
 
 // Queue of claimed tiles from the producer to the other roles of the CTA.

@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       for (;;) {
         if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
         const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
-        ptx::mbar_arrive(&ss.tq_empty[qslot]);
+        ptx::mbar_arrive_after_reads(&ss.tq_empty[qslot]);
         if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
         if (tile < 0) break;
         const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       for (;;) {
         if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
         const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
-        ptx::mbar_arrive(&ss.tq_empty[qslot]);
+        ptx::mbar_arrive_after_reads(&ss.tq_empty[qslot]);
         if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
         if (tile < 0) break;
         const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
@@ -448,6 +448,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     for (;;) {
       if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
       const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
+      __threadfence_block();   // the slot is read before lane 0 hands it back
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ss.tq_empty[qslot]);
       if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
@@ -481,6 +482,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     for (;;) {
       if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
       const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
+      __threadfence_block();   // the slot is read before lane 0 hands it back
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ss.tq_empty[qslot]);
       if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
@@ -522,7 +524,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           c4[c] = *reinterpret_cast<const uint4*>(rowp + ((c ^ swz) << 4));
-        ptx::mbar_arrive(&ss.w8_empty[my_ws]);
+        ptx::mbar_arrive_after_reads(&ss.w8_empty[my_ws]);
         bad_exp |= !fp8::exp_ok(e);
         const uint32_t s2 = fp8::scale_pair(e);
         uint32_t w[32];

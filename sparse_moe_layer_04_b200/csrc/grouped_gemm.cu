@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       for (;;) {
         if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
         const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
-        ptx::mbar_arrive(&ss.tq_empty[qslot]);
+        ptx::mbar_arrive_after_reads(&ss.tq_empty[qslot]);
         if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
         if (tile < 0) break;
         const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       for (;;) {
         if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
         const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
-        ptx::mbar_arrive(&ss.tq_empty[qslot]);
+        ptx::mbar_arrive_after_reads(&ss.tq_empty[qslot]);
         if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
         if (tile < 0) break;
         const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
@@ -383,6 +383,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     for (;;) {
       if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
       const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
+      __threadfence_block();   // the slot is read before lane 0 hands it back
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ss.tq_empty[qslot]);
       if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
@@ -433,8 +434,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, TMEM_COLS);
   }
-  if (threadIdx.x == 0 && ss.abort && p.status) atomicOr(p.status, kStTimeout);
-  if (threadIdx.x == 0) reset_counters_at_exit(p);
+  if (threadIdx.x == 0) {
+    wait_shared_at_exit(p, &ss.abort);
+    if (ss.abort && p.status) atomicOr(p.status, kStTimeout);
+    reset_counters_at_exit(p);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -500,8 +504,9 @@ bool make_tensor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
   const cuuint64_t strides[1] = {cols * (cuuint64_t)elem_bytes};
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapDataType dt =
-      elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUtensorMapDataType dt = elem_bytes == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE,
             swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -640,7 +645,9 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, c
     p.sched = a.counters_s + a.S;
     p.exit_ticket = a.counters_s + a.S + 1;
     p.nreset = a.S;
+    p.done_flag = a.shared_done;
   }
+  if (a.part == kFfnRouted) p.wait_flag = a.shared_done;
   const int tiles_g = mt_r * ((a.F + half - 1) / half) + S * mt_s * ((a.Fs + half - 1) / half);
   const int nt_d = (a.D + nmma - 1) / nmma;
   const int tiles_d = mt_r * nt_d + S * mt_s * nt_d;

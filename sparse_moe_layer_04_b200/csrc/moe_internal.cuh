@@ -30,9 +30,18 @@ constexpr int kRouterTileD = 32;
 // FMAs; both produce `nsplit` partial-sum planes [T, E] added in order.
 struct RouterSplit {
   bool tensor;  // tensor-core path
+  bool fused;   // tensor-core path that splits the fp32 weight in the kernel
   int nsplit;   // partial-sum planes
-  int chunk;    // reduction range of one plane (over D for FMA, over 3D for tensor)
+  int chunk;    // reduction range of one plane (over D for FMA and fused, over 3D for tensor)
 };
+// The fused tensor-core router (router_tc.cu): batches of at most
+// kRouterTcMaxT tokens with D % 64 == 0 and E % 32 == 0.
+constexpr int kRouterTcMaxT = 256;
+bool router_tc_shape_ok(int T, int D, int E);
+void router_tc_split(int T, int D, int E, int* nsplit, int* kb_per);
+cudaError_t launch_router_tc_fused(const uint16_t* h, const float* Wr, int T, int D, int E,
+                                   int nsplit, int kb_per, float* partials, int* status,
+                                   cudaStream_t st, const char** why);
 RouterSplit router_split(int T, int D, int E);
 int router_tile_n(int T, int E);  // MMA N of the tensor-core router
 
@@ -48,7 +57,7 @@ cudaError_t noalloc_scratch(int32_t** out);
 struct WsLayout {
   size_t status, ticket, partials, wr3, idx, w, counts, offsets, perm, inv, blk_base, counters,
       counters_s, xperm,
-      act_r, act_s, y, touched, total;
+      act_r, act_s, y, touched, gmask, total;
 };
 bool ws_layout(const moe_dims_t& d, WsLayout* out);
 
@@ -95,6 +104,9 @@ struct RouteGrouping {
   int* ticket;  // nullptr: no grouping
   int* zero;    // nullable: `nzero` ints the last block also sets to zero (the
   int nzero;    // expert FFN's counters, when no row-gather kernel runs)
+  // [E][kPermBlockTokens / 32] token bitmask per expert, zero between calls:
+  // each token's block sets its bits, the last block reads and clears them
+  uint32_t* mask;
 };
 // Routing and grouping in one launch; T <= kPermBlockTokens.
 cudaError_t launch_route_and_group(const float* src, int nsplit, const float* bias, int T, int E,
@@ -133,6 +145,10 @@ struct FfnArgs {
   int part = 0;
   int* counters_s = nullptr;
   int max_ctas = 0;
+  // bf16 kernel, shared and routed parts on two streams: the word the shared
+  // part sets when its rows are stored and the routed part waits for before
+  // it completes (nullptr: the streams are joined by an event instead).
+  int* shared_done = nullptr;
   // T <= kDenseMaxT with bf16 weights: the routed gate/up A operand is h
   // itself (xperm is not used) and rows are placed by idx / inv [T, k].
   int dense_a = 0;

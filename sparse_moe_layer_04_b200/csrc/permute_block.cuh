@@ -125,4 +125,121 @@ __device__ __forceinline__ void permute_block(const int32_t* idx, int T, int E, 
   if (any_bad && status) atomicOr(status, kStBounds);
 }
 
+// Grouping from the per-expert token bitmasks `gmask` [E][kPermWords] that
+// the routing blocks filled (bit t of row e: token t chose expert e), by the
+// routing kernel's last block.  The counts are the rows' popcounts; the pair
+// (t, j) with expert e = idx[t, j] goes to row offsets[e] + (number of tokens
+// below t in row e), which is the (token, slot) order of permute_block.  The
+// block reads the rows (L2-coherent: other blocks of the grid just set them)
+// and clears them for the next call.  Same outputs as permute_block for idx
+// rows of distinct in-range experts, which the routing always produces; an
+// out-of-range expert raises kStBounds and leaves its pair's perm/inv rows
+// unwritten.  Must be called by every thread of the block; `sm` is
+// permute_block_smem(E) bytes.
+__device__ __forceinline__ void group_from_masks(const int32_t* idx, int T, int E, int k,
+                                                 uint32_t* gmask, int32_t* counts,
+                                                 int32_t* offsets, int32_t* perm, int32_t* inv,
+                                                 int* status, int32_t* touched, int* sm) {
+  int* cnt = sm;                                           // [E]
+  unsigned* mask = reinterpret_cast<unsigned*>(sm + E);    // [E][W]
+  __shared__ int warp_tot[32];
+  __shared__ int nz_total;
+  const int nthr = blockDim.x;
+  const int W = (T + 31) >> 5;                             // words per expert row in use
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (threadIdx.x == 0) nz_total = 0;
+  // The first batch of pairs' experts is loaded together with the row words
+  // (one round trip for both when T * k <= blockDim * kIdxBatch).
+  const int npairs = T * k;
+  int ev0[kIdxBatch];
+#pragma unroll
+  for (int u = 0; u < kIdxBatch; ++u) {
+    const int pr = u * nthr + threadIdx.x;
+    ev0[u] = pr < npairs ? __ldcg(idx + pr) : 0;
+  }
+  // the row words are loaded in batches with every load in flight before any
+  // is stored or cleared
+  for (int i0 = 0; i0 < E * W; i0 += nthr * kIdxBatch) {
+    uint32_t v[kIdxBatch];
+#pragma unroll
+    for (int u = 0; u < kIdxBatch; ++u) {
+      const int i = i0 + u * nthr + threadIdx.x;
+      const int e = i / W, q = i - e * W;
+      v[u] = i < E * W ? __ldcg(gmask + (size_t)e * kPermWords + q) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kIdxBatch; ++u) {
+      const int i = i0 + u * nthr + threadIdx.x;
+      if (i >= E * W) break;
+      const int e = i / W, q = i - e * W;
+      mask[i] = v[u];
+      gmask[(size_t)e * kPermWords + q] = 0u;
+    }
+  }
+  __syncthreads();
+  // per-expert counts, then an exclusive scan over experts: thread i owns
+  // experts [i*per, (i+1)*per)
+  const int per = (E + nthr - 1) / nthr;
+  const int e0 = threadIdx.x * per;
+  int local = 0;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    int c = 0;
+    for (int q = 0; q < W; ++q) c += __popc(mask[e * W + q]);
+    cnt[e] = c;
+    local += c;
+  }
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_tot[wid] = incl;
+  __syncthreads();
+  int base = incl - local;
+  for (int q = 0; q < wid; ++q) base += warp_tot[q];
+  int nz = 0;
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    const int c = cnt[e];
+    counts[e] = c;
+    offsets[e] = base;
+    cnt[e] = base;
+    base += c;
+    nz += c > 0;
+  }
+  if (threadIdx.x == nthr - 1) offsets[E] = base;  // the last thread ends at the total
+  if (nz) atomicAdd(&nz_total, nz);
+  __syncthreads();
+  if (touched && threadIdx.x == 0) *touched = nz_total;
+  // one pair per thread and round: row = offset + rank of t in its expert's row
+  bool bad = false;
+  for (int p0 = 0; p0 < npairs; p0 += nthr * kIdxBatch) {
+    int ev[kIdxBatch];
+#pragma unroll
+    for (int u = 0; u < kIdxBatch; ++u) {
+      const int pr = p0 + u * nthr + threadIdx.x;
+      ev[u] = p0 == 0 ? ev0[u] : (pr < npairs ? __ldcg(idx + pr) : 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kIdxBatch; ++u) {
+      const int pr = p0 + u * nthr + threadIdx.x;
+      if (pr >= npairs) break;
+      const int e = ev[u];
+      if (e < 0 || e >= E) {
+        bad = true;
+        continue;
+      }
+      const int t = pr / k;
+      const int word = t >> 5;
+      const unsigned* m = mask + e * W;
+      int rank = __popc(m[word] & ((1u << (t & 31)) - 1u));
+      for (int q = 0; q < word; ++q) rank += __popc(m[q]);
+      const int row = cnt[e] + rank;
+      perm[row] = t;
+      inv[pr] = row;
+    }
+  }
+  if (bad && status) atomicOr(status, kStBounds);
+}
+
 }  // namespace moe

@@ -26,6 +26,15 @@ int router_tile_n(int T, int E) { return (E <= 128 || T <= 512) ? 128 : 256; }
 
 RouterSplit router_split(int T, int D, int E) {
   RouterSplit sp;
+  sp.fused = false;
+  if (router_tc_shape_ok(T, D, E)) {
+    int kb_per = 1;
+    sp.tensor = true;
+    sp.fused = true;
+    router_tc_split(T, D, E, &sp.nsplit, &kb_per);
+    sp.chunk = kb_per * 64;
+    return sp;
+  }
   if (D % 64 == 0 && E % 8 == 0) {
     // tensor path: enough (row tile, column tile, K' chunk) work units for
     // about one wave; at most 64 planes
@@ -316,43 +325,99 @@ __device__ __forceinline__ bool score_and_key(const float* __restrict__ src, int
   return isfinite(l) && isfinite(*key);
 }
 
-// Routing with one block per token, one thread per expert.
+// Top-k of one token by warp 0 of the block from the block's shared arrays
+// s_ord (order key of every expert, 0 for none; EPL * 32 entries) and s_sc
+// (its score): lane l holds the keys of experts l, l + 32, ..., and each of
+// the k rounds takes the warp's best (key descending, index ascending),
+// removes it at its owner and reads its score, as route_warp_kernel does, so
+// the selection, the fp32 slot-order sum and the weights are those bits.
+// Lanes j < k write slot j and, when `gmask` is set, token t's bit in the row
+// of its expert.  Other warps return at once.
+template <int EPL>
+__device__ __forceinline__ void warp0_topk_write(const uint32_t* s_ord, const float* s_sc, int t,
+                                                 int k, int E, float scale,
+                                                 int32_t* __restrict__ idx,
+                                                 float* __restrict__ w, uint32_t* gmask) {
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  uint32_t ord[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) ord[i] = s_ord[lane + 32 * i];
+  int my_e = 0;
+  float my_s = 0.f, sum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    uint32_t bu = 0u;
+    int be = INT_MAX;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      // increasing i visits increasing experts: ties keep the lower index
+      if (ord[i] > bu) {
+        bu = ord[i];
+        be = lane + 32 * i;
+      }
+    }
+    warp_best(bu, be);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+      if (be == lane + 32 * i) ord[i] = 0u;
+    if (!bu) be = INT_MAX;
+    const float bs = bu ? s_sc[be] : 0.f;
+    if (lane == j) {
+      my_e = be;
+      my_s = bs;
+    }
+    sum = (j == 0) ? bs : __fadd_rn(sum, bs);
+  }
+  if (lane < k) {
+    idx[(size_t)t * k + lane] = my_e;
+    w[(size_t)t * k + lane] = __fmul_rn(__fdiv_rn(my_s, sum), scale);
+    // grouping: token t's bit in the row of each expert it chose
+    if (gmask && my_e >= 0 && my_e < E)
+      atomicOr(gmask + (size_t)my_e * kPermWords + (t >> 5), 1u << (t & 31));
+  }
+}
+
+// Routing with one block per token, one thread per expert (EPL * 32 threads,
+// EPL = ceil(E / 32)).
 //
 // With grp.ticket set (T <= kPermBlockTokens), the kernel also groups the
-// pairs by expert (permute_block) in whichever block finishes last, which
+// pairs by expert (group_from_masks) in whichever block finishes last, which
 // saves the grouping kernel's launch on small batches.
+template <int EPL>
 __global__ void __launch_bounds__(1024) route_kernel(
     const float* __restrict__ src, int nsplit, const float* __restrict__ bias, int T, int E,
     int k, float scale, int32_t* __restrict__ idx, float* __restrict__ w,
     int* __restrict__ status, RouteGrouping grp) {
   ptx::pdl_launch_dependents();
   ptx::pdl_wait();
-  __shared__ uint32_t c_u[kMaxSlots * kMaxSlots];
-  __shared__ int c_e[kMaxSlots * kMaxSlots];
-  __shared__ float s_sc[1024];
+  __shared__ uint32_t s_ord[32 * EPL];
+  __shared__ float s_sc[32 * EPL];
   const int t = blockIdx.x;
   const int e = threadIdx.x;
-  float key = -INFINITY, sc = 0.f;
-  int me = INT_MAX, bad = 0;
+  int bad = 0;
   if (e < E) {
+    float key, sc;
     bad = !score_and_key(src, nsplit, (size_t)T * E, (size_t)t * E + e, bias[e], &sc, &key);
-    me = e;
+    s_ord[e] = key_order(key);
+    s_sc[e] = sc;
+  } else {
+    s_ord[e] = 0u;
   }
   if (__syncthreads_or(bad) && e == 0 && status) atomicOr(status, kStNonFinite);
-  block_topk_write(key, sc, me, t, k, scale, idx, w, c_u, c_e, s_sc);
+  warp0_topk_write<EPL>(s_ord, s_sc, t, k, E, scale, idx, w, grp.mask);
   if (!grp.ticket) return;
-  // The last block to finish groups every token's pairs by expert: each
-  // block's indices are visible GPU-wide before it takes its ticket.
+  // The last block to finish groups every token's pairs by expert.  The
+  // block barrier orders this block's index, weight and bit writes before
+  // thread 0's ticket, whose release makes them visible GPU-wide; the last
+  // block's ticket acquires every other block's writes.
   __shared__ int s_last;
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(grp.ticket, 1) == T - 1;
+  if (threadIdx.x == 0) s_last = ptx::atom_add_acq_rel_gpu(grp.ticket, 1) == T - 1;
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   extern __shared__ int grp_smem[];
-  permute_block(idx, T, E, k, grp.counts, grp.offsets, grp.perm, grp.inv, status, grp.touched,
-                grp_smem);
+  group_from_masks(idx, T, E, k, grp.mask, grp.counts, grp.offsets, grp.perm, grp.inv, status,
+                   grp.touched, grp_smem);
   if (grp.zero)
     for (int i = threadIdx.x; i < grp.nzero; i += blockDim.x) grp.zero[i] = 0;
   if (threadIdx.x == 0) *grp.ticket = 0;  // ready for the next call
@@ -515,13 +580,53 @@ cudaError_t launch_route_grouped(const float* logits, const float* bias, int T, 
 // chains); beyond that a warp per token.
 constexpr int kRouteBlockPerTokenMaxT = 1024;
 
+// One route_kernel<EPL> launch (EPL = ceil(E / 32) rounded up to a power of
+// two, EPL * 32 threads); `grouped`: with the grouping tail and its shared
+// memory.
+template <int EPL>
+cudaError_t launch_route_block(const float* src, int nsplit, const float* bias, int T, int E,
+                               int k, float scale, int32_t* idx, float* w, int* status,
+                               const RouteGrouping& grp, bool grouped, cudaStream_t st) {
+  size_t smem = 0;
+  if (grouped) {
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_dev != dev) {
+      e = cudaFuncSetAttribute(route_kernel<EPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)permute_block_smem(1024));
+      if (e != cudaSuccess) return e;
+      configured_dev = dev;
+    }
+    smem = permute_block_smem(E);
+  }
+  return launch_pdl(route_kernel<EPL>, dim3(T), dim3(32 * EPL), smem, st, src, nsplit, bias, T, E,
+                    k, scale, idx, w, status, grouped ? grp : RouteGrouping{});
+}
+
+cudaError_t launch_route_block_any(const float* src, int nsplit, const float* bias, int T, int E,
+                                   int k, float scale, int32_t* idx, float* w, int* status,
+                                   const RouteGrouping& grp, bool grouped, cudaStream_t st) {
+  const int epl = (E + 31) / 32;
+  if (epl <= 1)
+    return launch_route_block<1>(src, nsplit, bias, T, E, k, scale, idx, w, status, grp, grouped, st);
+  if (epl <= 2)
+    return launch_route_block<2>(src, nsplit, bias, T, E, k, scale, idx, w, status, grp, grouped, st);
+  if (epl <= 4)
+    return launch_route_block<4>(src, nsplit, bias, T, E, k, scale, idx, w, status, grp, grouped, st);
+  if (epl <= 8)
+    return launch_route_block<8>(src, nsplit, bias, T, E, k, scale, idx, w, status, grp, grouped, st);
+  if (epl <= 16)
+    return launch_route_block<16>(src, nsplit, bias, T, E, k, scale, idx, w, status, grp, grouped, st);
+  return launch_route_block<32>(src, nsplit, bias, T, E, k, scale, idx, w, status, grp, grouped, st);
+}
+
 cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T, int E, int k,
                          float scale, int32_t* idx, float* w, int* status, cudaStream_t st) {
-  if (T <= kRouteBlockPerTokenMaxT) {
-    const int threads = (E + 31) / 32 * 32;
-    return launch_pdl(route_kernel, dim3(T), dim3(threads), 0, st, src, nsplit, bias, T, E, k,
-                      scale, idx, w, status, RouteGrouping{});
-  }
+  if (T <= kRouteBlockPerTokenMaxT)
+    return launch_route_block_any(src, nsplit, bias, T, E, k, scale, idx, w, status,
+                                  RouteGrouping{}, false, st);
   const int epl = (E + 31) / 32;
   if (epl <= 1) return launch_route_warp<1>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
   if (epl <= 2) return launch_route_warp<2>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
@@ -534,20 +639,8 @@ cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T,
 cudaError_t launch_route_and_group(const float* src, int nsplit, const float* bias, int T, int E,
                                    int k, float scale, int32_t* idx, float* w, int* status,
                                    const RouteGrouping& grp, cudaStream_t st) {
-  if (T > kPermBlockTokens || !grp.ticket) return cudaErrorInvalidValue;
-  static int configured_dev = -1;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (configured_dev != dev) {
-    e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)permute_block_smem(1024));
-    if (e != cudaSuccess) return e;
-    configured_dev = dev;
-  }
-  const int threads = (E + 31) / 32 * 32;
-  return launch_pdl(route_kernel, dim3(T), dim3(threads), permute_block_smem(E), st, src, nsplit,
-                    bias, T, E, k, scale, idx, w, status, grp);
+  if (T > kPermBlockTokens || !grp.ticket || !grp.mask) return cudaErrorInvalidValue;
+  return launch_route_block_any(src, nsplit, bias, T, E, k, scale, idx, w, status, grp, true, st);
 }
 
 }  // namespace moe

@@ -34,6 +34,18 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// Arrives on `bar` once this thread's earlier shared-memory reads are done.
+// The arrival alone does not keep a preceding shared load from being
+// performed after it: a load of a ring stage could then return what the
+// producer wrote into the stage after seeing the arrival.  The CTA-scope
+// fence ahead of it orders every earlier access of this thread.
+__device__ __forceinline__ void mbar_arrive_after_reads(uint64_t* bar) {
+  asm volatile(
+      "fence.acq_rel.cta;\n\t"
+      "mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
                "r"(bytes)
@@ -216,10 +228,26 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Makes this thread's generic-proxy writes to shared memory visible to the
+// async proxy (the tensor core reading an MMA operand).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Orders this thread's generic-proxy global accesses with async-proxy (TMA)
 // accesses to global memory.
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
