@@ -175,9 +175,10 @@ bool ws_layout(const moe_dims_t& d, WsLayout* L) {
   L->perm = take(T * k * 4);
   L->inv = take(T * k * 4);
   L->blk_base = take(nblk * E * 4);
-  L->counters = take((E + S + 1) * 4);   // per-group counters + the tile claim counter
-  L->counters_s = take((S + 3) * 4);     // the same for a shared-experts-only launch, + its exit
-                                         // ticket and its "rows stored" flag
+  L->counters = take((E + S + 2) * 4);   // per-group counters, the tile claim counter and
+                                         // the exit ticket of a launch that zeroes them itself
+  L->counters_s = take((S + 2) * 4);     // the same for a shared-experts-only launch, + its exit
+                                         // ticket
   L->xperm = take(T * k * D * 2);
   L->act_r = take(T * k * F * 2);
   L->act_s = take(S * T * Fs * 2);
@@ -404,7 +405,6 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
     FfnArgs as = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
     as.part = kFfnShared;
     as.counters_s = counters_s;
-    if (!wt.fp8) as.shared_done = counters_s + dims->S + 2;
     as.max_ctas = kSharedCtas;
     const char* swhy = "launch failed";
     e = launch_ffn(as, wt, side->s, &n, &swhy, nullptr);
@@ -422,14 +422,23 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
   if (e != cudaSuccess) return cuda_fail(e, rwhy);
   // Batches of at most 128 tokens with bf16 weights: the routed gate/up tiles
   // read the token matrix itself (one row tile holds the whole batch), so no
-  // gathered copy is made; the routing kernel's grouping zeroes the FFN's
-  // counters instead of the gather kernel.
+  // gathered copy is made.  No grouping pass runs either: the routing kernel
+  // only sets each token's bit in the rows of its experts, and the FFN
+  // derives the group offsets (and writes counts, offsets and inv) from
+  // them; its last CTA zeroes its counters and the merge clears the bits.
   const bool dense = !wt.fp8 && T <= kDenseMaxT;
-  if (T <= kPermBlockTokens) {
+  uint32_t* gmask = w.at<uint32_t>(w.L.gmask);
+  if (dense) {
+    e = launch_route_bits(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw, w.status(),
+                          gmask, st);
+    if (e == cudaSuccess) e = mark(2, st);
+    if (e == cudaSuccess) e = mark(3, st);
+    if (e != cudaSuccess) return cuda_fail(e, "route launch");
+    n += 1;
+  } else if (T <= kPermBlockTokens) {
     // small batches: the routing kernel's last block also groups the pairs
     const RouteGrouping grp{counts, offsets, perm, inv, w.at<int32_t>(w.L.touched),
-                            w.at<int>(w.L.ticket), dense ? counters : nullptr,
-                            E + dims->S + 1, w.at<uint32_t>(w.L.gmask)};
+                            w.at<int>(w.L.ticket), nullptr, 0, gmask};
     e = launch_route_and_group(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw,
                                w.status(), grp, st);
     if (e == cudaSuccess) e = mark(2, st);
@@ -453,37 +462,37 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
   if (e == cudaSuccess) e = mark(4, st);
   if (e != cudaSuccess) return cuda_fail(e, "gather launch");
   FfnArgs a = ffn_args(hb, xperm, offsets, wt, w, y, counters, dims);
-  if (overlap_shared) {
-    a.part = kFfnRouted;
-    if (!wt.fp8) a.shared_done = w.at<int32_t>(w.L.counters_s) + dims->S + 2;
-  }
+  if (overlap_shared) a.part = kFfnRouted;
   if (dense) {
     a.dense_a = 1;
     a.idx = idx;
     a.inv = inv;
+    a.mask = gmask;
+    a.mask_stride = kPermBlockTokens / 32;
+    a.counts_out = counts;
+    a.offsets_out = offsets;
+    a.touched_out = w.at<int32_t>(w.L.touched);
+    a.inv_out = inv;
+    a.self_reset = 1;
   }
   const char* why = "launch failed";
   e = launch_ffn(a, wt, st, &n, &why, g_prof_events ? g_prof_events + 5 : nullptr);
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "expert ffn: %s (%s)", why, cudaGetErrorString(e));
-  // With the flag hand-off the routed launch completes only after the shared
-  // rows are stored, so the merge follows it directly (its launch overlaps the
-  // FFN's tail) and the streams are joined after it; otherwise the join comes
-  // first.
-  const bool flag_join = overlap_shared && a.shared_done;
-  if (overlap_shared && !flag_join) {
+  // The merge reads the shared experts' rows: the streams are joined first.
+  // (A device-side hand-off from the shared launch to the routed one would
+  // let the merge launch behind the routed FFN, but a kernel that waits for
+  // a kernel of another stream can wait for one that never becomes
+  // resident.)
+  if (overlap_shared) {
     guard.join = nullptr;
     e = cudaStreamWaitEvent(st, side->join, 0);
     if (e != cudaSuccess) return cuda_fail(e, "shared-expert stream");
   }
-  e = launch_combine(y, rw, inv, T, D, k, dims->S, out, w.status(), st);
+  e = launch_combine(y, rw, inv, T, D, k, dims->S, out, w.status(), dense ? idx : nullptr,
+                     dense ? gmask : nullptr, kPermBlockTokens / 32, st);
   if (e == cudaSuccess) e = mark(6, st);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   n += 1;
-  if (flag_join) {
-    guard.join = nullptr;
-    e = cudaStreamWaitEvent(st, side->join, 0);
-    if (e != cudaSuccess) return cuda_fail(e, "shared-expert stream");
-  }
   g_launches = n;
   return MOE_OK;
 }
@@ -747,7 +756,7 @@ int moe_combine(const float* y, const float* w, const int32_t* inv, const moe_di
   int* status = ws ? reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status) : nullptr;
   if ((rc = check_device())) return rc;
   cudaError_t e = launch_combine(y, w, inv, dims->T, dims->D, dims->k, dims->S,
-                                 out, status,
+                                 out, status, nullptr, nullptr, 0,
                                  reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   g_launches = 1;

@@ -19,9 +19,16 @@ constexpr int kMaxK = 32;
 // per thread, the k + S row loads issued together.
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const float* __restrict__ y, const float* __restrict__ w, const int32_t* __restrict__ inv,
-    int T, int D, int k, int S, float* __restrict__ out, int* __restrict__ status) {
+    int T, int D, int k, int S, float* __restrict__ out, int* __restrict__ status,
+    const int32_t* __restrict__ idx, uint32_t* __restrict__ mask, int mask_stride) {
   ptx::pdl_launch_dependents();
   ptx::pdl_wait();
+  if (mask && blockIdx.y == 0 && threadIdx.x < k) {
+    // this token's bit in the row of each expert it chose (set by the routing)
+    const int t = blockIdx.x;
+    const int e = idx[(size_t)t * k + threadIdx.x];
+    if (e >= 0) atomicAnd(mask + (size_t)e * mask_stride + (t >> 5), ~(1u << (t & 31)));
+  }
   __shared__ int s_row[kMaxK];
   __shared__ float s_w[kMaxK];
   const int t = blockIdx.x;
@@ -73,11 +80,12 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
 }
 
 cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, int T, int D,
-                           int k, int S, float* out, int* status, cudaStream_t st) {
+                           int k, int S, float* out, int* status, const int32_t* idx,
+                           uint32_t* mask, int mask_stride, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const dim3 grid(T, (D / 4 + kCombineThreads - 1) / kCombineThreads);
   return launch_pdl(combine_kernel, grid, dim3(kCombineThreads), 0, st, y, w, inv, T, D, k, S, out,
-                    status);
+                    status, idx, mask, mask_stride);
 }
 
 }  // namespace moe

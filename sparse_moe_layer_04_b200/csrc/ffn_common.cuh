@@ -70,13 +70,19 @@ struct GemmParams {
   int k;
   const int32_t* idx;        // [T, k] (dense_a)
   const int32_t* inv;        // [T, k] (dense_a)
-  // Shared experts on an internal stream beside a routed-only launch: the
-  // shared launch's last CTA sets *done_flag once all its rows are stored;
-  // CTA 0 of the routed launch waits for *wait_flag (the same word) before it
-  // exits and clears it, so whatever follows the routed launch on its stream
-  // also sees the shared rows.  nullptr: no such hand-off.
-  int* done_flag;
-  int* wait_flag;
+  // Batches of at most 128 tokens routed without a grouping pass: `mask`
+  // [E][mask_stride] holds bit t of row e when token t chose expert e (rows
+  // of ceil(T / 32) words).  The group row offsets are then those of the
+  // pairs in (expert, token) order: each CTA derives them from the bit
+  // counts, CTA 0 also stores counts [E], offsets [E + 1] and the number of
+  // experts with pairs (touched), and the gate/up epilogue writes inv for
+  // the pairs it places.  nullptr: offsets come from `offsets`.
+  const uint32_t* mask;
+  int mask_stride;
+  int32_t* counts_out;
+  int32_t* offsets_out;
+  int32_t* touched_out;
+  int32_t* inv_out;
 };
 
 // Row blocks of the routed groups, built on the device from the group
@@ -101,31 +107,92 @@ struct TileInfo {
 
 __device__ __forceinline__ int col_tiles(int N, int bn) { return (N + bn - 1) / bn; }
 
-// One warp reads the group offsets 32 experts at a time, checks them and
-// writes the row-tile prefix; inconsistent offsets give an empty routed tile
-// space and raise kStBounds.
+// Token-bit mode (GemmParams::mask): rows of at most kMaskWords words (T <=
+// 128), read kMaskBatch chunks of 32 experts at a time.
+constexpr int kMaskWords = 4;
+constexpr int kMaskBatch = 8;
+
+// One warp reads the group offsets (or counts the token bits) 32 experts at
+// a time, checks them and writes the row-tile prefix; inconsistent offsets
+// give an empty routed tile space and raise kStBounds.
 template <int BR = BM>
 __device__ __forceinline__ void build_tile_map(TileMap& tm, const GemmParams& p, int lane) {
   int carry = 0;
   bool bad = false;
-  for (int base = 0; base < p.E; base += 32) {
-    const int e = base + lane;
-    int cnt = 0;
-    if (e < p.E) {
-      const int a = p.offsets[e], b = p.offsets[e + 1];
-      tm.off[e] = a;
-      if (e == p.E - 1) tm.off[p.E] = b;
-      if (a < 0 || b < a || b > p.rows_r || (e == 0 && a != 0)) bad = true;
-      cnt = b >= a ? (b - a + BR - 1) / BR : 0;
-    }
-    int incl = cnt;
+  if (p.mask) {
+    // token bits (T <= 128: at most kMaskWords words per expert row): the
+    // rows of kMaskBatch chunks of 32 experts are loaded together, then
+    // scanned chunk by chunk
+    int row_carry = 0, touched = 0;
+    const int words = (p.T + 31) >> 5;
+    const bool store = blockIdx.x == 0;
+    for (int base0 = 0; base0 < p.E; base0 += 32 * kMaskBatch) {
+      uint32_t m[kMaskBatch][kMaskWords];
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
+      for (int c = 0; c < kMaskBatch; ++c) {
+        const int e = base0 + 32 * c + lane;
+#pragma unroll
+        for (int q = 0; q < kMaskWords; ++q)
+          m[c][q] = (e < p.E && q < words) ? p.mask[(size_t)e * p.mask_stride + q] : 0u;
+      }
+#pragma unroll
+      for (int c = 0; c < kMaskBatch; ++c) {
+        const int e = base0 + 32 * c + lane;
+        int rows = 0;
+#pragma unroll
+        for (int q = 0; q < kMaskWords; ++q) rows += __popc(m[c][q]);
+        int rincl = rows, cnt = (rows + BR - 1) / BR, incl = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, rincl, off);
+          const int u = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) {
+            rincl += v;
+            incl += u;
+          }
+        }
+        if (e < p.E) {
+          const int a = row_carry + rincl - rows;
+          tm.off[e] = a;
+          tm.mt_prefix[e] = carry + incl - cnt;
+          if (store) {
+            p.counts_out[e] = rows;
+            p.offsets_out[e] = a;
+          }
+        }
+        row_carry += __shfl_sync(0xffffffffu, rincl, 31);
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+        touched += __popc(__ballot_sync(0xffffffffu, rows > 0));
+      }
     }
-    if (e < p.E) tm.mt_prefix[e] = carry + incl - cnt;
-    carry += __shfl_sync(0xffffffffu, incl, 31);
+    if (lane == 0) {
+      tm.off[p.E] = row_carry;
+      bad = row_carry != p.rows_r;   // every token has k distinct experts
+      if (store) {
+        p.offsets_out[p.E] = row_carry;
+        *p.touched_out = touched;
+      }
+    }
+  } else {
+    for (int base = 0; base < p.E; base += 32) {
+      const int e = base + lane;
+      int cnt = 0;
+      if (e < p.E) {
+        const int a = p.offsets[e], b = p.offsets[e + 1];
+        tm.off[e] = a;
+        if (e == p.E - 1) tm.off[p.E] = b;
+        if (a < 0 || b < a || b > p.rows_r || (e == 0 && a != 0)) bad = true;
+        cnt = b >= a ? (b - a + BR - 1) / BR : 0;
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      if (e < p.E) tm.mt_prefix[e] = carry + incl - cnt;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
   }
   bad = __any_sync(0xffffffffu, bad);
   if (lane == 0) {
@@ -227,20 +294,28 @@ __device__ __forceinline__ void reset_counters_at_exit(const GemmParams& p) {
     *p.sched = 0;
     *p.exit_ticket = 0;
     __threadfence();
-    if (p.done_flag) ptx::st_release_gpu(p.done_flag, 1);
   }
 }
 
-// CTA 0 of a routed-only launch: waits (bounded) until the shared launch on
-// the internal stream has stored all its rows, then clears the flag for the
-// next call.  Only this one CTA waits, once its own tiles are done; the other
-// CTAs exit and leave their SMs to the shared launch if it is still running.
-// Returns false if the wait gave up.
-__device__ __forceinline__ bool wait_shared_at_exit(const GemmParams& p, volatile int* abort) {
-  if (!p.wait_flag || blockIdx.x != 0) return true;
-  if (!ptx::counter_wait(p.wait_flag, 1, abort)) return false;
-  *p.wait_flag = 0;
-  return true;
+// The same at block scope, called by every thread of the CTA after its final
+// barrier (`s_last`: a shared int): thread 0 takes the ticket, and all
+// threads of the last CTA zero the counters.
+__device__ __forceinline__ void reset_counters_at_exit_block(const GemmParams& p, int* s_last) {
+  if (!p.exit_ticket) return;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    *s_last = atomicAdd(p.exit_ticket, 1) == (int)gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!*s_last) return;
+  __threadfence();
+  for (int i = threadIdx.x; i < p.nreset; i += blockDim.x) p.counters[i] = 0;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    *p.sched = 0;
+    *p.exit_ticket = 0;
+    __threadfence();
+  }
 }
 
 // Queue of claimed tiles from the producer to the other roles of the CTA.

@@ -70,6 +70,8 @@ namespace {
 using namespace ffn;
 
 constexpr int THREADS = 256;             // warps 0-7
+static_assert(kDenseMaxT <= 32 * kMaskWords, "token-bit rows of a dense batch");
+
 constexpr int MMA_WARP1 = 6;             // second MMA issuer (N = 128)
 constexpr int BPROD_WARP = 7;            // weight producer and tile claimer
 constexpr int RING_BYTES = 192 * 1024;   // budget of the two operand rings
@@ -119,6 +121,7 @@ struct SharedState {
   uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
+  int last;        // this CTA took the last exit ticket
   TileMap tm;
 };
 
@@ -415,7 +418,18 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           }
           if (hit >= 0) {
             row_ok = true;
-            out_row = (size_t)__ldcg(p.inv + (size_t)r * p.k + hit);
+            if (p.mask) {
+              // the pair's row: the group's offset plus the tokens below r
+              // that chose the same expert; column tile 0 records it in inv
+              const uint32_t* m = p.mask + (size_t)ti.grp * p.mask_stride;
+              const int word = r >> 5;
+              int rank = __popc(__ldg(m + word) & ((1u << (r & 31)) - 1u));
+              for (int w = 0; w < word; ++w) rank += __popc(__ldg(m + w));
+              out_row = (size_t)ss.tm.off[ti.grp] + rank;
+              if (ti.n0 == 0) p.inv_out[(size_t)r * p.k + hit] = (int32_t)out_row;
+            } else {
+              out_row = (size_t)__ldcg(p.inv + (size_t)r * p.k + hit);
+            }
           }
         }
       }
@@ -434,11 +448,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, TMEM_COLS);
   }
-  if (threadIdx.x == 0) {
-    wait_shared_at_exit(p, &ss.abort);
-    if (ss.abort && p.status) atomicOr(p.status, kStTimeout);
-    reset_counters_at_exit(p);
-  }
+  if (threadIdx.x == 0 && ss.abort && p.status) atomicOr(p.status, kStTimeout);
+  reset_counters_at_exit_block(p, &ss.last);
 }
 
 // ---------------------------------------------------------------------------
@@ -645,9 +656,19 @@ cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t st, int* nlaunch, c
     p.sched = a.counters_s + a.S;
     p.exit_ticket = a.counters_s + a.S + 1;
     p.nreset = a.S;
-    p.done_flag = a.shared_done;
   }
-  if (a.part == kFfnRouted) p.wait_flag = a.shared_done;
+  if (a.mask) {
+    p.mask = a.mask;
+    p.mask_stride = a.mask_stride;
+    p.counts_out = a.counts_out;
+    p.offsets_out = a.offsets_out;
+    p.touched_out = a.touched_out;
+    p.inv_out = a.inv_out;
+  }
+  if (a.self_reset && a.part != kFfnShared) {
+    p.exit_ticket = a.counters + a.E + a.S + 1;
+    p.nreset = a.E + a.S;
+  }
   const int tiles_g = mt_r * ((a.F + half - 1) / half) + S * mt_s * ((a.Fs + half - 1) / half);
   const int nt_d = (a.D + nmma - 1) / nmma;
   const int tiles_d = mt_r * nt_d + S * mt_s * nt_d;

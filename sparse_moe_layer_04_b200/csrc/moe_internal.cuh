@@ -108,6 +108,11 @@ struct RouteGrouping {
   // each token's block sets its bits, the last block reads and clears them
   uint32_t* mask;
 };
+// Routing that also sets token t's bit in row idx[t, j] of `mask`
+// [E][kPermBlockTokens / 32] (zero on entry) for every slot j; T <= kPermBlockTokens.
+cudaError_t launch_route_bits(const float* src, int nsplit, const float* bias, int T, int E,
+                              int k, float scale, int32_t* idx, float* w, int* status,
+                              uint32_t* mask, cudaStream_t st);
 // Routing and grouping in one launch; T <= kPermBlockTokens.
 cudaError_t launch_route_and_group(const float* src, int nsplit, const float* bias, int T, int E,
                                    int k, float scale, int32_t* idx, float* w, int* status,
@@ -123,8 +128,11 @@ cudaError_t launch_permute(const int32_t* idx, int T, int E, int k, int32_t* cou
 // (`ncounters` ints).
 cudaError_t launch_gather_rows(const uint16_t* h, const int32_t* perm, int rows, int D, int T,
                                uint16_t* xperm, int* counters, int ncounters, cudaStream_t st);
+// With `mask` set, the blocks of column chunk 0 also clear every token's bits
+// in the rows [E][mask_stride] of the experts idx names (the routing set them).
 cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, int T, int D,
-                           int k, int S, float* out, int* status, cudaStream_t st);
+                           int k, int S, float* out, int* status, const int32_t* idx,
+                           uint32_t* mask, int mask_stride, cudaStream_t st);
 
 // Expert MLPs: gate/up GEMM with the SiLU gate fused, then the down GEMM.
 struct FfnArgs {
@@ -145,10 +153,16 @@ struct FfnArgs {
   int part = 0;
   int* counters_s = nullptr;
   int max_ctas = 0;
-  // bf16 kernel, shared and routed parts on two streams: the word the shared
-  // part sets when its rows are stored and the routed part waits for before
-  // it completes (nullptr: the streams are joined by an event instead).
-  int* shared_done = nullptr;
+  // dense_a batches routed without a grouping pass (GemmParams::mask)
+  const uint32_t* mask = nullptr;
+  int mask_stride = 0;
+  int32_t* counts_out = nullptr;
+  int32_t* offsets_out = nullptr;
+  int32_t* touched_out = nullptr;
+  int32_t* inv_out = nullptr;
+  // 1: the launch's last CTA zeroes `counters` (E + S group counters, the
+  // claim counter and the exit ticket at [E + S + 1]) itself
+  int self_reset = 0;
   // T <= kDenseMaxT with bf16 weights: the routed gate/up A operand is h
   // itself (xperm is not used) and rows are placed by idx / inv [T, k].
   int dense_a = 0;

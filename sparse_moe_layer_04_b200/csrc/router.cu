@@ -601,8 +601,12 @@ cudaError_t launch_route_block(const float* src, int nsplit, const float* bias, 
     }
     smem = permute_block_smem(E);
   }
+  // without the grouping tail only the bitmask rows (if any) are passed on
+  RouteGrouping g{};
+  if (grouped) g = grp;
+  else g.mask = grp.mask;
   return launch_pdl(route_kernel<EPL>, dim3(T), dim3(32 * EPL), smem, st, src, nsplit, bias, T, E,
-                    k, scale, idx, w, status, grouped ? grp : RouteGrouping{});
+                    k, scale, idx, w, status, g);
 }
 
 cudaError_t launch_route_block_any(const float* src, int nsplit, const float* bias, int T, int E,
@@ -634,6 +638,15 @@ cudaError_t launch_route(const float* src, int nsplit, const float* bias, int T,
   if (epl <= 8) return launch_route_warp<8>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
   if (epl <= 16) return launch_route_warp<16>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
   return launch_route_warp<32>(src, nsplit, bias, T, E, k, scale, idx, w, status, st);
+}
+
+cudaError_t launch_route_bits(const float* src, int nsplit, const float* bias, int T, int E,
+                              int k, float scale, int32_t* idx, float* w, int* status,
+                              uint32_t* mask, cudaStream_t st) {
+  if (T > kPermBlockTokens || !mask) return cudaErrorInvalidValue;
+  RouteGrouping grp{};
+  grp.mask = mask;
+  return launch_route_block_any(src, nsplit, bias, T, E, k, scale, idx, w, status, grp, false, st);
 }
 
 cudaError_t launch_route_and_group(const float* src, int nsplit, const float* bias, int T, int E,
