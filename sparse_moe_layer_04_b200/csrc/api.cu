@@ -334,7 +334,12 @@ cudaError_t side_stream(SideStream** out) {
   if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
   SideStream& r = per_dev[dev];
   if (!r.s) {
-    e = cudaStreamCreateWithFlags(&r.s, cudaStreamNonBlocking);
+    // The highest priority: when the shared launch and the routing kernels
+    // become ready together, the block scheduler places the shared CTAs
+    // first, so the routed FFN launched behind them cannot take their SMs.
+    int lo = 0, hi = 0;
+    e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&r.s, cudaStreamNonBlocking, hi);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming);
     if (e != cudaSuccess) {
