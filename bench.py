@@ -475,7 +475,9 @@ def config_inputs(moe, cfg, rank: int, dev, cache: dict, fp8_mode: bool):
     """Device inputs of a workload: the weights of its family (generated once
     per family and shared, with their FP8 codes in FP8 mode), its bias and its
     hidden states (seeded by rank)."""
-    fam = cfg.weight_family
+    # weights are shared by the workloads of one family and one shape only (a
+    # run with --experts / --tokens has its own)
+    fam = (cfg.weight_family, cfg.E, cfg.D, cfg.F, cfg.S, cfg.Fs)
     if fam not in cache:
         w = mi.layer_weights(cfg, 0, device=dev)
         w8 = None
