@@ -15,8 +15,13 @@ namespace moe {
 constexpr int kCombineThreads = 256;
 constexpr int kMaxK = 32;
 
-// Block (t, c) merges columns [c*1024, c*1024 + 1024) of token t; one float4
-// per thread, the k + S row loads issued together.
+// Block (t, c) merges columns [c * 2048, c * 2048 + 2048) of token t: each
+// thread takes the float4 at column group v and then the one at v + 256, with
+// the k + S row loads of each issued together.  Two column groups per thread
+// keep the whole grid resident in one wave (at one group per thread the
+// registers of a decode batch's 768 blocks need two).
+constexpr int kCombineGroups = 2;
+
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const float* __restrict__ y, const float* __restrict__ w, const int32_t* __restrict__ inv,
     int T, int D, int k, int S, float* __restrict__ out, int* __restrict__ status,
@@ -43,47 +48,51 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     s_w[threadIdx.x] = w[(size_t)t * k + threadIdx.x];
   }
   __syncthreads();
-  const int v = blockIdx.y * kCombineThreads + threadIdx.x;
-  if (v >= D / 4) return;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  // the first shared row is loaded with the first batch of routed rows, so a
-  // layer with one shared expert and k <= 8 reads all its rows in one round
-  float4 sh0 = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (S > 0) sh0 = reinterpret_cast<const float4*>(y + (rows_r + t) * D)[v];
-  for (int j0 = 0; j0 < k; j0 += 8) {
-    float4 a[8];
+#pragma unroll 1
+  for (int g = 0; g < kCombineGroups; ++g) {
+    const int v = (blockIdx.y * kCombineGroups + g) * kCombineThreads + threadIdx.x;
+    if (v >= D / 4) break;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // the first shared row is loaded with the first batch of routed rows, so a
+    // layer with one shared expert and k <= 8 reads all its rows in one round
+    float4 sh0 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (S > 0) sh0 = reinterpret_cast<const float4*>(y + (rows_r + t) * D)[v];
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      float4 a[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int r = (j0 + q < k) ? s_row[j0 + q] : -1;
-      a[q] = r >= 0 ? reinterpret_cast<const float4*>(y + (size_t)r * D)[v]
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    if (j0 == 0) {
-      // shared experts first, in order
-      acc.x += sh0.x; acc.y += sh0.y; acc.z += sh0.z; acc.w += sh0.w;
-      for (int s = 1; s < S; ++s) {
-        const float4 b = reinterpret_cast<const float4*>(y + (rows_r + (size_t)s * T + t) * D)[v];
-        acc.x += b.x; acc.y += b.y; acc.z += b.z; acc.w += b.w;
+      for (int q = 0; q < 8; ++q) {
+        const int r = (j0 + q < k) ? s_row[j0 + q] : -1;
+        a[q] = r >= 0 ? reinterpret_cast<const float4*>(y + (size_t)r * D)[v]
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      if (j0 == 0) {
+        // shared experts first, in order
+        acc.x += sh0.x; acc.y += sh0.y; acc.z += sh0.z; acc.w += sh0.w;
+        for (int s = 1; s < S; ++s) {
+          const float4 b = reinterpret_cast<const float4*>(y + (rows_r + (size_t)s * T + t) * D)[v];
+          acc.x += b.x; acc.y += b.y; acc.z += b.z; acc.w += b.w;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (j0 + q >= k || s_row[j0 + q] < 0) continue;
+        const float wj = s_w[j0 + q];
+        acc.x = fmaf(wj, a[q].x, acc.x);
+        acc.y = fmaf(wj, a[q].y, acc.y);
+        acc.z = fmaf(wj, a[q].z, acc.z);
+        acc.w = fmaf(wj, a[q].w, acc.w);
       }
     }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (j0 + q >= k || s_row[j0 + q] < 0) continue;
-      const float wj = s_w[j0 + q];
-      acc.x = fmaf(wj, a[q].x, acc.x);
-      acc.y = fmaf(wj, a[q].y, acc.y);
-      acc.z = fmaf(wj, a[q].z, acc.z);
-      acc.w = fmaf(wj, a[q].w, acc.w);
-    }
+    reinterpret_cast<float4*>(out + (size_t)t * D)[v] = acc;
   }
-  reinterpret_cast<float4*>(out + (size_t)t * D)[v] = acc;
 }
 
 cudaError_t launch_combine(const float* y, const float* w, const int32_t* inv, int T, int D,
                            int k, int S, float* out, int* status, const int32_t* idx,
                            uint32_t* mask, int mask_stride, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  const dim3 grid(T, (D / 4 + kCombineThreads - 1) / kCombineThreads);
+  const int per_block = kCombineThreads * kCombineGroups;   // float4 column groups
+  const dim3 grid(T, (D / 4 + per_block - 1) / per_block);
   return launch_pdl(combine_kernel, grid, dim3(kCombineThreads), 0, st, y, w, inv, T, D, k, S, out,
                     status, idx, mask, mask_stride);
 }
