@@ -443,7 +443,7 @@ int forward_impl(const void* h, const float* Wr, const float* bias, const Expert
   } else if (T <= kPermBlockTokens) {
     // small batches: the routing kernel's last block also groups the pairs
     const RouteGrouping grp{counts, offsets, perm, inv, w.at<int32_t>(w.L.touched),
-                            w.at<int>(w.L.ticket), nullptr, 0, gmask};
+                            w.at<int>(w.L.ticket), gmask};
     e = launch_route_and_group(partials, sp.nsplit, bias, T, E, k, dims->scale, idx, rw,
                                w.status(), grp, st);
     if (e == cudaSuccess) e = mark(2, st);

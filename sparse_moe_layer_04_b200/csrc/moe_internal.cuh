@@ -102,8 +102,6 @@ struct RouteGrouping {
   int32_t* inv;
   int32_t* touched;
   int* ticket;  // nullptr: no grouping
-  int* zero;    // nullable: `nzero` ints the last block also sets to zero (the
-  int nzero;    // expert FFN's counters, when no row-gather kernel runs)
   // [E][kPermBlockTokens / 32] token bitmask per expert, zero between calls:
   // each token's block sets its bits, the last block reads and clears them
   uint32_t* mask;

@@ -418,8 +418,6 @@ __global__ void __launch_bounds__(1024) route_kernel(
   extern __shared__ int grp_smem[];
   group_from_masks(idx, T, E, k, grp.mask, grp.counts, grp.offsets, grp.perm, grp.inv, status,
                    grp.touched, grp_smem);
-  if (grp.zero)
-    for (int i = threadIdx.x; i < grp.nzero; i += blockDim.x) grp.zero[i] = 0;
   if (threadIdx.x == 0) *grp.ticket = 0;  // ready for the next call
 }
 
