@@ -142,16 +142,18 @@ cudaError_t launch_router(const uint16_t* h, const float* Wr, const moe_dims_t& 
 }  // namespace
 
 int num_sms() {
-  static int cache[kMaxDev] = {0};
+  // per-device cache; threads racing on the first call store the same value
+  static std::atomic<int> cache[kMaxDev];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= kMaxDev) return 148;
-  if (!cache[dev]) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (!n) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 148;
+    if (n <= 0) n = 148;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 bool ws_layout(const moe_dims_t& d, WsLayout* L) {

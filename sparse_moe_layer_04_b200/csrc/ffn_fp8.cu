@@ -571,16 +571,9 @@ static_assert(smem_bytes8<128>() > 114 * 1024, "one CTA per SM");
 
 template <int NT>
 cudaError_t launch_one8(const GemmParams& p, int tiles_upper, cudaStream_t st, int max_ctas) {
-  static int configured_dev = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(ffn_fp8_kernel<NT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_bytes8<NT>());
-    if (e != cudaSuccess) return e;
-    configured_dev = dev;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = set_smem_once(ffn_fp8_kernel<NT>, (int)smem_bytes8<NT>(), smem_set);
+  if (e != cudaSuccess) return e;
   int grid = num_sms();
   if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
   if (tiles_upper < grid) grid = tiles_upper;

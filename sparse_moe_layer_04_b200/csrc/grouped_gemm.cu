@@ -469,16 +469,9 @@ static_assert(smem_bytes<256>() <= 227 * 1024 && smem_bytes<128>() <= 227 * 1024
 
 template <int MMA_N>
 cudaError_t launch_one(const GemmParams& p, int tiles_upper, cudaStream_t st, int max_ctas = 0) {
-  static int configured_dev = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MMA_N>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_bytes<MMA_N>());
-    if (e != cudaSuccess) return e;
-    configured_dev = dev;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = set_smem_once(grouped_gemm_kernel<MMA_N>, (int)smem_bytes<MMA_N>(), smem_set);
+  if (e != cudaSuccess) return e;
   int grid = num_sms();
   if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
   if (tiles_upper < grid) grid = tiles_upper;
@@ -495,15 +488,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  // looked up once (a function-local static is initialised once, thread-safely)
+  static const EncodeTiledFn fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+      return reinterpret_cast<EncodeTiledFn>(ptr);
+    return static_cast<EncodeTiledFn>(nullptr);
+  }();
   return fn;
 }
 

@@ -1,6 +1,8 @@
 // Internal declarations shared by the library's translation units.
 #pragma once
 
+#include <atomic>
+
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -60,6 +62,22 @@ struct WsLayout {
       act_r, act_s, y, touched, gmask, total;
 };
 bool ws_layout(const moe_dims_t& d, WsLayout* out);
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per device: `done` holds one bit per device ordinal (two host
+// threads that race on a device's first call both set the attribute, which
+// is harmless).
+template <typename Kernel>
+cudaError_t set_smem_once(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Launch with programmatic dependent launch allowed: the kernel may start
 // while the previous kernel in the stream finishes; every kernel of the

@@ -587,16 +587,9 @@ cudaError_t launch_route_block(const float* src, int nsplit, const float* bias, 
                                const RouteGrouping& grp, bool grouped, cudaStream_t st) {
   size_t smem = 0;
   if (grouped) {
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::atomic<uint64_t> smem_set{0};
+    const cudaError_t e = set_smem_once(route_kernel<EPL>, (int)permute_block_smem(1024), smem_set);
     if (e != cudaSuccess) return e;
-    if (configured_dev != dev) {
-      e = cudaFuncSetAttribute(route_kernel<EPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)permute_block_smem(1024));
-      if (e != cudaSuccess) return e;
-      configured_dev = dev;
-    }
     smem = permute_block_smem(E);
   }
   // without the grouping tail only the bitmask rows (if any) are passed on

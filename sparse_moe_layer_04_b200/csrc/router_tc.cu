@@ -265,16 +265,9 @@ cudaError_t launch_router_tc_fused(const uint16_t* h, const float* Wr, int T, in
   p.E = E;
   p.kb_total = D / kRtBK;
   p.kb_per = kb_per;
-  static int configured_dev = -1;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = set_smem_once(router_tc_kernel, (int)kRtSmem, smem_set);
   if (e != cudaSuccess) return e;
-  if (configured_dev != dev) {
-    e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kRtSmem);
-    if (e != cudaSuccess) return e;
-    configured_dev = dev;
-  }
   const dim3 grid(E / kRtN, nsplit, (T + kRtM - 1) / kRtM);
   return launch_pdl(router_tc_kernel, grid, dim3(kRtThreads), kRtSmem, st, p);
 }
