@@ -134,6 +134,14 @@ def workload_name(cfg) -> str:
             f"F={cfg.F} S={cfg.S} Fs={cfg.Fs} scale={cfg.scale}")
 
 
+def workload_config(cfg, n_gpus: int, fp8: bool) -> dict:
+    """The workload a line measures, the same in both arms' lines (the
+    measurement's own details go under "run")."""
+    return {"workload": workload_name(cfg), "T": cfg.T, "global_batch": n_gpus * cfg.T,
+            "weights": ("fp8 e4m3 codes + power-of-two 128x128 block exponents, decoded "
+                        "exactly to bf16" if fp8 else "bf16")}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -618,15 +626,13 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded counter-based generator; random-init weights of the layer's shapes)",
-        "config": {"workload": workload_name(cfg),
-                   "T": cfg.T, "touched_experts": U, "global_batch": world * cfg.T,
-                   "weights": ("fp8 e4m3 codes + power-of-two 128x128 block exponents, decoded "
-                               "exactly to bf16 in the kernel" if w8 is not None else "bf16"),
-                   "parallelism": f"replicas x{world} (token-parallel, no exchange)",
-                   "l2": "flushed: 256 MiB memset before every timed step, outside its events",
-                   "ms_p10_p90": [float(np.percentile(t["step_ms"], 10)),
-                                  float(np.percentile(t["step_ms"], 90))],
-                   "stage_ms": t["stage_ms"], "profiled_step_ms": t["profiled_ms"]},
+        "config": workload_config(cfg, world, w8 is not None),
+        "run": {"touched_experts": U,
+                "parallelism": f"replicas x{world} (token-parallel, no exchange)",
+                "l2": "flushed: 256 MiB memset before every timed step, outside its events",
+                "ms_p10_p90": [float(np.percentile(t["step_ms"], 10)),
+                               float(np.percentile(t["step_ms"], 90))],
+                "stage_ms": t["stage_ms"], "profiled_step_ms": t["profiled_ms"]},
         "roofline": roof,
         "layer_roofline": layer,
         "e2e": {"value": aggregate_tokens_per_s(cfg.T, world, e2e), "unit": "tokens/s",
@@ -729,8 +735,8 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded counter-based generator)",
-        "config": {"workload": workload_name(cfg), "T": cfg.T,
-                   "sample_tokens": n, "weights": args.weights},
+        "config": workload_config(cfg, args.gpus, args.weights == "fp8"),
+        "run": {"sample_tokens": n},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -738,7 +744,7 @@ def run_reference(args):
     }
     if n < cfg.T:
         # linear extrapolation of the sample's rate to the whole batch (marked)
-        res["config"]["full_batch_s_extrapolated"] = cfg.T / value
+        res["run"]["full_batch_s_extrapolated"] = cfg.T / value
     return res
 
 
