@@ -17,6 +17,7 @@ constexpr int BK = 64;                    // one 128-byte swizzle row of bf16
 constexpr int A_BYTES = BM * BK * 2;      // 16 KiB
 constexpr int MAX_E = 1024;
 constexpr int EPI_WARPS = 4;              // each releases its rows of a gate/up tile
+constexpr unsigned kWarpMask = 0xffffffffu;
 
 // One grouped GEMM.  Routed group e has rows [off[e], off[e+1]) of the routed
 // A / output matrices; shared group s has rows s*T .. s*T + T - 1 of the

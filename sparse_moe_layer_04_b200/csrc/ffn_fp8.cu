@@ -38,11 +38,12 @@
 //   warps 1,11  MMA issuers (warp 1 also allocates the 512 TMEM columns):
 //               tcgen05.mma.cta_group::1.kind::f16, M = 128, N <= NT, K = 16.
 //               The weights are bf16 in the MMA, so a stage of 8 KB of codes
-//               costs as many MMAs as 16 KB of bf16 weights, and one thread
-//               issues a tcgen05.mma only every ~100+ cycles at N <= 128: for
+//               costs as many MMAs as 16 KB of bf16 weights, and one warp
+//               issues a tcgen05.mma only every ~150 cycles whatever N: for
 //               NT = 128 two warps take alternate K-blocks into an accumulator
 //               each (the epilogue adds them); one commit per K-block frees
-//               both the token and the decoded-weight stage.
+//               both the token and the decoded-weight stage.  Each issuing
+//               warp walks its loop together and an elected lane issues.
 //   warps 2-5   epilogue (tcgen05.ld of the accumulators, SiLU gate or fp32
 //               store).
 //   warps 6-9,  decoders, two sets of four taking alternate stages: each
@@ -386,59 +387,63 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
   } else if (mma_index(warp) >= 0 && mma_index(warp) < MW) {
     // ---------------- MMA issuers ----------------
     // Issuer m takes the K-blocks kb with kb % MW == m of every tile into
-    // accumulator D_m; all issuers walk the same stage sequence.
+    // accumulator D_m; all issuers walk the same stage sequence.  The whole
+    // warp walks the loop, its waits decided by a warp vote, and an elected
+    // lane issues each tcgen05 operation (warp-uniform operands issue faster).
     const int m = mma_index(warp);
-    if (lane == 0) {
-      int st = 0;
-      uint32_t sph = 0, acc_phase = 0;
-      const uint32_t d_tmem = tmem_base + m * NT;
-      int qslot = 0;
-      uint32_t qphase = 0;
-      for (;;) {
-        if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
-        const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
-        ptx::mbar_arrive_after_reads(&ss.tq_empty[qslot]);
-        if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
-        if (tile < 0) break;
-        const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
-        const Problem& P = p.pr[ti.prob];
-        const int nk = tile_k_blocks(ti, P);
-        const uint32_t idesc = ptx::idesc_bf16_f32(W_ROWS, block_n<NT>(ti.rows - ti.m0));
-        if (!ptx::mbar_wait(&ss.tmem_empty, acc_phase ^ 1u, abort)) break;
-        ptx::tc_fence_after();
-        bool ok = true;
-        uint32_t accumulate = 0;
-        for (int kb = 0; kb < round_up(nk, MW); ++kb) {
-          const int cur = st;
-          const uint32_t cur_ph = sph;
-          if (++st == S) { st = 0; sph ^= 1u; }
-          if (kb % MW != m) continue;
-          if (!ptx::mbar_wait(&ss.a_full[cur], cur_ph, abort) ||
-              !ptx::mbar_wait(&ss.tok_full[cur], cur_ph, abort)) {
-            ok = false;
-            break;
-          }
-          if (kb < nk) {
-            ptx::tc_fence_after();
-            const uint32_t a_tmem = tmem_base + C::A_COL0 + cur * A_STAGE_COLS;
-            // descriptor start-address field counts 16-byte units: +2 per K step
-            const uint64_t b_desc =
-                ptx::smem_desc_sw128(ptx::smem_addr(tok_ring + cur * C::TOK_STAGE_BYTES));
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              ptx::mma_f16_ts(d_tmem, a_tmem + kk * 8, b_desc + 2 * kk, idesc, accumulate);
-              accumulate = 1;
-            }
-          }
-          ptx::mma_commit(&ss.stage_empty[cur]);   // token and weight stage free
+    int st = 0;
+    uint32_t sph = 0, acc_phase = 0;
+    const uint32_t d_tmem = tmem_base + m * NT;
+    int qslot = 0;
+    uint32_t qphase = 0;
+    for (;;) {
+      if (!__all_sync(kWarpMask, ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort))) break;
+      const int tile = __shfl_sync(kWarpMask, *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]), 0);
+      __threadfence_block();   // the slot is read before the warp hands it back
+      __syncwarp();
+      ptx::mbar_arrive_elect(&ss.tq_empty[qslot]);
+      if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+      if (tile < 0) break;
+      const TileInfo ti = decode_tile<NT>(tile, ss.tm, p, tiles0);
+      const Problem& P = p.pr[ti.prob];
+      const int nk = tile_k_blocks(ti, P);
+      const uint32_t idesc = ptx::idesc_bf16_f32(W_ROWS, block_n<NT>(ti.rows - ti.m0));
+      if (!__all_sync(kWarpMask, ptx::mbar_wait(&ss.tmem_empty, acc_phase ^ 1u, abort))) break;
+      ptx::tc_fence_after();
+      bool ok = true;
+      uint32_t accumulate = 0;
+      for (int kb = 0; kb < round_up(nk, MW); ++kb) {
+        const int cur = st;
+        const uint32_t cur_ph = sph;
+        if (++st == S) { st = 0; sph ^= 1u; }
+        if (kb % MW != m) continue;
+        const bool ready = ptx::mbar_wait(&ss.a_full[cur], cur_ph, abort) &&
+                           ptx::mbar_wait(&ss.tok_full[cur], cur_ph, abort);
+        if (!__all_sync(kWarpMask, ready)) {
+          ok = false;
+          break;
         }
-        if (!ok) break;
-        ptx::mma_commit(&ss.tmem_full);
-        acc_phase ^= 1u;
+        if (kb < nk) {
+          ptx::tc_fence_after();
+          const uint32_t a_tmem = tmem_base + C::A_COL0 + cur * A_STAGE_COLS;
+          // descriptor start-address field counts 16-byte units: +2 per K step
+          const uint64_t b_desc =
+              ptx::smem_desc_sw128(ptx::smem_addr(tok_ring + cur * C::TOK_STAGE_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            ptx::mma_f16_ts_elect(d_tmem, a_tmem + kk * 8, b_desc + 2 * kk, idesc, accumulate);
+            accumulate = 1;
+          }
+        }
+        ptx::mma_commit_elect(&ss.stage_empty[cur]);   // token and weight stage free
       }
-      ptx::mma_commit(&ss.drain[m]);
-      wait_drain(&ss.drain[m], 0, abort);
+      if (!ok) break;
+      ptx::mma_commit_elect(&ss.tmem_full);
+      acc_phase ^= 1u;
     }
+    __syncwarp();
+    ptx::mma_commit_elect(&ss.drain[m]);
+    wait_drain(&ss.drain[m], 0, abort);
   } else if (warp >= 2 && warp < 6) {
     // ---------------- epilogue (warps 2..5) ----------------
     const int q = warp & 3;

@@ -53,11 +53,13 @@
 //   warp 1      TMEM allocator (512 columns) and MMA issuer:
 //               tcgen05.mma.cta_group::1.kind::f16, M = 128, N, K = 16,
 //               fp32 accumulators in TMEM, two accumulator buffers so the
-//               epilogue of tile i overlaps the main loop of tile i+1.
-//   warp 6      second MMA issuer for N = 128: a thread issues one
-//               tcgen05.mma per ~100 cycles at best, longer than an N = 128
-//               MMA runs, so warps 1 and 6 take alternate K-blocks of a tile
-//               into two accumulators of its buffer (idle for N = 256).
+//               epilogue of tile i overlaps the main loop of tile i+1.  The
+//               whole warp walks the issue loop and an elected lane issues.
+//   warp 6      second MMA issuer for N = 128: one warp issues a tcgen05.mma
+//               per ~150 cycles (measured, whatever N), longer than an
+//               N = 128 MMA runs (64 cycles), so warps 1 and 6 take alternate
+//               K-blocks of a tile into two accumulators of its buffer (idle
+//               for N = 256).
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator(s) (warp w reads TMEM
 //               lanes 32*(w%4) .. +31), fused activation, global stores.
 #include <cuda_bf16.h>
@@ -320,62 +322,69 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     // ---------------- MMA issuers ----------------
     // Issuer m takes the K-blocks kb with kb % MW == m of every tile into
     // accumulator m of the tile's buffer; all issuers walk the same stages.
+    // The whole warp walks the loop, its waits decided by a warp vote, and an
+    // elected lane issues each tcgen05 operation (the operands stay
+    // warp-uniform, which issues the MMAs about a quarter faster than one lane
+    // looping alone).
     const int m = warp == 1 ? 0 : 1;
-    if (lane == 0) {
-      int astage = 0, bstage = 0;
-      uint32_t aphase = 0, bphase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      int qslot = 0;
-      uint32_t qphase = 0;
-      for (;;) {
-        if (!ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort)) break;
-        const int tile = *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]);
-        ptx::mbar_arrive_after_reads(&ss.tq_empty[qslot]);
-        if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
-        if (tile < 0) break;
-        const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
-        int kbeg, K;
-        tile_k_range(ti, p.pr[ti.prob], &kbeg, &K);
-        const int nk = (K + BK - 1) / BK;
-        if (!ptx::mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1u, abort)) break;
-        ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BUF_COLS + m * ACC_COLS;
-        bool ok = true;
-        uint32_t accumulate = 0;
-        for (int kb = 0; kb < round_up(nk, MW); ++kb) {
-          const int ca = astage, cb = bstage;
-          const uint32_t pa = aphase, pb = bphase;
-          if (++astage == A_STAGES) { astage = 0; aphase ^= 1u; }
-          if (++bstage == B_STAGES) { bstage = 0; bphase ^= 1u; }
-          if (kb % MW != m) continue;
-          if (!ptx::mbar_wait(&ss.a_full[ca], pa, abort) ||
-              !ptx::mbar_wait(&ss.b_full[cb], pb, abort)) {
-            ok = false;
-            break;
-          }
-          if (kb < nk) {
-            ptx::tc_fence_after();
-            // descriptor start-address fields count 16-byte units: +2 per K step
-            const uint64_t a_desc = ptx::smem_desc_sw128(ptx::smem_addr(ring_a + ca * A_BYTES));
-            const uint64_t b_desc = ptx::smem_desc_sw128(ptx::smem_addr(ring_b + cb * B_BYTES));
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              ptx::mma_f16_ss(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, IDESC, accumulate);
-              accumulate = 1;
-            }
-          }
-          // frees the weight stage, and the token stage to the producer's next
-          // lap, when these MMAs finish
-          ptx::mma_commit(&ss.b_empty[cb]);
+    int astage = 0, bstage = 0;
+    uint32_t aphase = 0, bphase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int qslot = 0;
+    uint32_t qphase = 0;
+    for (;;) {
+      if (!__all_sync(kWarpMask, ptx::mbar_wait(&ss.tq_full[qslot], qphase, abort))) break;
+      const int tile = __shfl_sync(kWarpMask, *reinterpret_cast<volatile int*>(&ss.tq_tile[qslot]), 0);
+      __threadfence_block();   // the slot is read before the warp hands it back
+      __syncwarp();
+      ptx::mbar_arrive_elect(&ss.tq_empty[qslot]);
+      if (++qslot == TILE_Q) { qslot = 0; qphase ^= 1u; }
+      if (tile < 0) break;
+      const TileInfo ti = decode_tile(tile, ss.tm, p, tiles0);
+      int kbeg, K;
+      tile_k_range(ti, p.pr[ti.prob], &kbeg, &K);
+      const int nk = (K + BK - 1) / BK;
+      if (!__all_sync(kWarpMask, ptx::mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1u, abort)))
+        break;
+      ptx::tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BUF_COLS + m * ACC_COLS;
+      bool ok = true;
+      uint32_t accumulate = 0;
+      for (int kb = 0; kb < round_up(nk, MW); ++kb) {
+        const int ca = astage, cb = bstage;
+        const uint32_t pa = aphase, pb = bphase;
+        if (++astage == A_STAGES) { astage = 0; aphase ^= 1u; }
+        if (++bstage == B_STAGES) { bstage = 0; bphase ^= 1u; }
+        if (kb % MW != m) continue;
+        const bool ready =
+            ptx::mbar_wait(&ss.a_full[ca], pa, abort) && ptx::mbar_wait(&ss.b_full[cb], pb, abort);
+        if (!__all_sync(kWarpMask, ready)) {
+          ok = false;
+          break;
         }
-        if (!ok) break;
-        ptx::mma_commit(&ss.tmem_full[acc]);   // accumulator ready for the epilogue
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (kb < nk) {
+          ptx::tc_fence_after();
+          // descriptor start-address fields count 16-byte units: +2 per K step
+          const uint64_t a_desc = ptx::smem_desc_sw128(ptx::smem_addr(ring_a + ca * A_BYTES));
+          const uint64_t b_desc = ptx::smem_desc_sw128(ptx::smem_addr(ring_b + cb * B_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            ptx::mma_f16_ss_elect(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, IDESC, accumulate);
+            accumulate = 1;
+          }
+        }
+        // frees the weight stage, and the token stage to the producer's next
+        // lap, when these MMAs finish
+        ptx::mma_commit_elect(&ss.b_empty[cb]);
       }
-      ptx::mma_commit(&ss.drain[m]);
-      wait_drain(&ss.drain[m], 0, abort);
+      if (!ok) break;
+      ptx::mma_commit_elect(&ss.tmem_full[acc]);   // accumulator ready for the epilogue
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    __syncwarp();
+    ptx::mma_commit_elect(&ss.drain[m]);
+    wait_drain(&ss.drain[m], 0, abort);
   } else if (warp >= 2 && warp < 6) {
     // ---------------- epilogue (warps 2..5) ----------------
     const int q = warp & 3;  // TMEM lane quarter this warp may access
