@@ -35,21 +35,22 @@
 //   warp 10     weight producer: TMA of FP8 weight tiles (64-byte swizzle) on
 //               a ring of its own (12 stages for NT = 128, 8 for NT = 256),
 //               running ahead of the tokens.
-//   warps 1,11  MMA issuers (warp 1 also allocates the 512 TMEM columns):
+//   warp 1      MMA issuer and TMEM allocator (512 columns):
 //               tcgen05.mma.cta_group::1.kind::f16, M = 128, N <= NT, K = 16.
 //               The weights are bf16 in the MMA, so a stage of 8 KB of codes
-//               costs as many MMAs as 16 KB of bf16 weights, and one warp
-//               issues a tcgen05.mma only every ~150 cycles whatever N: for
-//               NT = 128 two warps take alternate K-blocks into an accumulator
-//               each (the epilogue adds them); one commit per K-block frees
-//               both the token and the decoded-weight stage.  Each issuing
-//               warp walks its loop together and an elected lane issues.
+//               costs as many MMAs as 16 KB of bf16 weights.  The whole warp
+//               walks the issue loop and an elected lane issues (~150 cycles
+//               per MMA); one commit per K-block frees both the token and the
+//               decoded-weight stage.  (Warp 11 is a second issuer when
+//               Cfg::MMA_WARPS = 2: K-blocks alternate between two
+//               accumulators that the epilogue adds.)
 //   warps 2-5   epilogue (tcgen05.ld of the accumulators, SiLU gate or fp32
 //               store).
 //   warps 6-9,  decoders, two sets of four taking alternate stages: each
 //   12-15       warp reads its 32 weight rows of a stage (one row per thread,
 //               64 codes), decodes, and stores them to its TMEM lane quarter.
-// TMEM columns: accumulators first (two of 128 for NT = 128, one of 256 for
+// TMEM columns: accumulator buffers first (two of 128 for NT = 128, so the
+// epilogue of one tile overlaps the MMAs of the next; one of 256 for
 // NT = 256), then the decoded-weight stages (32 columns each).
 #include <cuda_bf16.h>
 
@@ -93,17 +94,23 @@ __device__ __forceinline__ int decoder_set(int warp) {
 //              their "empty" barrier, so one tcgen05.commit per K-block
 //              releases both.
 //   W8_STAGES  depth of the FP8 code ring (HBM latency is the longest).
-//   MMA_WARPS  a single thread issues a tcgen05.mma every ~100 cycles at best,
-//              far slower than an M = 128, N <= 128 MMA executes, so NT = 128
-//              blocks split each tile's K-blocks between two issuing warps with
-//              an accumulator each (K-block kb -> D_{kb mod 2}); the epilogue
-//              adds them.  NT = 256 MMAs are long enough for one.
+//   MMA_WARPS  issuing warps; with two, a tile's K-blocks alternate between
+//              two accumulators (K-block kb -> D_{kb mod 2}) that the epilogue
+//              adds.  One warp issuing with elect.sync is faster than two at
+//              decode (FFN 0.161 vs 0.165 ms) and leaves TMEM for a second
+//              accumulator buffer.
+//   ACC_BUFS   accumulator buffers: two where TMEM holds them next to the
+//              weight stages, so a tile's epilogue does not hold up the next
+//              tile's MMAs (decode down tiles run only 32 K-blocks).
 template <int NT>
 struct Cfg {
   static constexpr int TOK_STAGE_BYTES = NT * BK * 2;
-  static constexpr int MMA_WARPS = NT == 128 ? 2 : 1;
-  static constexpr uint32_t A_COL0 = MMA_WARPS * NT;      // weight stages follow the accumulators
+  static constexpr int MMA_WARPS = 1;
   static constexpr int STAGES = NT == 128 ? 6 : 4;
+  static constexpr int ACC_BUFS =
+      2 * MMA_WARPS * NT + STAGES * (int)A_STAGE_COLS <= (int)TMEM_COLS ? 2 : 1;
+  static constexpr uint32_t BUF_COLS = MMA_WARPS * NT;    // one accumulator buffer
+  static constexpr uint32_t A_COL0 = ACC_BUFS * BUF_COLS; // weight stages follow the accumulators
   static constexpr int W8_STAGES = NT == 128 ? 12 : 8;
   static_assert(STAGES <= MAX_STAGES && W8_STAGES <= MAX_W8_STAGES, "ring sizes");
   static_assert(MMA_WARPS <= MAX_MMA_WARPS, "one drain barrier per MMA issuer");
@@ -121,7 +128,7 @@ struct SharedState8 {
   uint64_t a_full[MAX_STAGES];        // decoded weights stored in TMEM (decoder threads)
   uint64_t stage_empty[MAX_STAGES];   // the K-block's MMAs completed (tcgen05.commit)
   uint64_t w8_full[MAX_W8_STAGES], w8_empty[MAX_W8_STAGES];
-  uint64_t tmem_full, tmem_empty;
+  uint64_t tmem_full[2], tmem_empty[2];   // per accumulator buffer
   uint64_t drain[MAX_MMA_WARPS];      // one per MMA issuer: its last MMAs completed
   uint64_t tq_full[TILE_Q], tq_empty[TILE_Q];   // claimed tiles, weight producer -> the rest
   int tq_tile[TILE_Q];
@@ -240,8 +247,10 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       ptx::mbar_init(&ss.w8_full[i], 1);
       ptx::mbar_init(&ss.w8_empty[i], DEC_THREADS);
     }
-    ptx::mbar_init(&ss.tmem_full, MW);
-    ptx::mbar_init(&ss.tmem_empty, EPI_WARPS);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&ss.tmem_full[i], MW);
+      ptx::mbar_init(&ss.tmem_empty[i], EPI_WARPS);
+    }
     for (int i = 0; i < MAX_MMA_WARPS; ++i) ptx::mbar_init(&ss.drain[i], 1);
     // readers of the tile queue: token producer, MMA issuers, 4 epilogue and
     // 8 decoder warps
@@ -393,7 +402,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     const int m = mma_index(warp);
     int st = 0;
     uint32_t sph = 0, acc_phase = 0;
-    const uint32_t d_tmem = tmem_base + m * NT;
+    int acc = 0;
     int qslot = 0;
     uint32_t qphase = 0;
     for (;;) {
@@ -408,8 +417,10 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       const Problem& P = p.pr[ti.prob];
       const int nk = tile_k_blocks(ti, P);
       const uint32_t idesc = ptx::idesc_bf16_f32(W_ROWS, block_n<NT>(ti.rows - ti.m0));
-      if (!__all_sync(kWarpMask, ptx::mbar_wait(&ss.tmem_empty, acc_phase ^ 1u, abort))) break;
+      if (!__all_sync(kWarpMask, ptx::mbar_wait(&ss.tmem_empty[acc], acc_phase ^ 1u, abort)))
+        break;
       ptx::tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * C::BUF_COLS + m * NT;
       bool ok = true;
       uint32_t accumulate = 0;
       for (int kb = 0; kb < round_up(nk, MW); ++kb) {
@@ -438,8 +449,8 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
         ptx::mma_commit_elect(&ss.stage_empty[cur]);   // token and weight stage free
       }
       if (!ok) break;
-      ptx::mma_commit_elect(&ss.tmem_full);
-      acc_phase ^= 1u;
+      ptx::mma_commit_elect(&ss.tmem_full[acc]);
+      if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
     }
     __syncwarp();
     ptx::mma_commit_elect(&ss.drain[m]);
@@ -448,6 +459,7 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
     // ---------------- epilogue (warps 2..5) ----------------
     const int q = warp & 3;
     uint32_t acc_phase = 0;
+    int acc = 0;
     int qslot = 0;
     uint32_t qphase = 0;
     for (;;) {
@@ -462,15 +474,16 @@ __global__ void __launch_bounds__(THREADS, 1) ffn_fp8_kernel(const __grid_consta
       const Problem& P = p.pr[ti.prob];
       const int n = block_n<NT>(ti.rows - ti.m0);
       const int nacc = min(MW, tile_k_blocks(ti, P));
-      if (!ptx::mbar_wait(&ss.tmem_full, acc_phase, abort)) break;
+      if (!ptx::mbar_wait(&ss.tmem_full[acc], acc_phase, abort)) break;
       ptx::tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::BUF_COLS;
       if (P.gateup) store_gateup(ti, P, taddr, NT, nacc, n, q, lane);
       else store_down(ti, P, taddr, NT, nacc, n, q, lane);
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&ss.tmem_empty);
-      acc_phase ^= 1u;
+      if (lane == 0) ptx::mbar_arrive(&ss.tmem_empty[acc]);
+      if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
       if (p.nprob > 1 && ti.prob == 0) release_rows(p, ti, lane);
     }
   } else if (decoder_set(warp) >= 0) {
