@@ -211,6 +211,22 @@ def test_forward_fp8_deterministic(moe):
     assert torch.equal(a.view(torch.int32), b.view(torch.int32)) and torch.equal(ia, ib)
 
 
+def test_forward_fp8_small_batch_many_tiles_per_cta(moe):
+    """128 tokens over 64 experts of D=2048, F=512: ~1500 tiles, about ten per
+    CTA, so every CTA cycles through both accumulator buffers of the 128-token
+    path many times.  Every token against the oracle, and a second call gives
+    the same bits."""
+    cfg = mi.custom_config("decode", T=128, D=2048, E=64, k=8, F=512, S=1, Fs=512,
+                           hidden_std=1.0, name="fp8_many_tiles")
+    inp = layer_on_device(cfg)
+    q = mi.fp8_layer_weights(inp)
+    a, ia, wa = _forward_fp8(moe, cfg, inp, q)
+    _check_layer_fp8(cfg, inp, q, a, ia, np.arange(cfg.T))
+    b, ib, wb = _forward_fp8(moe, cfg, inp, q)
+    assert torch.equal(ia, ib) and torch.equal(wa.view(torch.int32), wb.view(torch.int32))
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
 @pytest.fixture(scope="module")
 def glm52_fp8():
     cfg = mi.CONFIGS["decode"]
