@@ -72,7 +72,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int TPROD_WARP = 0;                    // token producer
 constexpr int MMA_WARP0 = 1;                     // MMA issuer (and TMEM allocator)
 constexpr int WPROD_WARP = 10;                   // weight producer
-constexpr int MMA_WARP1 = 11;                    // further MMA issuers (NT = 128)
+constexpr int MMA_WARP1 = 11;                    // second MMA issuer (Cfg::MMA_WARPS = 2)
 constexpr int MAX_MMA_WARPS = 2;
 constexpr int DEC_SETS = 2;                      // decoder sets: warps 6-9, 12-15
 constexpr int THREADS = 16 * 32;
@@ -604,7 +604,7 @@ int cdiv(int a, int b) { return (a + b - 1) / b; }
 }  // namespace
 
 // Batches of at most 128 tokens fit every group in one 128-token block (two
-// MMA issuers); larger batches use 256-token blocks.
+// accumulator buffers); larger batches use 256-token blocks.
 cudaError_t launch_expert_ffn_fp8(const FfnArgs& a, const Fp8Weights& w, cudaStream_t st,
                                   int* nlaunch, const char** why, void* const* marks) {
   const bool small = a.T <= 128;

@@ -88,9 +88,10 @@ struct Shape {
   // flight on them set the rate at which a decode batch reads its experts.
   static constexpr int B_STAGES = (RING_BYTES - A_STAGES * A_BYTES) / B_BYTES;
   static constexpr int ACC_COLS = MMA_N;                     // fp32 TMEM columns per accumulator
-  // One thread issues a tcgen05.mma every ~100 cycles at best, longer than an
-  // N = 128 MMA executes: N = 128 tiles split their K-blocks between two
-  // issuing warps with an accumulator each (the epilogue adds them).
+  // One issuing warp (elected lane) issues a tcgen05.mma every ~150 cycles,
+  // longer than an N = 128 MMA executes (64): N = 128 tiles split their
+  // K-blocks between two issuing warps (~105 cycles per MMA together) with an
+  // accumulator each (the epilogue adds them).
   static constexpr int MMA_WARPS = MMA_N == 128 ? 2 : 1;
   static constexpr int BUF_COLS = MMA_WARPS * ACC_COLS;      // one accumulator buffer
   static constexpr uint32_t TMEM_COLS = 2 * BUF_COLS;        // double buffered
