@@ -2,6 +2,7 @@
 layer and of the expert-FFN launch (the roofline numerators), FP8 weight
 bytes, whole-job throughput, and the traffic record keyed by kernel sources."""
 import json
+import subprocess
 import os
 import sys
 
@@ -106,3 +107,21 @@ def test_both_arms_name_the_workload_alike():
         w = bench.workload_name(mi.CONFIGS[name])
         assert w.startswith(name + ": ") and f"T={mi.CONFIGS[name].T} " in w
     assert "GLM-4.5-Air" in bench.workload_name(mi.CONFIGS["air"])
+
+
+def test_both_arms_print_the_same_config():
+    """The reference (oracle) arm, run as the driver runs it, prints the same
+    `config` object as `workload_config` gives our arm for that workload."""
+    cfg = mi.CONFIGS["tiny"]
+    ours = bench.workload_config(cfg, 1, False)
+    assert ours == {"workload": bench.workload_name(cfg), "T": cfg.T, "global_batch": cfg.T,
+                    "weights": "bf16"}
+    assert bench.workload_config(cfg, 4, False)["global_batch"] == 4 * cfg.T
+    assert bench.workload_config(cfg, 1, True)["weights"].startswith("fp8")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--config", "tiny", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == ours
