@@ -158,19 +158,6 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T: the A operand (M = 128 rows, one row per
-// TMEM lane, K = 16 bf16 packed two per 32-bit column, 8 columns) is read
-// from tensor memory at `a_tmem`.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Arrives once on `bar` when every tcgen05 operation this thread issued so far
 // has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -200,6 +187,9 @@ __device__ __forceinline__ void mma_f16_ss_elect(uint32_t d_tmem, uint64_t a_des
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, warp-collective: the A operand (M = 128
+// rows, one row per TMEM lane, K = 16 bf16 packed two per 32-bit column, 8
+// columns) is read from tensor memory at `a_tmem`.
 __device__ __forceinline__ void mma_f16_ts_elect(uint32_t d_tmem, uint32_t a_tmem,
                                                  uint64_t b_desc, uint32_t idesc,
                                                  uint32_t accumulate) {
